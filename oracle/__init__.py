@@ -1,0 +1,17 @@
+"""CPU oracle (test infrastructure only; see llm_int8.py)."""
+from .llm_int8 import (  # noqa: F401
+    QMAX_INT8,
+    absmax_codes,
+    quantize_per_tensor,
+    step_size,
+    dequantize_codes,
+    quantize_weight_rows,
+    find_outlier_cols,
+    quantize_act_rows,
+    int32_gemm,
+    int32_dot,
+    dequantize,
+    outlier_gemm,
+    llm_int8_matmul,
+    llm_int8_matmul_at,
+)

@@ -1,0 +1,46 @@
+"""Planted mistakes in a copy of the oracle must each fail a pin.
+
+Each mutant rewrites one line of a temporary copy of oracle/llm_int8.py
+(a dropped term, a wrong comparison, a wrong rounding mode, a transposed
+or reversed operand, a wrong sign) and runs tests/test_oracle_pins.py
+against it in a subprocess. Nothing here touches a GPU.
+"""
+import os
+import shutil
+import subprocess
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+MUTANTS = {
+    "dequant_over_127_not_127sq": ("/ float(QMAX_INT8 * QMAX_INT8))\n\n\n#", "/ float(QMAX_INT8))\n\n\n#"),
+    "detect_ge_not_gt": ("np.abs(X32) > thr", "np.abs(X32) >= thr"),
+    "round_half_up": ("q = np.rint(quot)", "q = np.floor(quot + 0.5)"),
+    "gemm_reversed_k": ("C = A @ B.T", "C = A @ B[:, ::-1].T"),
+    "act_absmax_over_all_cols": ("normal = np.where(keep[None, :], np.abs(X32), np.float32(0))",
+                                 "normal = np.abs(X32)"),
+    "outlier_sign_flipped": ("return np.asarray(X, np.float64)[:, idx] @",
+                             "return -np.asarray(X, np.float64)[:, idx] @"),
+    "outlier_term_dropped": ("Y = (Cn + Co).astype(np.float16)", "Y = (Cn).astype(np.float16)"),
+    "w_scale_index_reversed": ("* np.asarray(w_scale, np.float64)[None, :] /",
+                               "* np.asarray(w_scale, np.float64)[::-1][None, :] /"),
+    "weight_absmax_per_tensor": ("aw = np.max(np.abs(W32), axis=1)",
+                                 "aw = np.max(np.abs(W32), axis=1) * 0 + np.max(np.abs(W32))"),
+}
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_pins_catch_planted_mistake(name, tmp_path):
+    src = open(os.path.join(ROOT, "oracle", "llm_int8.py")).read()
+    old, new = MUTANTS[name]
+    assert old in src, f"mutation site for {name} no longer exists"
+    for d in ("oracle", "synth", "tests"):
+        shutil.copytree(os.path.join(ROOT, d), tmp_path / d,
+                        ignore=shutil.ignore_patterns("__pycache__", "test_oracle_mutants.py"))
+    (tmp_path / "oracle" / "llm_int8.py").write_text(src.replace(old, new, 1))
+    r = subprocess.run([sys.executable, "-m", "pytest", "-q", "-x", "-p", "no:cacheprovider",
+                        "tests/test_oracle_pins.py"], cwd=tmp_path, capture_output=True, text=True,
+                       timeout=300)
+    assert r.returncode != 0, f"mutant {name} survived the pins:\n{r.stdout[-2000:]}"
