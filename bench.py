@@ -1,0 +1,457 @@
+"""Benchmark of the LLM.int8() mixed-precision matmul on B200.
+
+One step = one int8_mixed_matmul call (outlier detection, per-token INT8
+quantisation with outlier compaction, tcgen05 INT8 GEMM + fp16 outlier GEMM
++ dequantising epilogue) over one batch of synthetic activations, with the
+weight already quantised (int8_quantize_weight_rows runs once, untimed, as
+a deployed layer would).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+Multi-GPU (torchrun, one rank per GPU): the op does not shard across ranks
+here, so every rank runs an independent replica of the same workload; the
+timed region is bracketed by barriers, the time is the max over ranks and
+`value` counts the work of all ranks ("scaling": "weak").
+
+Prints one JSON line (rank 0).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+METRIC = "int8_mixed_matmul TOPS & % of B200 INT8 peak; decode-shape HBM GB/s"
+DEFAULT_WORKLOAD = "opt-6.7b-ffn-up-prefill"
+DECODE_WORKLOAD = "decode"
+# Fallback denominators when MEASURED_PEAKS.json is absent (earlier pool measurement).
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+# Dense INT8 : dense BF16 tensor throughput on B200 (4.5 : 2.25 PFLOP/s nominal).
+INT8_OVER_BF16 = 2.0
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+# --------------------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi sampling of SM clock and throttle reasons during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            import tempfile
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.out = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-i", str(self.gpu), "-lms", "100"], stdout=self.out, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.out.close()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        smax = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "reasons": reasons, "samples": len(rows),
+                "power_w_max": max(float(r[3]) for r in rows if r[3].replace(".", "").isdigit())
+                if any(r[3].replace(".", "").isdigit() for r in rows) else None}
+
+
+# --------------------------------------------------------------------------- oracle timing
+def oracle_sample_step(X, W, Wq, w_scale, threshold, rows):
+    """The CPU oracle on a `rows`-token batch of the workload (detection over that batch)."""
+    import oracle
+    Xs = X[:rows]
+    return oracle.llm_int8_matmul(Xs, W, threshold, Wq=Wq, w_scale=w_scale)
+
+
+def oracle_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        info = threadpool_info()
+        return max((i.get("num_threads", 1) for i in info), default=1)
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def time_oracle(w, X, W, Wq, w_scale, budget_s: float, max_rows: int | None = None):
+    """Times the oracle on a bounded row sample; returns (TOPS, rows, seconds per step)."""
+    rows = min(w.M, 16)
+    t0 = time.perf_counter()
+    oracle_sample_step(X, W, Wq, w_scale, w.threshold, rows)
+    t = time.perf_counter() - t0
+    target = max(1, int(rows * budget_s / max(t, 1e-6)))
+    rows = min(w.M, target if max_rows is None else min(target, max_rows))
+    t0 = time.perf_counter()
+    oracle_sample_step(X, W, Wq, w_scale, w.threshold, rows)
+    t = time.perf_counter() - t0
+    return 2.0 * rows * w.N * w.K / t / 1e12, rows, t
+
+
+# --------------------------------------------------------------------------- distributed
+def dist_setup(n_gpus: int):
+    import torch
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if ws > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(0)
+    return ws, rank, local
+
+
+def barrier(ws):
+    if ws > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x: float, ws: int) -> float:
+    if ws == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# --------------------------------------------------------------------------- our arm
+class Problem:
+    """Device buffers for one workload, replicated into rotating sets."""
+
+    def __init__(self, w, X, W, n_sets):
+        import torch
+        import w8a8_quantized_matmul_b200 as m
+        self.w = w
+        Xd = torch.from_numpy(X).cuda()
+        Wd = torch.from_numpy(W).cuda()
+        Wq, ws = m.int8_quantize_weight_rows(Wd)       # offline, untimed
+        need = m.int8_mixed_matmul_workspace_size(w.M, w.N, w.K)
+        self.sets = []
+        for i in range(n_sets):
+            s = dict(X=Xd if i == 0 else Xd.clone(), Wq=Wq if i == 0 else Wq.clone(),
+                     ws=ws if i == 0 else ws.clone(), W=Wd if i == 0 else Wd.clone(),
+                     Y=torch.empty((w.M, w.N), dtype=torch.float16, device="cuda"),
+                     work=torch.empty((need,), dtype=torch.uint8, device="cuda"))
+            self.sets.append(s)
+        torch.cuda.synchronize()
+
+    def step(self, i, events=None):
+        import w8a8_quantized_matmul_b200 as m
+        s = self.sets[i % len(self.sets)]
+        if events is None:
+            m.int8_mixed_matmul(s["X"], s["Wq"], s["ws"], s["W"], self.w.threshold, Y=s["Y"],
+                                workspace=s["work"])
+        else:
+            m.int8_mixed_matmul_profiled(s["X"], s["Wq"], s["ws"], s["W"], self.w.threshold,
+                                         s["Y"], s["work"], events)
+
+    def bytes_touched(self):
+        w = self.w
+        return 2 * w.M * w.K + w.M * w.K + w.N * w.K + 2 * w.M * w.N
+
+
+def n_sets_for(w, l2_bytes):
+    per = 2 * w.M * w.K + w.M * w.K + w.N * w.K + 2 * w.M * w.N
+    return int(min(32, max(2, math.ceil(2 * l2_bytes / per) + 1)))
+
+
+def quantize_stage_bytes(w, count):
+    """Algorithmic bytes of detection + quantisation + compaction per call."""
+    pad = (count + 63) // 64 * 64
+    return (2 * w.M * w.K            # read X (once from HBM; detection and quantisation)
+            + w.M * w.K + 4 * w.M    # write Xq, x_scale
+            + 2 * w.M * pad          # write X_O
+            + 32 * w.N * count       # W_O gather: one 32-byte sector per outlier per row
+            + 2 * w.N * pad)         # write W_O
+
+
+def run_ours(args, ws, rank, local):
+    import torch
+    import w8a8_quantized_matmul_b200 as m
+    from w8a8_quantized_matmul_b200 import build as _b
+    if rank == 0:
+        _b.build()
+    barrier(ws)
+    m.load()
+    peaks, peaks_kind = load_peaks()
+    props = torch.cuda.get_device_properties(torch.cuda.current_device())
+    l2 = getattr(props, "L2_cache_size", 126 * 2 ** 20) or 126 * 2 ** 20
+
+    w = synth.WORKLOADS[args.workload]
+    X, W, planted = synth.make_workload(w)
+    n_sets = n_sets_for(w, l2)
+    prob = Problem(w, X, W, n_sets)
+
+    stream = torch.cuda.current_stream()
+    for i in range(args.warmup):
+        prob.step(i)
+    torch.cuda.synchronize()
+    views = m.workspace_views(prob.sets[0]["work"], w.M, w.N, w.K)
+    count = int(views["n_outliers"].item())
+
+    # ---- timed region: K steps, barrier + sync on both sides, per-stage events
+    n_ev = args.steps
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(n_ev)]
+    for e in evs:                      # create the underlying events before timing
+        for x in e:
+            x.record(stream)
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    barrier(ws)
+    torch.cuda.synchronize()
+    start.record(stream)
+    for i in range(args.steps):
+        prob.step(i, evs[i])
+    end.record(stream)
+    torch.cuda.synchronize()
+    barrier(ws)
+    clk = clocks.stop()
+    ms = start.elapsed_time(end)
+    ms_max = max_over_ranks(ms, ws)
+    q_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
+    g_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
+
+    ops_per_step = 2.0 * w.M * w.N * w.K
+    value = ops_per_step * args.steps * ws / (ms_max / 1e3) / 1e12
+    bf16 = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+    int8_peak = bf16 * INT8_OVER_BF16
+    hbm = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
+    gemm_tops = ops_per_step / (g_ms / 1e3) / 1e12
+    qbytes = quantize_stage_bytes(w, count)
+    q_gbs = qbytes / (q_ms / 1e3) / 1e9
+
+    # ---- end to end through the public API with host buffers
+    e2e_steps = min(args.steps, 200)
+    Xh = torch.from_numpy(X).pin_memory()
+    Yh = torch.empty((w.M, w.N), dtype=torch.float16).pin_memory()
+    s0 = prob.sets[0]
+    for _ in range(2):
+        s0["X"].copy_(Xh, non_blocking=True)
+        prob.step(0)
+        Yh.copy_(s0["Y"], non_blocking=True)
+    torch.cuda.synchronize()
+    barrier(ws)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(e2e_steps):
+        s0["X"].copy_(Xh, non_blocking=True)
+        prob.step(0)
+        Yh.copy_(s0["Y"], non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), ws)
+    e2e_value = ops_per_step * e2e_steps * ws / (e2e_ms / 1e3) / 1e12
+
+    # ---- decode-shape line (weight-read bound), same process, rank-local
+    decode = None
+    if args.workload != DECODE_WORKLOAD and not args.no_decode:
+        decode = bench_decode(args, stream, l2, hbm)
+
+    result = {
+        "metric": METRIC,
+        "value": round(value, 3),
+        "unit": "TOPS",
+        "n_gpus": ws,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": ms_max / args.steps,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "int8",
+        "data": "synthetic",
+        "config": {"workload": w.name, "M": w.M, "K": w.K, "N": w.N, "threshold": w.threshold,
+                   "planted_outliers": int(len(planted)), "detected_outliers": count,
+                   "parallelism": f"replicas x{ws}",
+                   "l2": f"rotating {n_sets} buffer sets of {prob.bytes_touched() / 1e6:.0f} MB "
+                         f"touched per step (> 2x L2 of {l2 / 1e6:.0f} MB)"},
+        "roofline": {"kernel": "gemm_i8_mixed_kernel (tcgen05 kind::i8 + kind::f16)",
+                     "bound": "tensor", "achieved": round(gemm_tops, 2),
+                     "peak": round(int8_peak, 1), "unit": "TOPS",
+                     "frac": round(gemm_tops / int8_peak, 4), "traffic": None,
+                     "peak_note": f"{peaks_kind} bf16 burst {bf16} TFLOP/s x {INT8_OVER_BF16} "
+                                  "(dense int8 : bf16 nominal ratio)",
+                     "gemm_ms": g_ms},
+        "roofline_quantize": {"kernel": "detect_outliers_kernel + quantize_rows_kernel<.., true>",
+                              "bound": "hbm", "achieved": round(q_gbs, 1), "peak": hbm,
+                              "unit": "GB/s", "frac": round(q_gbs / hbm, 4),
+                              "algorithmic_bytes": qbytes, "stage_ms": q_ms,
+                              "peak_note": f"{peaks_kind} hbm_gbs"},
+        "e2e": {"value": round(e2e_value, 3), "unit": "TOPS", "steps": e2e_steps,
+                "h2d_bytes_per_step": 2 * w.M * w.K, "d2h_bytes_per_step": 2 * w.M * w.N},
+        "gpu_launches": 3 * args.steps,
+        "gpu_launches_note": "per step: detect, quantize+compact, GEMM kernels (plus one "
+                             "cudaMemsetAsync of the bitmap)",
+        "clocks": clk,
+    }
+    if decode is not None:
+        result["decode"] = decode
+    if rank == 0 and not args.no_cpu_baseline:
+        import oracle
+        Wq_o, ws_o = oracle.quantize_weight_rows(W)
+        tops, rows, t = time_oracle(w, X, W, Wq_o, ws_o, budget_s=args.cpu_budget)
+        result["cpu_baseline"] = {"value": round(tops, 6), "unit": "TOPS",
+                                  "cores": oracle_threads(), "kind": "oracle",
+                                  "sample": f"{rows} of {w.M} tokens of the same workload "
+                                            f"(detection over those tokens), {t:.1f} s"}
+    return result
+
+
+def bench_decode(args, stream, l2, hbm):
+    """Decode shape (16 tokens): HBM GB/s of one int8_mixed_matmul call."""
+    import torch
+    w = synth.WORKLOADS[DECODE_WORKLOAD]
+    X, W, _ = synth.make_workload(w)
+    n_sets = n_sets_for(w, l2)
+    prob = Problem(w, X, W, n_sets)
+    for i in range(max(3, args.warmup)):
+        prob.step(i)
+    steps = max(50, min(args.steps, 2000))
+    s = torch.cuda.Event(enable_timing=True)
+    e = torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    s.record(stream)
+    for i in range(steps):
+        prob.step(i)
+    e.record(stream)
+    torch.cuda.synchronize()
+    ms = s.elapsed_time(e) / steps
+    # Algorithmic bytes: read Wq, w_scale, X; write Y (the outlier columns of W are tiny).
+    nbytes = w.N * w.K + 4 * w.N + 2 * w.M * w.K + 2 * w.M * w.N
+    gbs = nbytes / (ms / 1e3) / 1e9
+    return {"workload": w.name, "M": w.M, "K": w.K, "N": w.N, "us_per_call": round(ms * 1e3, 2),
+            "value": round(gbs, 1), "unit": "GB/s", "frac_of_hbm": round(gbs / hbm, 4),
+            "algorithmic_bytes": nbytes, "rotating_sets": n_sets, "steps": steps}
+
+
+# --------------------------------------------------------------------------- reference arm
+def run_reference(args, ws, rank):
+    """The CPU oracle as the reference arm, on bounded samples of the same workload."""
+    import oracle
+    w = synth.WORKLOADS[args.workload]
+    X, W, _ = synth.make_workload(w)
+    Wq, w_scale = oracle.quantize_weight_rows(W)
+    total = args.steps + args.warmup
+    per_step_budget = max(0.02, 120.0 / max(total, 1))
+    rows = min(w.M, 16)
+    t0 = time.perf_counter()
+    oracle_sample_step(X, W, Wq, w_scale, w.threshold, rows)
+    t1 = time.perf_counter() - t0
+    rows = max(1, min(w.M, int(rows * per_step_budget / max(t1, 1e-6))))
+    for _ in range(args.warmup):
+        oracle_sample_step(X, W, Wq, w_scale, w.threshold, rows)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle_sample_step(X, W, Wq, w_scale, w.threshold, rows)
+    t = time.perf_counter() - t0
+    tops = 2.0 * rows * w.N * w.K * args.steps / t / 1e12
+    cores = oracle_threads()
+    sample = f"{rows} of {w.M} tokens per step (detection over those tokens)"
+    return {
+        "impl": "reference", "metric": METRIC, "value": round(tops, 6), "unit": "TOPS",
+        "n_gpus": ws, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": t / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "int8", "data": "synthetic",
+        "config": {"workload": w.name, "M": w.M, "K": w.K, "N": w.N, "threshold": w.threshold},
+        "cpu_baseline": {"value": round(tops, 6), "unit": "TOPS", "cores": cores,
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": round(tops, 6), "unit": "TOPS", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(synth.WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--cpu-budget", type=float, default=15.0,
+                    help="seconds of oracle work for the cpu_baseline sample")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-decode", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    if args.impl == "reference":
+        ws = int(os.environ.get("WORLD_SIZE", "1"))
+        rank = int(os.environ.get("RANK", "0"))
+        if rank != 0:
+            return
+        print(json.dumps(run_reference(args, ws, rank)), flush=True)
+        return
+
+    ws, rank, local = dist_setup(args.gpus)
+    try:
+        res = run_ours(args, ws, rank, local)
+        if rank == 0:
+            print(json.dumps(res), flush=True)
+    finally:
+        if ws > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,183 @@
+/*
+ * int8mm.h - C ABI of libint8mm, the B200 (sm_100a) LLM.int8() mixed-precision
+ * decomposition matmul  Y = X . W^T.
+ *
+ * Method (AIInfra "05Infer/06CompDistill/05Quantization01", LLM.int8() section;
+ * tanjunchen "quantization explained part 2", section 1.2):
+ *   1. outlier feature columns O of the FP16 activations: any |x| > threshold;
+ *   2. per-token (row) absmax INT8 quantisation of the non-outlier columns,
+ *      per-output-row absmax INT8 quantisation of W (done once, offline);
+ *   3. INT8 x INT8 -> INT32 matrix product;
+ *   4. dequantisation by the outer product of the row and column absmax / 127^2;
+ *   5. FP16 product over the outlier columns, added into the result.
+ *
+ * Conventions for every entry point:
+ *   - All array pointers are DEVICE pointers, allocated and owned by the
+ *     caller. The library never allocates or frees device memory.
+ *   - Matrices are row-major and dense (row stride = number of columns):
+ *     X [M][K] fp16, W [N][K] fp16 (out-features x in-features), Wq [N][K]
+ *     int8, Y [M][N] fp16. fp16 is IEEE binary16, passed as `const void*`.
+ *   - Every call is asynchronous on `stream` (a cudaStream_t; NULL = the
+ *     legacy default stream) and does no host synchronisation. Device-side
+ *     results such as the outlier count stay on the device.
+ *   - Argument errors are detected on the host BEFORE anything is launched
+ *     and returned as a negative i8mm_status; nothing is written then.
+ *     No exception or abort crosses the ABI.
+ *   - Requirements: K a positive multiple of 16 and <= 65536; M, N <= 2^22;
+ *     every pointer 16-byte aligned; threshold not NaN and >= 0 (+inf
+ *     allowed). M == 0 or N == 0 is a valid empty problem and returns
+ *     I8MM_OK without launching (int8_find_outlier_cols with M == 0 still
+ *     writes a count of 0).
+ *   - X is assumed finite; NaN/Inf activations are outside the contract.
+ *   - Codes are clamp(rint((x*127)/absmax), -127, 127) with one fp32
+ *     product and one correctly rounded fp32 division, rint = round half to
+ *     even; a group whose absmax is 0 gets scale 0 and all-zero codes.
+ *   - Scales are stored as the absmax itself (fp32); dequantisation
+ *     multiplies by x_scale[i] * w_scale[n] / 127^2.
+ */
+#ifndef INT8MM_H_
+#define INT8MM_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same object as cudaStream_t; declared here so the header needs no CUDA include. */
+typedef struct CUstream_st* i8mm_stream_t;
+
+typedef enum {
+  I8MM_OK = 0,
+  I8MM_ERR_INVALID_ARG = -1,        /* null pointer, bad size, NaN/negative threshold */
+  I8MM_ERR_ALIGNMENT = -2,          /* a pointer is not 16-byte aligned, or K % 16 != 0 */
+  I8MM_ERR_WORKSPACE = -3,          /* workspace null or smaller than the required size */
+  I8MM_ERR_CUDA = -4,               /* a CUDA runtime/driver call or launch failed */
+  I8MM_ERR_TIMEOUT = -5,            /* a bounded device-side wait gave up (see int8_device_status) */
+  I8MM_ERR_UNSUPPORTED_DEVICE = -6  /* the current device is not sm_100 (B200) */
+} i8mm_status;
+
+/*
+ * Offline weight quantisation (AIInfra LLM.int8() section, "vector-wise
+ * quantisation": one scale per weight column of the h x o matrix, i.e. per
+ * output row of the [N][K] layout used here).
+ *   W        in : fp16 [N][K]
+ *   Wq       out: int8 [N][K], codes over the whole row
+ *   w_scale  out: fp32 [N], absmax of each row over all K columns
+ * Off the per-call hot path: a deployed layer quantises its weight once.
+ */
+int int8_quantize_weight_rows(const void* W, int N, int K, int8_t* Wq, float* w_scale,
+                              i8mm_stream_t stream);
+
+/*
+ * Outlier feature-column detection (AIInfra LLM.int8() section, "detection:
+ * set a magnitude threshold"; tanjunchen section 1.2: a channel whose
+ * activation magnitude exceeds the threshold, 6.0 by default).
+ * Column j is an outlier iff |float(X[i][j])| > threshold for some row i
+ * of this X (strict comparison in fp32).
+ *   X           in : fp16 [M][K]
+ *   col_bitmap  out: uint32 [ceil(K/32)], bit (j%32) of word (j/32) set for outliers
+ *   n_outliers  out: int32 [1] on the device, the number of outlier columns
+ *   col_idx     out: int32 [K], outlier column indices in ascending order in the
+ *                    first n_outliers entries (the rest is unspecified); may be NULL
+ */
+int int8_find_outlier_cols(const void* X, int M, int K, float threshold,
+                           uint32_t* col_bitmap, int32_t* n_outliers, int32_t* col_idx,
+                           i8mm_stream_t stream);
+
+/*
+ * Per-token absmax INT8 quantisation of the non-outlier part (AIInfra
+ * LLM.int8() section, vector-wise quantisation of each row of X after the
+ * outliers are separated; tanjunchen section 1.2, the 4096-dim example).
+ *   X          in : fp16 [M][K]
+ *   col_bitmap in : uint32 [ceil(K/32)] as produced by int8_find_outlier_cols
+ *   Xq         out: int8 [M][K], 0 at outlier columns
+ *   x_scale    out: fp32 [M], absmax of each row over the non-outlier columns
+ */
+int int8_quantize_act_rows(const void* X, int M, int K, const uint32_t* col_bitmap,
+                           int8_t* Xq, float* x_scale, i8mm_stream_t stream);
+
+/* Bytes of device workspace int8_mixed_matmul needs for these sizes (0 on bad sizes). */
+size_t int8_mixed_matmul_workspace_size(int M, int N, int K);
+
+/*
+ * Where int8_mixed_matmul leaves its intermediates inside the workspace
+ * (byte offsets from the workspace base; each at least 16-byte aligned). Lets a
+ * caller or a test read the outlier set, codes and scales of the last call.
+ * The outlier panels have row stride panel_ld elements (fp16) and hold the
+ * compacted outlier columns, zero-padded to a multiple of 64.
+ */
+typedef struct {
+  size_t n_outliers;   /* int32 [1] */
+  size_t status;       /* int32 [1], device status word (0 = ok) */
+  size_t col_bitmap;   /* uint32 [ceil(K/32)] */
+  size_t col_idx;      /* int32 [K] */
+  size_t x_scale;      /* fp32 [M] */
+  size_t Xq;           /* int8 [M][K] */
+  size_t X_O;          /* fp16 [M][panel_ld] */
+  size_t W_O;          /* fp16 [N][panel_ld] */
+  size_t total;        /* == int8_mixed_matmul_workspace_size(M, N, K) */
+  int panel_ld;        /* = K rounded up to a multiple of 64 */
+} i8mm_workspace_layout;
+
+int int8_mixed_matmul_workspace_layout(int M, int N, int K, i8mm_workspace_layout* out);
+
+/*
+ * The whole decomposition (AIInfra LLM.int8() section: C_i32 = X_i8 x W_i8,
+ * C_normal = C_i32 / (c_x (x) c_w), C_outlier = sum_{h in O} X_f16^h W_f16^h,
+ * C_f16 = C_outlier + C_normal).
+ *   X          in : fp16 [M][K] activations
+ *   Wq,w_scale in : from int8_quantize_weight_rows
+ *   W_fp16     in : fp16 [N][K], the unquantised weight; only its outlier
+ *                   columns are read
+ *   threshold  in : outlier magnitude threshold (6.0 in the pages)
+ *   Y          out: fp16 [M][N], Y = fp16(C_i32*x_scale*w_scale/127^2 + C_outlier),
+ *                   the sum formed in fp32 and rounded once
+ *   workspace  in : device scratch of at least int8_mixed_matmul_workspace_size(M,N,K)
+ *                   bytes, 256-byte aligned; contents on entry are ignored
+ * One call launches the detection, quantisation/compaction and GEMM kernels
+ * back to back on `stream`; the outlier count never leaves the device.
+ */
+int int8_mixed_matmul(const void* X, const int8_t* Wq, const float* w_scale,
+                      const void* W_fp16, int M, int N, int K, float threshold, void* Y,
+                      void* workspace, size_t workspace_bytes, i8mm_stream_t stream);
+
+/*
+ * Measurement hook: exactly int8_mixed_matmul, and in addition records three
+ * CUDA events (cudaEvent_t, created by the caller) on `stream`:
+ *   events[0] before the first operation of the call,
+ *   events[1] after the detection and quantisation/compaction kernels,
+ *   events[2] after the GEMM kernel.
+ * The elapsed times events[0]->events[1] and events[1]->events[2] are the
+ * device durations of the memory-bound stage and of the tensor-core GEMM.
+ */
+int int8_mixed_matmul_profiled(const void* X, const int8_t* Wq, const float* w_scale,
+                               const void* W_fp16, int M, int N, int K, float threshold,
+                               void* Y, void* workspace, size_t workspace_bytes,
+                               i8mm_stream_t stream, void* const* events);
+
+/*
+ * Test hook: the INT8 x INT8 -> INT32 product alone (AIInfra LLM.int8()
+ * section, "C_i32 = X_i8 x W_i8", accumulated in INT32), on the same
+ * tensor-core kernel the full path uses.
+ *   C out: int32 [M][N], C[i][n] = sum_k Xq[i][k] * Wq[n][k]
+ */
+int int8_debug_gemm_i32(const int8_t* Xq, const int8_t* Wq, int M, int N, int K, int32_t* C,
+                        i8mm_stream_t stream);
+
+/*
+ * Reads the device status word a previous int8_mixed_matmul left in its
+ * workspace (synchronises `stream`). Returns I8MM_OK, I8MM_ERR_TIMEOUT if
+ * a bounded device-side wait gave up, or I8MM_ERR_CUDA.
+ */
+int int8_device_status(const void* workspace, i8mm_stream_t stream);
+
+/* Static string for a status code. */
+const char* int8_status_string(int status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* INT8MM_H_ */

@@ -1,0 +1,200 @@
+"""LLM.int8() mixed-precision decomposition matmul for B200 (sm_100a).
+
+Thin Python binding over the C ABI of libint8mm (include/int8mm.h). Each
+function has the name of the C entry point it calls; PyTorch supplies only
+device memory and the current CUDA stream, and every step of the path runs
+in the library's CUDA kernels. There is no CPU fallback: calling any compute
+entry point without the built library or without a B200 raises.
+"""
+from __future__ import annotations
+
+import ctypes
+
+import torch
+
+from ._lib import (  # noqa: F401
+    I8MM_ERR_ALIGNMENT,
+    I8MM_ERR_CUDA,
+    I8MM_ERR_INVALID_ARG,
+    I8MM_ERR_TIMEOUT,
+    I8MM_ERR_UNSUPPORTED_DEVICE,
+    I8MM_ERR_WORKSPACE,
+    I8MM_OK,
+    Int8mmError,
+    WorkspaceLayout,
+    check,
+    load,
+    status_string,
+)
+
+__all__ = [
+    "int8_quantize_weight_rows",
+    "int8_find_outlier_cols",
+    "int8_quantize_act_rows",
+    "int8_mixed_matmul_workspace_size",
+    "int8_mixed_matmul_workspace_layout",
+    "int8_mixed_matmul",
+    "int8_mixed_matmul_profiled",
+    "int8_debug_gemm_i32",
+    "int8_device_status",
+    "Int8mmError",
+]
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _ptr(t: torch.Tensor | None) -> ctypes.c_void_p:
+    return ctypes.c_void_p(0 if t is None else t.data_ptr())
+
+
+def _need(t: torch.Tensor, name: str, dtype: torch.dtype, shape: tuple) -> None:
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def int8_quantize_weight_rows(W, Wq=None, w_scale=None, stream=None):
+    """W fp16 [N, K] -> (Wq int8 [N, K], w_scale fp32 [N] row absmax)."""
+    N, K = W.shape
+    _need(W, "W", torch.float16, (N, K))
+    Wq = torch.empty((N, K), dtype=torch.int8, device=W.device) if Wq is None else Wq
+    w_scale = torch.empty((N,), dtype=torch.float32, device=W.device) if w_scale is None else w_scale
+    _need(Wq, "Wq", torch.int8, (N, K))
+    _need(w_scale, "w_scale", torch.float32, (N,))
+    check("int8_quantize_weight_rows",
+          load().int8_quantize_weight_rows(_ptr(W), N, K, _ptr(Wq), _ptr(w_scale), _stream(stream)))
+    return Wq, w_scale
+
+
+def int8_find_outlier_cols(X, threshold=6.0, col_bitmap=None, n_outliers=None, col_idx=None,
+                           stream=None):
+    """X fp16 [M, K] -> (bitmap uint32-as-int32 [ceil(K/32)], count int32 [1], col_idx int32 [K])."""
+    M, K = X.shape
+    _need(X, "X", torch.float16, (M, K))
+    words = (K + 31) // 32
+    dev = X.device
+    col_bitmap = torch.empty((words,), dtype=torch.int32, device=dev) if col_bitmap is None else col_bitmap
+    n_outliers = torch.empty((4,), dtype=torch.int32, device=dev)[:1] if n_outliers is None else n_outliers
+    col_idx = torch.empty((K,), dtype=torch.int32, device=dev) if col_idx is None else col_idx
+    _need(col_bitmap, "col_bitmap", torch.int32, (words,))
+    _need(col_idx, "col_idx", torch.int32, (K,))
+    check("int8_find_outlier_cols",
+          load().int8_find_outlier_cols(_ptr(X), M, K, float(threshold), _ptr(col_bitmap),
+                                        _ptr(n_outliers), _ptr(col_idx), _stream(stream)))
+    return col_bitmap, n_outliers, col_idx
+
+
+def int8_quantize_act_rows(X, col_bitmap, Xq=None, x_scale=None, stream=None):
+    """X fp16 [M, K] + outlier bitmap -> (Xq int8 [M, K], x_scale fp32 [M])."""
+    M, K = X.shape
+    _need(X, "X", torch.float16, (M, K))
+    _need(col_bitmap, "col_bitmap", torch.int32, ((K + 31) // 32,))
+    Xq = torch.empty((M, K), dtype=torch.int8, device=X.device) if Xq is None else Xq
+    x_scale = torch.empty((M,), dtype=torch.float32, device=X.device) if x_scale is None else x_scale
+    _need(Xq, "Xq", torch.int8, (M, K))
+    _need(x_scale, "x_scale", torch.float32, (M,))
+    check("int8_quantize_act_rows",
+          load().int8_quantize_act_rows(_ptr(X), M, K, _ptr(col_bitmap), _ptr(Xq), _ptr(x_scale),
+                                        _stream(stream)))
+    return Xq, x_scale
+
+
+def int8_mixed_matmul_workspace_size(M: int, N: int, K: int) -> int:
+    return int(load().int8_mixed_matmul_workspace_size(M, N, K))
+
+
+def int8_mixed_matmul_workspace_layout(M: int, N: int, K: int) -> WorkspaceLayout:
+    lay = WorkspaceLayout()
+    check("int8_mixed_matmul_workspace_layout",
+          load().int8_mixed_matmul_workspace_layout(M, N, K, ctypes.byref(lay)))
+    return lay
+
+
+def int8_mixed_matmul(X, Wq, w_scale, W_fp16, threshold=6.0, Y=None, workspace=None, stream=None):
+    """Y = LLM.int8() decomposition of X . W^T; returns (Y fp16 [M, N], workspace uint8)."""
+    M, K = X.shape
+    N = Wq.shape[0]
+    _need(X, "X", torch.float16, (M, K))
+    _need(Wq, "Wq", torch.int8, (N, K))
+    _need(w_scale, "w_scale", torch.float32, (N,))
+    _need(W_fp16, "W_fp16", torch.float16, (N, K))
+    Y = torch.empty((M, N), dtype=torch.float16, device=X.device) if Y is None else Y
+    _need(Y, "Y", torch.float16, (M, N))
+    need = int8_mixed_matmul_workspace_size(M, N, K)
+    if workspace is None:
+        workspace = torch.empty((max(need, 1),), dtype=torch.uint8, device=X.device)
+    check("int8_mixed_matmul",
+          load().int8_mixed_matmul(_ptr(X), _ptr(Wq), _ptr(w_scale), _ptr(W_fp16), M, N, K,
+                                   float(threshold), _ptr(Y), _ptr(workspace),
+                                   workspace.numel() * workspace.element_size(), _stream(stream)))
+    return Y, workspace
+
+
+def int8_mixed_matmul_profiled(X, Wq, w_scale, W_fp16, threshold, Y, workspace, events,
+                               stream=None):
+    """int8_mixed_matmul that also records three torch.cuda.Event objects on the stream:
+    before the call, between the quantisation stage and the GEMM, and after the GEMM."""
+    M, K = X.shape
+    N = Wq.shape[0]
+    s = torch.cuda.current_stream() if stream is None else stream
+    handles = []
+    for ev in events:
+        if not ev.cuda_event:
+            ev.record(s)   # torch creates the underlying cudaEvent_t lazily
+        handles.append(ev.cuda_event)
+    arr = (ctypes.c_void_p * 3)(*handles)
+    check("int8_mixed_matmul_profiled",
+          load().int8_mixed_matmul_profiled(_ptr(X), _ptr(Wq), _ptr(w_scale), _ptr(W_fp16), M, N, K,
+                                            float(threshold), _ptr(Y), _ptr(workspace),
+                                            workspace.numel() * workspace.element_size(),
+                                            ctypes.c_void_p(s.cuda_stream), arr))
+    return Y
+
+
+def int8_debug_gemm_i32(Xq, Wq, C=None, stream=None):
+    """C int32 [M, N] = Xq . Wq^T on the tensor-core kernel (test hook)."""
+    M, K = Xq.shape
+    N = Wq.shape[0]
+    _need(Xq, "Xq", torch.int8, (M, K))
+    _need(Wq, "Wq", torch.int8, (N, K))
+    C = torch.empty((M, N), dtype=torch.int32, device=Xq.device) if C is None else C
+    _need(C, "C", torch.int32, (M, N))
+    check("int8_debug_gemm_i32",
+          load().int8_debug_gemm_i32(_ptr(Xq), _ptr(Wq), M, N, K, _ptr(C), _stream(stream)))
+    return C
+
+
+def int8_device_status(workspace, stream=None) -> int:
+    """Device status word left by the last int8_mixed_matmul in `workspace` (syncs)."""
+    return int(load().int8_device_status(_ptr(workspace), _stream(stream)))
+
+
+def workspace_views(workspace: torch.Tensor, M: int, N: int, K: int) -> dict:
+    """Tensor views of the intermediates int8_mixed_matmul leaves in its workspace."""
+    lay = int8_mixed_matmul_workspace_layout(M, N, K)
+    words = (K + 31) // 32
+    ld = lay.panel_ld
+
+    def view(off, nbytes, dtype, shape):
+        return workspace[off:off + nbytes].view(dtype).view(shape)
+
+    return dict(
+        n_outliers=view(lay.n_outliers, 4, torch.int32, (1,)),
+        status=view(lay.status, 4, torch.int32, (1,)),
+        col_bitmap=view(lay.col_bitmap, 4 * words, torch.int32, (words,)),
+        col_idx=view(lay.col_idx, 4 * K, torch.int32, (K,)),
+        x_scale=view(lay.x_scale, 4 * M, torch.float32, (M,)),
+        Xq=view(lay.Xq, M * K, torch.int8, (M, K)),
+        X_O=view(lay.X_O, 2 * M * ld, torch.float16, (M, ld)),
+        W_O=view(lay.W_O, 2 * N * ld, torch.float16, (N, ld)),
+    )

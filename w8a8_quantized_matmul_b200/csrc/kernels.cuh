@@ -1,0 +1,65 @@
+// Kernel declarations and launch-shape constants shared by the kernel files
+// and the C-ABI layer of libint8mm.
+#pragma once
+
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+namespace i8mm {
+
+constexpr int kDetectRows = 32;        // rows of X per detection CTA
+constexpr int kQuantRowsPerWarp = 1;   // rows of X per warp in the quantisation kernel
+constexpr int kGatherRows = 32;        // rows of W per W_O gather CTA
+constexpr int kPanelAlign = 64;        // outlier panels are padded to this many columns
+
+__global__ void quantize_weight_rows_kernel(const __half* W, int N, int K, int8_t* Wq,
+                                            float* w_scale);
+
+__global__ void detect_outliers_kernel(const __half* X, int M, int K, float threshold,
+                                       uint32_t* bitmap, int32_t* counter, int32_t* col_idx,
+                                       int32_t* word_prefix);
+
+struct QuantArgs {
+  const __half* X;
+  int M, K;
+  const uint32_t* bitmap;
+  const int32_t* word_prefix;  // COMPACT only
+  const int32_t* n_outliers;   // COMPACT only
+  const int32_t* col_idx;      // COMPACT only
+  int8_t* Xq;
+  float* x_scale;
+  __half* X_O;                 // COMPACT only
+  const __half* W;             // COMPACT only
+  int N;
+  __half* W_O;                 // COMPACT only
+  int ld;
+  int quant_blocks;            // CTAs [0, quant_blocks) quantise rows; the rest gather W_O
+};
+
+// Quantisation (+ compaction) launch; vpl = 16-byte vectors per lane kept in
+// registers (1..32, K <= 256*vpl) or 0 for rows streamed twice.
+cudaError_t launch_quantize_rows(bool compact, int vpl, int grid, size_t smem, cudaStream_t s,
+                                 const QuantArgs& a);
+
+// Host-side launchers of the tensor-core GEMM (gemm_sm100.cu). They encode the
+// TMA tensor maps and launch; the return value is the cudaError_t of the launch.
+struct GemmArgs {
+  const int8_t* Xq;           // [M][K]
+  const int8_t* Wq;           // [N][K]
+  const __half* X_O;          // [M][ld] compacted outlier columns of X (or nullptr)
+  const __half* W_O;          // [N][ld] compacted outlier columns of W (or nullptr)
+  int ld;                     // row stride of the panels, multiple of 64
+  const float* x_scale;       // [M]
+  const float* w_scale;       // [N]
+  const int32_t* n_outliers;  // device count, or nullptr for no outlier pass
+  void* out;                  // fp16 Y [M][N] or int32 C [M][N]
+  int M, N, K;
+  int32_t* status;            // device status word (may be nullptr)
+};
+
+cudaError_t launch_gemm_mixed(const GemmArgs& a, cudaStream_t s);
+cudaError_t launch_gemm_i32(const GemmArgs& a, cudaStream_t s);
+
+}  // namespace i8mm

@@ -1,0 +1,346 @@
+// Memory-bound kernels of the LLM.int8() path on sm_100a:
+//   * quantize_weight_rows_kernel  - offline per-output-row absmax INT8 codes of W
+//   * detect_outliers_kernel        - outlier-column bitmap of X (|x| > threshold),
+//                                     finished by the last CTA into a count, the
+//                                     ascending column list and per-word prefix counts
+//   * quantize_rows_kernel          - per-token absmax over the non-outlier columns,
+//                                     INT8 codes (0 at outliers) and, in the fused
+//                                     path, the compacted fp16 outlier panels of X and W
+//
+// Method: AIInfra "05Infer/06CompDistill/05Quantization01", LLM.int8() section
+// (magnitude-threshold detection, vector-wise absmax quantisation, FP16 outlier
+// columns); tanjunchen "quantization explained part 2", section 1.2 (threshold
+// 6.0; absmax of the remaining dims after the split).
+//
+// All loads of X and W are 128-bit (8 fp16 per lane) and coalesced along K.
+// K is a multiple of 16, so a 16-byte vector never straddles a row end.
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+#include "kernels.cuh"
+
+namespace i8mm {
+
+namespace {
+
+__device__ __forceinline__ void unpack8(const uint4& u, float (&f)[8]) {
+  const __half2* h = reinterpret_cast<const __half2*>(&u);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float2 t = __half22float2(h[i]);
+    f[2 * i] = t.x;
+    f[2 * i + 1] = t.y;
+  }
+}
+
+// clamp(rint((x*127)/a), -127, 127): one exact fp32 product, one IEEE divide,
+// round half to even. a == 0 gives 0.
+__device__ __forceinline__ int quant_code(float x, float a) {
+  if (a == 0.0f) return 0;
+  int q = __float2int_rn(__fdiv_rn(__fmul_rn(x, 127.0f), a));
+  return max(-127, min(127, q));
+}
+
+__device__ __forceinline__ uint32_t pack4(int a, int b, int c, int d) {
+  return (static_cast<uint32_t>(a) & 0xFFu) | ((static_cast<uint32_t>(b) & 0xFFu) << 8) |
+         ((static_cast<uint32_t>(c) & 0xFFu) << 16) | ((static_cast<uint32_t>(d) & 0xFFu) << 24);
+}
+
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+
+// Absmax of the non-outlier entries among the 8 columns 8v..8v+7.
+__device__ __forceinline__ float masked_absmax8(const uint4& u, const uint32_t* s_bits, int v) {
+  const uint32_t m8 = (s_bits[v >> 2] >> (8 * (v & 3))) & 0xFFu;
+  float f[8];
+  unpack8(u, f);
+  float a = 0.0f;
+#pragma unroll
+  for (int i = 0; i < 8; ++i)
+    if (!((m8 >> i) & 1u)) a = fmaxf(a, fabsf(f[i]));
+  return a;
+}
+
+// Codes of the 8 columns 8v..8v+7 (0 at outliers); with COMPACT the outlier
+// entries are also copied to their compacted position in the X_O row.
+template <bool COMPACT>
+__device__ __forceinline__ void quantize8(const uint4& u, const uint32_t* s_bits,
+                                          const int32_t* s_prefix, int v, float amax,
+                                          uint2* dst, __half* xo_row) {
+  const uint32_t wbits = s_bits[v >> 2];
+  const uint32_t m8 = (wbits >> (8 * (v & 3))) & 0xFFu;
+  float f[8];
+  unpack8(u, f);
+  int q[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) q[i] = ((m8 >> i) & 1u) ? 0 : quant_code(f[i], amax);
+  uint2 o;
+  o.x = pack4(q[0], q[1], q[2], q[3]);
+  o.y = pack4(q[4], q[5], q[6], q[7]);
+  dst[v] = o;
+  if (COMPACT && m8) {
+    const __half* hv = reinterpret_cast<const __half*>(&u);
+    const int base = s_prefix[v >> 2];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      if ((m8 >> i) & 1u) {
+        const int bit = 8 * (v & 3) + i;
+        xo_row[base + __popc(wbits & ((1u << bit) - 1u))] = hv[i];
+      }
+    }
+  }
+}
+
+}  // namespace
+
+// ---------------------------------------------------------------------------
+// Offline weight quantisation: one warp per output row n.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) quantize_weight_rows_kernel(const __half* __restrict__ W,
+                                                                   int N, int K,
+                                                                   int8_t* __restrict__ Wq,
+                                                                   float* __restrict__ w_scale) {
+  const int row = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (row >= N) return;
+  const uint4* src = reinterpret_cast<const uint4*>(W + static_cast<size_t>(row) * K);
+  const int nv = K >> 3;
+  float amax = 0.0f;
+  for (int v = lane; v < nv; v += 32) {
+    float f[8];
+    unpack8(__ldg(src + v), f);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(f[i]));
+  }
+  amax = warp_max(amax);
+  uint2* dst = reinterpret_cast<uint2*>(Wq + static_cast<size_t>(row) * K);
+  for (int v = lane; v < nv; v += 32) {
+    float f[8];
+    unpack8(__ldg(src + v), f);
+    uint2 o;
+    o.x = pack4(quant_code(f[0], amax), quant_code(f[1], amax), quant_code(f[2], amax),
+                quant_code(f[3], amax));
+    o.y = pack4(quant_code(f[4], amax), quant_code(f[5], amax), quant_code(f[6], amax),
+                quant_code(f[7], amax));
+    dst[v] = o;
+  }
+  if (lane == 0) w_scale[row] = amax;
+}
+
+// ---------------------------------------------------------------------------
+// Outlier detection. Grid: x = column slabs of 256 columns (32 lanes x 8),
+// y = row blocks of kDetectRows rows (each of the 8 warps takes every 8th row).
+// `bitmap` and `counter` must be zero on entry. The last CTA to finish turns the
+// bitmap into count / ascending list / per-word exclusive prefix, and leaves the
+// count in *counter (which doubles as the arrival counter until then).
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) detect_outliers_kernel(
+    const __half* __restrict__ X, int M, int K, float threshold, uint32_t* bitmap,
+    int32_t* counter, int32_t* __restrict__ col_idx, int32_t* __restrict__ word_prefix) {
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int v = blockIdx.x * 32 + lane;  // uint4 index along the row (8 columns)
+  const int nv = K >> 3;
+  const int r0 = blockIdx.y * kDetectRows;
+  const int r1 = min(M, r0 + kDetectRows);
+
+  uint32_t flags = 0;  // bit b: column 8v+b has |x| > threshold in some row seen here
+  if (v < nv) {
+    int r = r0 + warp;
+#pragma unroll 4
+    for (; r < r1; r += 8) {
+      float f[8];
+      unpack8(__ldg(reinterpret_cast<const uint4*>(X + static_cast<size_t>(r) * K) + v), f);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) flags |= (fabsf(f[i]) > threshold ? 1u : 0u) << i;
+    }
+  }
+  // Lanes 4w..4w+3 cover the 32 columns of one bitmap word.
+  uint32_t word = flags << (8 * (lane & 3));
+  word |= __shfl_xor_sync(0xffffffffu, word, 1);
+  word |= __shfl_xor_sync(0xffffffffu, word, 2);
+  if ((lane & 3) == 0 && word != 0 && v < nv) atomicOr(bitmap + (v >> 2), word);
+
+  // Last-CTA finalisation (fence + arrival counter; no waiting).
+  __shared__ bool is_last;
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    const int total = gridDim.x * gridDim.y;
+    const int prev = atomicAdd(counter, 1);
+    is_last = (prev == total - 1);
+  }
+  __syncthreads();
+  if (!is_last) return;
+  __threadfence();
+
+  const int words = (K + 31) >> 5;
+  __shared__ int32_t warp_sums[32];
+  __shared__ int32_t carry;
+  if (threadIdx.x == 0) carry = 0;
+  __syncthreads();
+  for (int base = 0; base < words; base += blockDim.x) {
+    const int w = base + threadIdx.x;
+    const uint32_t bits = (w < words) ? __ldcg(bitmap + w) : 0u;
+    const int c = __popc(bits);
+    // Block-wide exclusive scan of c.
+    int incl = c;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int t = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += t;
+    }
+    if (lane == 31) warp_sums[warp] = incl;
+    __syncthreads();
+    if (warp == 0) {
+      int s = (lane < (int)(blockDim.x >> 5)) ? warp_sums[lane] : 0;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int t = __shfl_up_sync(0xffffffffu, s, o);
+        if (lane >= o) s += t;
+      }
+      warp_sums[lane] = s;  // inclusive over warps
+    }
+    __syncthreads();
+    const int excl = carry + (warp > 0 ? warp_sums[warp - 1] : 0) + incl - c;
+    if (w < words) {
+      if (word_prefix) word_prefix[w] = excl;
+      if (col_idx) {
+        uint32_t b = bits;
+        int p = excl;
+        while (b) {
+          const int j = __ffs(b) - 1;
+          b &= b - 1;
+          col_idx[p++] = w * 32 + j;
+        }
+      }
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) carry += warp_sums[(blockDim.x >> 5) - 1];
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) *counter = carry;
+}
+
+// ---------------------------------------------------------------------------
+// Per-token quantisation. One warp per row; the row is held in registers
+// (VPL 16-byte vectors per lane, VPL*256 >= K), so X is read from memory once.
+// COMPACT additionally writes the outlier columns of the row into X_O (row
+// stride ld, zero-padded to a multiple of 64) and, in the CTAs past the
+// quantisation rows, gathers the outlier columns of W into W_O.
+// ---------------------------------------------------------------------------
+template <int VPL, bool COMPACT>
+__global__ void __launch_bounds__(256) quantize_rows_kernel(
+    const __half* __restrict__ X, int M, int K, const uint32_t* __restrict__ bitmap,
+    const int32_t* __restrict__ word_prefix, const int32_t* __restrict__ n_outliers,
+    const int32_t* __restrict__ col_idx, int8_t* __restrict__ Xq, float* __restrict__ x_scale,
+    __half* __restrict__ X_O, const __half* __restrict__ W, int N, __half* __restrict__ W_O,
+    int ld, int quant_blocks) {
+  extern __shared__ uint32_t qsmem[];
+  const int words = (K + 31) >> 5;
+  uint32_t* s_bits = qsmem;
+  int32_t* s_prefix = reinterpret_cast<int32_t*>(qsmem + words);
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (COMPACT && static_cast<int>(blockIdx.x) >= quant_blocks) {
+    // W_O[n][p] = W[n][col_idx[p]] for p < count, 0 up to the next multiple of 64.
+    const int count = *n_outliers;
+    const int pad = (count + 63) & ~63;
+    const int n0 = (blockIdx.x - quant_blocks) * kGatherRows;
+    const int n1 = min(N, n0 + kGatherRows);
+    for (int n = n0 + warp; n < n1; n += 8) {
+      const __half* wrow = W + static_cast<size_t>(n) * K;
+      __half* orow = W_O + static_cast<size_t>(n) * ld;
+      for (int p = lane; p < pad; p += 32)
+        orow[p] = (p < count) ? wrow[__ldg(col_idx + p)] : __float2half_rn(0.0f);
+    }
+    return;
+  }
+
+  for (int w = threadIdx.x; w < words; w += blockDim.x) {
+    s_bits[w] = bitmap[w];
+    if (COMPACT) s_prefix[w] = word_prefix[w];
+  }
+  __syncthreads();
+  int count = 0;
+  if (COMPACT) count = *n_outliers;
+  const int pad = (count + 63) & ~63;
+  const int nv = K >> 3;
+
+  const int rows_per_block = 8 * kQuantRowsPerWarp;
+  const int rbeg = blockIdx.x * rows_per_block;
+  for (int rr = warp; rr < rows_per_block; rr += 8) {
+    const int row = rbeg + rr;
+    if (row >= M) break;
+    const uint4* src = reinterpret_cast<const uint4*>(X + static_cast<size_t>(row) * K);
+    uint2* dst = reinterpret_cast<uint2*>(Xq + static_cast<size_t>(row) * K);
+    __half* xo_row = COMPACT ? X_O + static_cast<size_t>(row) * ld : nullptr;
+    float amax = 0.0f;
+    if constexpr (VPL > 0) {
+      uint4 buf[VPL];
+#pragma unroll
+      for (int t = 0; t < VPL; ++t) {
+        const int v = lane + 32 * t;
+        if (v < nv) buf[t] = __ldg(src + v);
+      }
+#pragma unroll
+      for (int t = 0; t < VPL; ++t) {
+        const int v = lane + 32 * t;
+        if (v < nv) amax = fmaxf(amax, masked_absmax8(buf[t], s_bits, v));
+      }
+      amax = warp_max(amax);
+#pragma unroll
+      for (int t = 0; t < VPL; ++t) {
+        const int v = lane + 32 * t;
+        if (v < nv) quantize8<COMPACT>(buf[t], s_bits, s_prefix, v, amax, dst, xo_row);
+      }
+    } else {
+      // Rows longer than the register budget: two passes, the second from L1/L2.
+      for (int v = lane; v < nv; v += 32) amax = fmaxf(amax, masked_absmax8(__ldg(src + v), s_bits, v));
+      amax = warp_max(amax);
+      for (int v = lane; v < nv; v += 32)
+        quantize8<COMPACT>(__ldg(src + v), s_bits, s_prefix, v, amax, dst, xo_row);
+    }
+    if (COMPACT) {
+      for (int p = count + lane; p < pad; p += 32) xo_row[p] = __float2half_rn(0.0f);
+    }
+    if (lane == 0) x_scale[row] = amax;
+  }
+}
+
+// Host-side dispatch on the register budget VPL (0 = streaming rows).
+cudaError_t launch_quantize_rows(bool compact, int vpl, int grid, size_t smem, cudaStream_t s,
+                                 const QuantArgs& a) {
+#define I8MM_CASE(V)                                                                          \
+  case V:                                                                                     \
+    if (compact)                                                                              \
+      quantize_rows_kernel<V, true><<<grid, 256, smem, s>>>(                                   \
+          a.X, a.M, a.K, a.bitmap, a.word_prefix, a.n_outliers, a.col_idx, a.Xq, a.x_scale,   \
+          a.X_O, a.W, a.N, a.W_O, a.ld, a.quant_blocks);                                       \
+    else                                                                                      \
+      quantize_rows_kernel<V, false><<<grid, 256, smem, s>>>(                                  \
+          a.X, a.M, a.K, a.bitmap, a.word_prefix, a.n_outliers, a.col_idx, a.Xq, a.x_scale,   \
+          a.X_O, a.W, a.N, a.W_O, a.ld, a.quant_blocks);                                       \
+    break;
+  switch (vpl) {
+    I8MM_CASE(0)
+    I8MM_CASE(1)
+    I8MM_CASE(2)
+    I8MM_CASE(4)
+    I8MM_CASE(8)
+    I8MM_CASE(16)
+    I8MM_CASE(32)
+    default:
+      return cudaErrorInvalidValue;
+  }
+#undef I8MM_CASE
+  return cudaGetLastError();
+}
+
+}  // namespace i8mm
