@@ -105,6 +105,7 @@ def test_other_entry_points_validation(lib):
     assert lib.int8_find_outlier_cols(A, 4, 64, math.nan, A, A, A, None) == _lib.I8MM_ERR_INVALID_ARG
     assert lib.int8_find_outlier_cols(A, 4, 64, -0.5, A, A, A, None) == _lib.I8MM_ERR_INVALID_ARG
     assert lib.int8_find_outlier_cols(A, 4, 64, 6.0, None, A, A, None) == _lib.I8MM_ERR_INVALID_ARG
+    assert lib.int8_find_outlier_cols(None, 4, 64, 6.0, A, A, A, None) == _lib.I8MM_ERR_INVALID_ARG
     assert lib.int8_find_outlier_cols(A, 4, 64, 6.0, A, None, A, None) == _lib.I8MM_ERR_INVALID_ARG
     assert lib.int8_find_outlier_cols(A, 4, 64, 6.0, A, A, MIS, None) == _lib.I8MM_ERR_ALIGNMENT
     assert lib.int8_find_outlier_cols(A, 4, 8, 6.0, A, A, A, None) == _lib.I8MM_ERR_ALIGNMENT

@@ -235,3 +235,46 @@ def test_empty_problem_is_a_noop():
     X = torch.empty((0, 64), dtype=torch.float16, device="cuda")
     Y, _ = m.int8_mixed_matmul(X, Wq, ws, W, 6.0)
     assert tuple(Y.shape) == (0, 64)
+
+
+# ---------------------------------------------------------------- every fp16 input value
+def _every_value_rows(amaxes):
+    """Row i holds amaxes[i] and every finite fp16 x with |x| <= amaxes[i] (zero-padded)."""
+    allh = np.arange(65536, dtype=np.uint16).view(np.float16)
+    allh = allh[np.isfinite(allh)]
+    rows = []
+    for a in amaxes:
+        a16 = np.float16(a)
+        v = allh[np.abs(allh.astype(np.float32)) <= np.float32(a16)]
+        rows.append(np.concatenate([[a16], v]))
+    K = (max(r.size for r in rows) + 15) // 16 * 16
+    X = np.zeros((len(rows), K), np.float16)
+    for i, r in enumerate(rows):
+        X[i, :r.size] = r
+    return X
+
+
+AMAXES = [127 / 64, 6.0, 5.99609375, 1.0, 0.5, 3.140625, 0.0078125, 2.0 ** -14, 1000.0, 0.333251953125]
+
+
+def test_quantize_every_fp16_value_standalone():
+    """All rounding cases (exact ties, near-ties, clamps) of the quantiser, bit-exact."""
+    X = _every_value_rows(AMAXES)
+    K = X.shape[1]
+    mask = np.zeros(K, bool)
+    bitmap = np.zeros((K + 31) // 32, np.uint32)
+    Xq, xs = mm().int8_quantize_act_rows(dev(X), dev(bitmap.view(np.int32)))
+    rq, rs = oracle.quantize_act_rows(X, mask)
+    assert np.array_equal(host(xs), rs)
+    assert np.array_equal(host(Xq), rq)
+
+
+def test_quantize_every_fp16_value_fused_path():
+    """The same sweep through int8_mixed_matmul (threshold=inf: no outliers)."""
+    X = _every_value_rows(AMAXES[:6])
+    K = X.shape[1]
+    W = synth.make_weight(8, K, 0.02, seed=77)
+    Y, got, Wq, ws = run_mixed(X, W, math.inf)
+    ref = oracle.llm_int8_matmul(X, W, math.inf)
+    check_intermediates(ref, got, K)
+    assert_y_close(Y, ref["Y"], "every-value")

@@ -2,12 +2,11 @@
 // workspace carving, and the launch sequence of the LLM.int8() path.
 //
 // int8_mixed_matmul on one stream, no host synchronisation:
-//   1. cudaMemsetAsync   zero the outlier bitmap and the arrival counter
-//   2. detect            |x| > threshold column bitmap; the last CTA writes the
-//                        count, the ascending column list and per-word prefix counts
-//   3. quantize+compact  per-token absmax INT8 codes over the non-outlier columns,
-//                        compacted fp16 outlier panels X_O and W_O
-//   4. GEMM              tcgen05 INT8 GEMM + fp16 outlier GEMM + dequantising epilogue
+//   1. cudaMemsetAsync   zero the count/status/barrier words and the outlier bitmap
+//   2. fused K1          cooperative kernel: |x| > threshold column bitmap, grid
+//                        barrier, per-token absmax INT8 codes over the non-outlier
+//                        columns, compacted fp16 outlier panels X_O and W_O
+//   3. GEMM              tcgen05 INT8 GEMM + fp16 outlier GEMM + dequantising epilogue
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
@@ -76,7 +75,6 @@ int vpl_for(int K) {
 
 struct Layout {
   i8mm_workspace_layout l;
-  size_t word_prefix;
 };
 
 bool make_layout(int M, int N, int K, Layout* out) {
@@ -91,11 +89,10 @@ bool make_layout(int M, int N, int K, Layout* out) {
   };
   Layout L{};
   // The count and the bitmap sit together so one memset clears both.
-  L.l.n_outliers = take(16);              // [0] count / arrival counter, [1] status
+  L.l.n_outliers = take(16);              // [0] count, [1] status, [2] grid-barrier counter
   L.l.status = L.l.n_outliers + 4;
   L.l.col_bitmap = L.l.n_outliers + 16;   // directly after, inside the same memset span
   off = align_up(L.l.col_bitmap + words * 4, kAlign);
-  L.word_prefix = take(words * 4);
   L.l.col_idx = take(static_cast<size_t>(K) * 4);
   L.l.x_scale = take(static_cast<size_t>(M) * 4);
   L.l.Xq = take(static_cast<size_t>(M) * K);
@@ -159,7 +156,7 @@ int int8_find_outlier_cols(const void* X, int M, int K, float threshold, uint32_
   int st = check_sizes(M, 1, K);
   if (st != I8MM_OK) return st;
   if ((st = check_threshold(threshold)) != I8MM_OK) return st;
-  if (!X || !col_bitmap || !n_outliers) return I8MM_ERR_INVALID_ARG;
+  if ((M > 0 && !X) || !col_bitmap || !n_outliers) return I8MM_ERR_INVALID_ARG;
   if (!aligned16(X) || !aligned16(col_bitmap) || !aligned16(n_outliers) ||
       (col_idx && !aligned16(col_idx)))
     return I8MM_ERR_ALIGNMENT;
@@ -171,7 +168,7 @@ int int8_find_outlier_cols(const void* X, int M, int K, float threshold, uint32_
   const int nv = K / 8;
   dim3 grid((nv + 31) / 32, M > 0 ? (M + kDetectRows - 1) / kDetectRows : 1);
   detect_outliers_kernel<<<grid, 256, 0, stream>>>(static_cast<const __half*>(X), M, K, threshold,
-                                                  col_bitmap, n_outliers, col_idx, nullptr);
+                                                  col_bitmap, n_outliers, col_idx);
   return cuda_status(cudaGetLastError());
 }
 
@@ -187,7 +184,7 @@ int int8_quantize_act_rows(const void* X, int M, int K, const uint32_t* col_bitm
   const int words = (K + 31) / 32;
   const int rows_per_block = 8 * kQuantRowsPerWarp;
   const int qb = (M + rows_per_block - 1) / rows_per_block;
-  const size_t smem = static_cast<size_t>(words) * 8;
+  const size_t smem = static_cast<size_t>(words) * 4;
   QuantArgs qa{};
   qa.X = static_cast<const __half*>(X);
   qa.M = M;
@@ -195,8 +192,7 @@ int int8_quantize_act_rows(const void* X, int M, int K, const uint32_t* col_bitm
   qa.bitmap = col_bitmap;
   qa.Xq = Xq;
   qa.x_scale = x_scale;
-  qa.quant_blocks = qb;
-  return cuda_status(launch_quantize_rows(false, vpl_for(K), qb, smem, stream, qa));
+  return cuda_status(launch_quantize_rows(vpl_for(K), qb, smem, stream, qa));
 }
 
 }  // extern "C"
@@ -219,14 +215,13 @@ int mixed_matmul_impl(const void* X, const int8_t* Wq, const float* w_scale, con
   if (!workspace || workspace_bytes < L.l.total) return I8MM_ERR_WORKSPACE;
   if ((reinterpret_cast<uintptr_t>(workspace) & (kAlign - 1)) != 0) return I8MM_ERR_ALIGNMENT;
   const int words = (K + 31) / 32;
-  const size_t qsmem = static_cast<size_t>(words) * 8;
   if ((st = check_device()) != I8MM_OK) return st;
 
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   int32_t* count = reinterpret_cast<int32_t*>(ws + L.l.n_outliers);
   int32_t* status = reinterpret_cast<int32_t*>(ws + L.l.status);
+  int32_t* sync_ctr = reinterpret_cast<int32_t*>(ws + L.l.status + 4);
   uint32_t* bitmap = reinterpret_cast<uint32_t*>(ws + L.l.col_bitmap);
-  int32_t* prefix = reinterpret_cast<int32_t*>(ws + L.word_prefix);
   int32_t* idx = reinterpret_cast<int32_t*>(ws + L.l.col_idx);
   float* xs = reinterpret_cast<float*>(ws + L.l.x_scale);
   int8_t* Xq = reinterpret_cast<int8_t*>(ws + L.l.Xq);
@@ -241,34 +236,25 @@ int mixed_matmul_impl(const void* X, const int8_t* Wq, const float* w_scale, con
                                   (L.l.col_bitmap - L.l.n_outliers) + static_cast<size_t>(words) * 4,
                                   stream);
   if (e != cudaSuccess) return I8MM_ERR_CUDA;
-  // 2. detection
-  const int nv = K / 8;
-  dim3 dgrid((nv + 31) / 32, (M + kDetectRows - 1) / kDetectRows);
-  detect_outliers_kernel<<<dgrid, 256, 0, stream>>>(Xh, M, K, threshold, bitmap, count, idx,
-                                                   prefix);
-  if ((e = cudaGetLastError()) != cudaSuccess) return I8MM_ERR_CUDA;
-  // 3. quantisation + compaction (+ W_O gather in the trailing CTAs)
-  const int rows_per_block = 8 * kQuantRowsPerWarp;
-  const int qb = (M + rows_per_block - 1) / rows_per_block;
-  const int gb = (N + kGatherRows - 1) / kGatherRows;
-  QuantArgs qa{};
-  qa.X = Xh;
-  qa.M = M;
-  qa.K = K;
-  qa.bitmap = bitmap;
-  qa.word_prefix = prefix;
-  qa.n_outliers = count;
-  qa.col_idx = idx;
-  qa.Xq = Xq;
-  qa.x_scale = xs;
-  qa.X_O = XO;
-  qa.W = Wh;
-  qa.N = N;
-  qa.W_O = WO;
-  qa.ld = L.l.panel_ld;
-  qa.quant_blocks = qb;
-  e = launch_quantize_rows(true, vpl_for(K), qb + gb, qsmem, stream, qa);
-  if (e != cudaSuccess) return I8MM_ERR_CUDA;
+  // 2+3. detection, quantisation and compaction: one cooperative kernel
+  FusedArgs fa{};
+  fa.X = Xh;
+  fa.M = M;
+  fa.K = K;
+  fa.N = N;
+  fa.threshold = threshold;
+  fa.bitmap = bitmap;
+  fa.sync_ctr = sync_ctr;
+  fa.n_outliers = count;
+  fa.col_idx = idx;
+  fa.Xq = Xq;
+  fa.x_scale = xs;
+  fa.X_O = XO;
+  fa.W = Wh;
+  fa.W_O = WO;
+  fa.ld = L.l.panel_ld;
+  fa.status = status;
+  if (launch_detect_quantize_compact(fa, stream) != cudaSuccess) return I8MM_ERR_CUDA;
   if (ev && cudaEventRecord(ev[1], stream) != cudaSuccess) return I8MM_ERR_CUDA;
   // 4. GEMM
   GemmArgs g{};

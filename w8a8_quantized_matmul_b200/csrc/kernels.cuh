@@ -11,37 +11,46 @@ namespace i8mm {
 
 constexpr int kDetectRows = 32;        // rows of X per detection CTA
 constexpr int kQuantRowsPerWarp = 1;   // rows of X per warp in the quantisation kernel
-constexpr int kGatherRows = 32;        // rows of W per W_O gather CTA
 constexpr int kPanelAlign = 64;        // outlier panels are padded to this many columns
 
 __global__ void quantize_weight_rows_kernel(const __half* W, int N, int K, int8_t* Wq,
                                             float* w_scale);
 
 __global__ void detect_outliers_kernel(const __half* X, int M, int K, float threshold,
-                                       uint32_t* bitmap, int32_t* counter, int32_t* col_idx,
-                                       int32_t* word_prefix);
+                                       uint32_t* bitmap, int32_t* counter, int32_t* col_idx);
 
 struct QuantArgs {
   const __half* X;
   int M, K;
   const uint32_t* bitmap;
-  const int32_t* word_prefix;  // COMPACT only
-  const int32_t* n_outliers;   // COMPACT only
-  const int32_t* col_idx;      // COMPACT only
   int8_t* Xq;
   float* x_scale;
-  __half* X_O;                 // COMPACT only
-  const __half* W;             // COMPACT only
-  int N;
-  __half* W_O;                 // COMPACT only
-  int ld;
-  int quant_blocks;            // CTAs [0, quant_blocks) quantise rows; the rest gather W_O
 };
 
-// Quantisation (+ compaction) launch; vpl = 16-byte vectors per lane kept in
+// Stand-alone quantisation launch; vpl = 16-byte vectors per lane kept in
 // registers (1..32, K <= 256*vpl) or 0 for rows streamed twice.
-cudaError_t launch_quantize_rows(bool compact, int vpl, int grid, size_t smem, cudaStream_t s,
+cudaError_t launch_quantize_rows(int vpl, int grid, size_t smem, cudaStream_t s,
                                  const QuantArgs& a);
+
+// Fused detection + quantisation + compaction (cooperative launch).
+struct FusedArgs {
+  const __half* X;
+  int M, K, N;
+  float threshold;
+  uint32_t* bitmap;       // [ceil(K/32)], zero on entry
+  int32_t* sync_ctr;      // zero on entry; grid-barrier arrival counter
+  int32_t* n_outliers;    // out: count
+  int32_t* col_idx;       // out: ascending outlier columns
+  int8_t* Xq;             // out: [M][K]
+  float* x_scale;         // out: [M]
+  __half* X_O;            // out: [M][ld]
+  const __half* W;        // in : [N][K]
+  __half* W_O;            // out: [N][ld]
+  int ld;
+  int32_t* status;        // device status word
+};
+
+cudaError_t launch_detect_quantize_compact(const FusedArgs& a, cudaStream_t s);
 
 // Host-side launchers of the tensor-core GEMM (gemm_sm100.cu). They encode the
 // TMA tensor maps and launch; the return value is the cudaError_t of the launch.
