@@ -106,7 +106,11 @@ size_t int8_mixed_matmul_workspace_size(int M, int N, int K);
  * (byte offsets from the workspace base; each at least 16-byte aligned). Lets a
  * caller or a test read the outlier set, codes and scales of the last call.
  * The outlier panels have row stride panel_ld elements (fp16) and hold the
- * compacted outlier columns, zero-padded to a multiple of 64.
+ * compacted outlier columns in ascending column order, zero-padded to 16
+ * columns when there are 1..16 outliers (the GEMM epilogue then adds the
+ * outlier product on CUDA cores) or to a multiple of 64 when there are more
+ * (the GEMM multiplies them on the tensor cores). Nothing is written when
+ * there are no outliers.
  */
 typedef struct {
   size_t n_outliers;   /* int32 [1] */
@@ -158,6 +162,21 @@ int int8_mixed_matmul_profiled(const void* X, const int8_t* Wq, const float* w_s
                                i8mm_stream_t stream, void* const* events);
 
 /*
+ * Measurement hook: one stage of int8_mixed_matmul on its own, so that each
+ * kernel can be timed back to back.
+ *   stage 1: clear the control words and run the detection / quantisation /
+ *            compaction kernel (writes the workspace intermediates);
+ *   stage 2: run only the GEMM kernel on the intermediates already in the
+ *            workspace (a previous stage 1 or full call with the same X, sizes,
+ *            threshold and workspace must have completed on the stream).
+ * Other arguments as for int8_mixed_matmul; any other stage value is
+ * I8MM_ERR_INVALID_ARG.
+ */
+int int8_mixed_matmul_stage(int stage, const void* X, const int8_t* Wq, const float* w_scale,
+                            const void* W_fp16, int M, int N, int K, float threshold, void* Y,
+                            void* workspace, size_t workspace_bytes, i8mm_stream_t stream);
+
+/*
  * Test hook: the INT8 x INT8 -> INT32 product alone (AIInfra LLM.int8()
  * section, "C_i32 = X_i8 x W_i8", accumulated in INT32), on the same
  * tensor-core kernel the full path uses.
@@ -175,6 +194,13 @@ int int8_device_status(const void* workspace, i8mm_stream_t stream);
 
 /* Static string for a status code. */
 const char* int8_status_string(int status);
+
+/*
+ * Text of the CUDA error behind the last I8MM_ERR_CUDA returned on the
+ * calling host thread (which call failed and the CUDA error name), or "" if
+ * none. The pointer stays valid until the thread's next failing call.
+ */
+const char* int8_last_error_string(void);
 
 #ifdef __cplusplus
 }

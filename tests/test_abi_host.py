@@ -116,6 +116,12 @@ def test_other_entry_points_validation(lib):
     assert lib.int8_debug_gemm_i32(A, None, 4, 4, 32, A, None) == _lib.I8MM_ERR_INVALID_ARG
     assert lib.int8_debug_gemm_i32(A, A, 0, 4, 32, A, None) == _lib.I8MM_OK
     assert lib.int8_device_status(None, None) == _lib.I8MM_ERR_INVALID_ARG
+    need = lib.int8_mixed_matmul_workspace_size(64, 64, 64)
+    assert lib.int8_mixed_matmul_stage(3, A, A, A, A, 64, 64, 64, 6.0, A, A, need, None) == _lib.I8MM_ERR_INVALID_ARG
+    assert lib.int8_mixed_matmul_stage(1, A, A, A, A, 64, 64, 24, 6.0, A, A, need, None) == _lib.I8MM_ERR_ALIGNMENT
+    assert lib.int8_mixed_matmul_stage(2, A, A, A, A, 64, 64, 64, 6.0, A, None, need, None) == _lib.I8MM_ERR_WORKSPACE
+    ev = (ctypes.c_void_p * 3)(None, None, None)
+    assert lib.int8_mixed_matmul_profiled(A, A, A, A, 64, 64, 64, 6.0, A, A, need, None, ev) == _lib.I8MM_ERR_INVALID_ARG
 
 
 @pytest.mark.parametrize("M,N,K", [(1, 1, 16), (16, 256, 256), (200, 264, 272), (2048, 16384, 4096),

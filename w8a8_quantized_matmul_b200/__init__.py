@@ -35,6 +35,7 @@ __all__ = [
     "int8_mixed_matmul_workspace_layout",
     "int8_mixed_matmul",
     "int8_mixed_matmul_profiled",
+    "int8_mixed_matmul_stage",
     "int8_debug_gemm_i32",
     "int8_device_status",
     "Int8mmError",
@@ -158,6 +159,18 @@ def int8_mixed_matmul_profiled(X, Wq, w_scale, W_fp16, threshold, Y, workspace, 
                                             float(threshold), _ptr(Y), _ptr(workspace),
                                             workspace.numel() * workspace.element_size(),
                                             ctypes.c_void_p(s.cuda_stream), arr))
+    return Y
+
+
+def int8_mixed_matmul_stage(stage, X, Wq, w_scale, W_fp16, threshold, Y, workspace, stream=None):
+    """One stage of int8_mixed_matmul (1: quantisation kernel, 2: GEMM kernel) for timing."""
+    M, K = X.shape
+    N = Wq.shape[0]
+    check("int8_mixed_matmul_stage",
+          load().int8_mixed_matmul_stage(int(stage), _ptr(X), _ptr(Wq), _ptr(w_scale), _ptr(W_fp16),
+                                         M, N, K, float(threshold), _ptr(Y), _ptr(workspace),
+                                         workspace.numel() * workspace.element_size(),
+                                         _stream(stream)))
     return Y
 
 

@@ -34,9 +34,11 @@ PROTOTYPES = {
     "int8_mixed_matmul": (_i, [_vp, _vp, _vp, _vp, _i, _i, _i, _f, _vp, _vp, _sz, _vp]),
     "int8_mixed_matmul_profiled": (_i, [_vp, _vp, _vp, _vp, _i, _i, _i, _f, _vp, _vp, _sz, _vp,
                                         ctypes.POINTER(_vp)]),
+    "int8_mixed_matmul_stage": (_i, [_i, _vp, _vp, _vp, _vp, _i, _i, _i, _f, _vp, _vp, _sz, _vp]),
     "int8_debug_gemm_i32": (_i, [_vp, _vp, _i, _i, _i, _vp, _vp]),
     "int8_device_status": (_i, [_vp, _vp]),
     "int8_status_string": (ctypes.c_char_p, [_i]),
+    "int8_last_error_string": (ctypes.c_char_p, []),
 }
 
 _lib = None
@@ -45,7 +47,10 @@ _lib = None
 class Int8mmError(RuntimeError):
     def __init__(self, fn: str, status: int):
         self.status = status
-        super().__init__(f"{fn} failed: {status} ({status_string(status)})")
+        detail = ""
+        if status == I8MM_ERR_CUDA:
+            detail = ": " + load().int8_last_error_string().decode()
+        super().__init__(f"{fn} failed: {status} ({status_string(status)}){detail}")
 
 
 def load() -> ctypes.CDLL:

@@ -12,8 +12,9 @@
 
 #include <cmath>
 #include <cstdint>
+#include <cstdio>
 
-#include "../../include/int8mm.h"
+#include "int8mm.h"
 #include "kernels.cuh"
 
 namespace {
@@ -59,7 +60,17 @@ int check_device() {
   return ok ? I8MM_OK : I8MM_ERR_UNSUPPORTED_DEVICE;
 }
 
-int cuda_status(cudaError_t e) { return e == cudaSuccess ? I8MM_OK : I8MM_ERR_CUDA; }
+thread_local char g_last_error[256] = "";
+
+// Records which step failed and why, and returns I8MM_ERR_CUDA (I8MM_OK on success).
+int cuda_fail(const char* what, cudaError_t e) {
+  if (e == cudaSuccess) return I8MM_OK;
+  std::snprintf(g_last_error, sizeof(g_last_error), "%s: %s (%s)", what, cudaGetErrorName(e),
+                cudaGetErrorString(e));
+  return I8MM_ERR_CUDA;
+}
+
+int cuda_status(cudaError_t e) { return cuda_fail("launch", e); }
 
 // Register-resident vectors per lane for a row of K fp16 values (0 = streaming).
 int vpl_for(int K) {
@@ -107,6 +118,8 @@ bool make_layout(int M, int N, int K, Layout* out) {
 }  // namespace
 
 extern "C" {
+
+const char* int8_last_error_string(void) { return g_last_error; }
 
 const char* int8_status_string(int status) {
   switch (status) {
@@ -199,9 +212,11 @@ int int8_quantize_act_rows(const void* X, int M, int K, const uint32_t* col_bitm
 
 namespace {
 
+// stages: bit 0 = control-word clear + fused quantisation kernel, bit 1 = GEMM.
 int mixed_matmul_impl(const void* X, const int8_t* Wq, const float* w_scale, const void* W_fp16,
                       int M, int N, int K, float threshold, void* Y, void* workspace,
-                      size_t workspace_bytes, cudaStream_t stream, cudaEvent_t const* ev) {
+                      size_t workspace_bytes, cudaStream_t stream, cudaEvent_t const* ev,
+                      int stages = 3) {
   int st = check_sizes(M, N, K);
   if (st != I8MM_OK) return st;
   if ((st = check_threshold(threshold)) != I8MM_OK) return st;
@@ -231,37 +246,43 @@ int mixed_matmul_impl(const void* X, const int8_t* Wq, const float* w_scale, con
   const __half* Wh = static_cast<const __half*>(W_fp16);
 
   if (ev && cudaEventRecord(ev[0], stream) != cudaSuccess) return I8MM_ERR_CUDA;
-  // 1. count, status and bitmap are contiguous: one memset.
-  cudaError_t e = cudaMemsetAsync(ws + L.l.n_outliers, 0,
-                                  (L.l.col_bitmap - L.l.n_outliers) + static_cast<size_t>(words) * 4,
-                                  stream);
-  if (e != cudaSuccess) return I8MM_ERR_CUDA;
-  // 2+3. detection, quantisation and compaction: one cooperative kernel
-  FusedArgs fa{};
-  fa.X = Xh;
-  fa.M = M;
-  fa.K = K;
-  fa.N = N;
-  fa.threshold = threshold;
-  fa.bitmap = bitmap;
-  fa.sync_ctr = sync_ctr;
-  fa.n_outliers = count;
-  fa.col_idx = idx;
-  fa.Xq = Xq;
-  fa.x_scale = xs;
-  fa.X_O = XO;
-  fa.W = Wh;
-  fa.W_O = WO;
-  fa.ld = L.l.panel_ld;
-  fa.status = status;
-  if (launch_detect_quantize_compact(fa, stream) != cudaSuccess) return I8MM_ERR_CUDA;
+  if (stages & 1) {
+    // 1. count, status, barrier counter and bitmap are contiguous: one memset.
+    const size_t ctrl = (L.l.col_bitmap - L.l.n_outliers) + static_cast<size_t>(words) * 4;
+    cudaError_t e = cudaMemsetAsync(ws + L.l.n_outliers, 0, ctrl, stream);
+    if (e != cudaSuccess) return cuda_fail("control-word memset", e);
+    // 2. detection, quantisation and compaction: one cooperative kernel
+    FusedArgs fa{};
+    fa.X = Xh;
+    fa.M = M;
+    fa.K = K;
+    fa.N = N;
+    fa.threshold = threshold;
+    fa.bitmap = bitmap;
+    fa.sync_ctr = sync_ctr;
+    fa.n_outliers = count;
+    fa.col_idx = idx;
+    fa.Xq = Xq;
+    fa.x_scale = xs;
+    fa.X_O = XO;
+    fa.W = Wh;
+    fa.W_O = WO;
+    fa.ld = L.l.panel_ld;
+    fa.status = status;
+    e = launch_detect_quantize_compact(fa, stream);
+    if (e != cudaSuccess) return cuda_fail("detect_quantize_compact_kernel launch", e);
+  }
   if (ev && cudaEventRecord(ev[1], stream) != cudaSuccess) return I8MM_ERR_CUDA;
-  // 4. GEMM
+  if (!(stages & 2)) return I8MM_OK;
+  // 3. GEMM
   GemmArgs g{};
   g.Xq = Xq;
   g.Wq = Wq;
   g.X_O = XO;
   g.W_O = WO;
+  g.X = Xh;
+  g.W = Wh;
+  g.col_idx = idx;
   g.ld = L.l.panel_ld;
   g.x_scale = xs;
   g.w_scale = w_scale;
@@ -271,7 +292,8 @@ int mixed_matmul_impl(const void* X, const int8_t* Wq, const float* w_scale, con
   g.N = N;
   g.K = K;
   g.status = status;
-  if ((e = launch_gemm_mixed(g, stream)) != cudaSuccess) return I8MM_ERR_CUDA;
+  const cudaError_t ge = launch_gemm_mixed(g, stream);
+  if (ge != cudaSuccess) return cuda_fail("GEMM kernel launch", ge);
   if (ev && cudaEventRecord(ev[2], stream) != cudaSuccess) return I8MM_ERR_CUDA;
   return I8MM_OK;
 }
@@ -285,6 +307,14 @@ int int8_mixed_matmul(const void* X, const int8_t* Wq, const float* w_scale, con
                       size_t workspace_bytes, i8mm_stream_t stream) {
   return mixed_matmul_impl(X, Wq, w_scale, W_fp16, M, N, K, threshold, Y, workspace,
                            workspace_bytes, stream, nullptr);
+}
+
+int int8_mixed_matmul_stage(int stage, const void* X, const int8_t* Wq, const float* w_scale,
+                            const void* W_fp16, int M, int N, int K, float threshold, void* Y,
+                            void* workspace, size_t workspace_bytes, i8mm_stream_t stream) {
+  if (stage != 1 && stage != 2) return I8MM_ERR_INVALID_ARG;
+  return mixed_matmul_impl(X, Wq, w_scale, W_fp16, M, N, K, threshold, Y, workspace,
+                           workspace_bytes, stream, nullptr, stage);
 }
 
 int int8_mixed_matmul_profiled(const void* X, const int8_t* Wq, const float* w_scale,

@@ -16,12 +16,13 @@
 //               continuously across tiles
 //   warp 1      owns the 512-column TMEM allocation; one lane issues the MMAs
 //               (4 x K=32 per K-block) and commits
-//   warps 2-9   epilogue: tcgen05.ld (thread = output row, two warps per TMEM
+//   warps 2-17  epilogue: tcgen05.ld (thread = output row, four warps per TMEM
 //               lane quarter splitting the 256 columns), dequantise, add the
 //               outlier product, round to fp16, store
 // Two ways of forming C_out, chosen on the device from the outlier count:
-//   count <= kCcMax  on CUDA cores in the epilogue (fp16 products are exact in
-//                    fp32; <= 16 FMAs per output). The two 256-column INT32
+//   count <= kCcMax  on CUDA cores in the epilogue from the 16-column compacted
+//                    panels (fp16 products are exact in fp32; <= 16 FMAs per
+//                    output). The two 256-column INT32
 //                    accumulators are double-buffered, so the epilogue of one
 //                    tile overlaps the MMAs of the next.
 //   count >  kCcMax  on the tensor cores: the compacted fp16 panels X_O, W_O are
@@ -40,6 +41,7 @@
 #include <cstdint>
 #include <cstring>
 #include <mutex>
+#include <type_traits>
 
 #include "kernels.cuh"
 #include "ptx.cuh"
@@ -48,26 +50,39 @@ namespace i8mm {
 
 namespace {
 
-constexpr int BM = 128;              // rows of the output tile (TMEM lanes)
+constexpr int BM = 128;              // output rows per CTA (TMEM lanes)
 constexpr int BN = 256;              // columns of the output tile
 constexpr int KB_I8 = 128;           // int8 columns per K-block (128 bytes)
 constexpr int KB_F16 = 64;           // fp16 columns per panel block (128 bytes)
-constexpr int STAGES = 4;
-constexpr int kEpiWarps = 8;
+constexpr int kEpiWarps = 16;          // four per TMEM lane quarter, 64 columns each
 constexpr int kThreads = 64 + 32 * kEpiWarps;
-constexpr int kCcMax = 16;           // outlier counts handled on CUDA cores
+constexpr int kCcMax = kCcMaxOutliers;   // outlier counts handled on CUDA cores
 constexpr int kStatusTimeout = -5;   // == I8MM_ERR_TIMEOUT
-
-constexpr int A_BYTES = BM * 128;
-constexpr int B_BYTES = BN * 128;
-constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-constexpr int RING_BYTES = STAGES * STAGE_BYTES;
-constexpr int WO_BYTES = kCcMax * BN * 4;   // W_O tile, fp32, [j][column]
-constexpr int SW_BYTES = BN * 4;            // w_scale tile
-constexpr int BAR_OFF = RING_BYTES + WO_BYTES + SW_BYTES;
-constexpr int BAR_BYTES = (2 * STAGES + 4) * 8 + 16;
-constexpr int SMEM_BYTES = 1024 /*alignment slack*/ + BAR_OFF + BAR_BYTES;
 constexpr uint32_t TMEM_COLS = 512;
+
+// PAIR: a CTA pair (cta_group::2) computes a 256 x 256 tile; each CTA stages its
+// 128 rows of A and 128 of the 256 rows of B, so a stage is 32 KB; five fit next
+// to the output staging buffers. Single CTA: 128 x 256 tiles, 48 KB stages, three.
+// Output staging: two 1 KB buffers per epilogue warp (32 rows x 16 fp16 columns,
+// 32-byte swizzle) drained by TMA stores.
+constexpr int STG_BUF_BYTES = 32 * 16 * 2;
+
+template <bool PAIR>
+struct Cfg {
+  static constexpr int TILE_M = PAIR ? 2 * BM : BM;
+  static constexpr int B_ROWS = PAIR ? BN / 2 : BN;
+  static constexpr int STAGES = PAIR ? 5 : 3;
+  static constexpr int A_BYTES = BM * 128;
+  static constexpr int B_BYTES = B_ROWS * 128;
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int RING_BYTES = STAGES * STAGE_BYTES;
+  static constexpr int STG_BYTES = kEpiWarps * 2 * STG_BUF_BYTES;
+  static constexpr int WO_BYTES = kCcMax * BN * 2;   // W outlier tile, fp16, [j][column]
+  static constexpr int SW_BYTES = BN * 4;            // w_scale tile
+  static constexpr int BAR_OFF = RING_BYTES + STG_BYTES + WO_BYTES + SW_BYTES;
+  static constexpr int BAR_BYTES = (2 * STAGES + 4) * 8 + 16;
+  static constexpr int SMEM_BYTES = 1024 /*alignment slack*/ + BAR_OFF + BAR_BYTES;
+};
 
 __device__ __forceinline__ void record_error(int32_t* status, int code) {
   if (status) atomicCAS(status, 0, code);
@@ -77,24 +92,30 @@ __device__ __forceinline__ void epi_sync() {
   asm volatile("bar.sync 1, %0;" ::"n"(32 * kEpiWarps) : "memory");
 }
 
-template <bool OUT_I32>
+// 18 warps: two of the four SM sub-partitions hold five warps, so the register
+// budget is 96 per thread (16K registers per sub-partition).
+template <bool OUT_I32, bool PAIR>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_i8_persistent_kernel(const __grid_constant__ CUtensorMap tmA,
                               const __grid_constant__ CUtensorMap tmB,
                               const __grid_constant__ CUtensorMap tmXO,
                               const __grid_constant__ CUtensorMap tmWO,
+                              const __grid_constant__ CUtensorMap tmY, int y_tma,
                               const float* __restrict__ x_scale,
                               const float* __restrict__ w_scale,
                               const int32_t* __restrict__ n_outliers,
                               const __half* __restrict__ X_O, const __half* __restrict__ W_O,
                               int ld, void* __restrict__ out, int M, int N, int K,
                               int32_t* status) {
+  using C = Cfg<PAIR>;
+  constexpr int STAGES = C::STAGES;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  float* wo_s = reinterpret_cast<float*>(smem + RING_BYTES);            // [kCcMax][BN]
-  float* sw_s = reinterpret_cast<float*>(smem + RING_BYTES + WO_BYTES);  // [BN]
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + BAR_OFF);
+  uint8_t* stg = smem + C::RING_BYTES;                                          // staging
+  __half* wo_s = reinterpret_cast<__half*>(stg + C::STG_BYTES);                // [kCcMax][BN]
+  float* sw_s = reinterpret_cast<float*>(stg + C::STG_BYTES + C::WO_BYTES);     // [BN]
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::BAR_OFF);
   uint64_t* empty = full + STAGES;
   uint64_t* acc_full = empty + STAGES;   // [2]
   uint64_t* acc_empty = acc_full + 2;    // [2]
@@ -103,7 +124,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int m_tiles = (M + BM - 1) / BM;
+  // A pair walks the tiles as one unit; rank 0 of the pair issues the MMAs.
+  const uint32_t rank = PAIR ? cluster_ctarank() : 0u;
+  const int unit = PAIR ? static_cast<int>(blockIdx.x >> 1) : static_cast<int>(blockIdx.x);
+  const int units = PAIR ? static_cast<int>(gridDim.x >> 1) : static_cast<int>(gridDim.x);
+  const int m_tiles = (M + C::TILE_M - 1) / C::TILE_M;
   const int n_tiles = (N + BN - 1) / BN;
   const int num_tiles = m_tiles * n_tiles;
 
@@ -114,7 +139,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&acc_full[b], 1);
-      mbar_init(&acc_empty[b], kEpiWarps);
+      mbar_init(&acc_empty[b], (PAIR ? 2 : 1) * kEpiWarps);   // epilogue warps of the pair
     }
     *abort_flag = 0;
     fence_mbarrier_init();
@@ -126,11 +151,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   }
   if (warp == 1) {
-    tmem_alloc(tmem_slot, TMEM_COLS);
-    tmem_relinquish();
+    if constexpr (PAIR) {
+      tmem_alloc_pair(tmem_slot, TMEM_COLS);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(tmem_slot, TMEM_COLS);
+      tmem_relinquish();
+    }
   }
   tc_fence_before();
   __syncthreads();
+  if constexpr (PAIR) cluster_sync();   // barriers and TMEM of both CTAs are ready
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
@@ -144,9 +175,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       // ------------------------------------------------------------ producer
       uint32_t g = 0;
-      for (int tile = blockIdx.x; tile < num_tiles && !*abort_flag; tile += gridDim.x) {
-        const int m0 = (tile % m_tiles) * BM;
-        const int n0 = (tile / m_tiles) * BN;
+      for (int tile = unit; tile < num_tiles && !*abort_flag; tile += units) {
+        const int m0 = (tile % m_tiles) * C::TILE_M + static_cast<int>(rank) * BM;
+        const int n0 = (tile / m_tiles) * BN + static_cast<int>(rank) * C::B_ROWS;
         for (int it = 0; it < iters; ++it, ++g) {
           const int s = g % STAGES;
           const uint32_t ph = (g / STAGES) & 1;
@@ -155,28 +186,35 @@ __global__ void __launch_bounds__(kThreads, 1)
             *abort_flag = 1;
             break;
           }
-          uint8_t* a = smem + s * STAGE_BYTES;
-          uint8_t* b = a + A_BYTES;
-          mbar_arrive_expect_tx(&full[s], STAGE_BYTES);
-          if (it < nk) {
-            tma_load_2d(a, &tmA, &full[s], it * KB_I8, m0);
-            tma_load_2d(b, &tmB, &full[s], it * KB_I8, n0);
+          uint8_t* a = smem + s * C::STAGE_BYTES;
+          uint8_t* b = a + C::A_BYTES;
+          const bool panel = it >= nk;
+          const CUtensorMap* ta = panel ? &tmXO : &tmA;
+          const CUtensorMap* tb = panel ? &tmWO : &tmB;
+          const int x = panel ? (it - nk) * KB_F16 : it * KB_I8;
+          if constexpr (PAIR) {
+            // Both CTAs' loads complete on the full barrier of rank 0, which waits
+            // for the bytes of the whole pair.
+            if (rank == 0) mbar_arrive_expect_tx(&full[s], 2 * C::STAGE_BYTES);
+            const uint32_t bar0 = cluster_addr(&full[s], 0);
+            tma_load_2d_pair(a, ta, bar0, x, m0);
+            tma_load_2d_pair(b, tb, bar0, x, n0);
           } else {
-            const int p = it - nk;
-            tma_load_2d(a, &tmXO, &full[s], p * KB_F16, m0);
-            tma_load_2d(b, &tmWO, &full[s], p * KB_F16, n0);
+            mbar_arrive_expect_tx(&full[s], C::STAGE_BYTES);
+            tma_load_2d(a, ta, &full[s], x, m0);
+            tma_load_2d(b, tb, &full[s], x, n0);
           }
         }
       }
     }
   } else if (warp == 1) {
-    if (lane == 0) {
+    if (lane == 0 && rank == 0) {
       // ------------------------------------------------------------ MMA issuer
-      constexpr uint32_t idesc_i8 = make_idesc(2 /*s32*/, 1 /*signed*/, BM, BN);
-      constexpr uint32_t idesc_f16 = make_idesc(1 /*f32*/, 0 /*fp16*/, BM, BN);
+      constexpr uint32_t idesc_i8 = make_idesc(2 /*s32*/, 1 /*signed*/, C::TILE_M, BN);
+      constexpr uint32_t idesc_f16 = make_idesc(1 /*f32*/, 0 /*fp16*/, C::TILE_M, BN);
       uint32_t g = 0;
       int local = 0;
-      for (int tile = blockIdx.x; tile < num_tiles && !*abort_flag; tile += gridDim.x, ++local) {
+      for (int tile = unit; tile < num_tiles && !*abort_flag; tile += units, ++local) {
         const int buf = tc_out ? 0 : (local & 1);
         const uint32_t aph = tc_out ? (local & 1) : ((local >> 1) & 1);
         if (!mbar_wait(&acc_empty[buf], aph ^ 1)) {
@@ -198,154 +236,266 @@ __global__ void __launch_bounds__(kThreads, 1)
             break;
           }
           tc_fence_after();
-          const uint32_t a = smem_addr(smem + s * STAGE_BYTES);
-          const uint32_t b = a + A_BYTES;
+          const uint32_t a = smem_addr(smem + s * C::STAGE_BYTES);
+          const uint32_t b = a + C::A_BYTES;
           if (it < nk) {
 #pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
-              mma_i8(d_i32, sw128_kmajor_desc(a + 32 * kk), sw128_kmajor_desc(b + 32 * kk),
-                     idesc_i8, (it | kk) != 0);
+            for (int kk = 0; kk < 4; ++kk) {
+              const uint64_t ad = sw128_kmajor_desc(a + 32 * kk);
+              const uint64_t bd = sw128_kmajor_desc(b + 32 * kk);
+              if constexpr (PAIR)
+                mma_i8_pair(d_i32, ad, bd, idesc_i8, (it | kk) != 0);
+              else
+                mma_i8(d_i32, ad, bd, idesc_i8, (it | kk) != 0);
+            }
           } else {
             const int p = it - nk;
             const int steps = min(4, (count - p * KB_F16 + 15) / 16);
-            for (int kk = 0; kk < steps; ++kk)
-              mma_f16(d_f32, sw128_kmajor_desc(a + 32 * kk), sw128_kmajor_desc(b + 32 * kk),
-                      idesc_f16, (p | kk) != 0);
+            for (int kk = 0; kk < steps; ++kk) {
+              const uint64_t ad = sw128_kmajor_desc(a + 32 * kk);
+              const uint64_t bd = sw128_kmajor_desc(b + 32 * kk);
+              if constexpr (PAIR)
+                mma_f16_pair(d_f32, ad, bd, idesc_f16, (p | kk) != 0);
+              else
+                mma_f16(d_f32, ad, bd, idesc_f16, (p | kk) != 0);
+            }
           }
-          mma_commit(&empty[s]);
+          if constexpr (PAIR)
+            mma_commit_pair(&empty[s], 0x3);
+          else
+            mma_commit(&empty[s]);
         }
-        mma_commit(&acc_full[buf]);
+        if constexpr (PAIR)
+          mma_commit_pair(&acc_full[buf], 0x3);
+        else
+          mma_commit(&acc_full[buf]);
         if (!ok) break;
       }
     }
   } else {
     // -------------------------------------------------------------- epilogue
-    const int q = warp & 3;                 // TMEM lane quarter this warp may read
-    const int half = (warp - 2) >> 2;       // which 128 of the 256 columns
-    const int et = threadIdx.x - 64;        // 0..255
+    // Warp w reads TMEM lane quarter (w % 4) and the 64 columns [part*64, part*64+64)
+    // of the tile. The per-tile operands of the epilogue (w_scale of the tile's
+    // columns, the outlier panel rows) are fetched one tile ahead into registers.
+    const int q = warp & 3;
+    const int part = (warp - 2) >> 2;
+    const int et = threadIdx.x - 64;        // 0 .. 32*kEpiWarps-1
     const bool cc_out = !OUT_I32 && !tc_out && count > 0;
     const bool vec_ok = (N % 8) == 0;
+    const int col_lo = part * (BN / 4);
+
+    float sw_next = 0.0f;
+    uint4 wo_next[2] = {make_uint4(0, 0, 0, 0), make_uint4(0, 0, 0, 0)};
+    uint4 xo_next[2] = {make_uint4(0, 0, 0, 0), make_uint4(0, 0, 0, 0)};
+    float rs_next = 0.0f;
+    auto prefetch = [&](int tile) {
+      if (OUT_I32 || tile >= num_tiles) return;
+      const int m0 = (tile % m_tiles) * C::TILE_M + static_cast<int>(rank) * BM;
+      const int n0 = (tile / m_tiles) * BN;
+      const int row = m0 + q * 32 + lane;
+      rs_next = (row < M) ? x_scale[row] * (1.0f / 16129.0f) : 0.0f;
+      if (et < BN) {
+        const int n = n0 + et;
+        sw_next = (n < N) ? w_scale[n] : 0.0f;
+        if (cc_out && n < N) {
+          const uint4* src = reinterpret_cast<const uint4*>(W_O + static_cast<size_t>(n) * ld);
+          wo_next[0] = src[0];
+          wo_next[1] = src[1];
+        } else {
+          wo_next[0] = wo_next[1] = make_uint4(0, 0, 0, 0);
+        }
+      }
+      if (cc_out && row < M) {
+        const uint4* src = reinterpret_cast<const uint4*>(X_O + static_cast<size_t>(row) * ld);
+        xo_next[0] = src[0];
+        xo_next[1] = src[1];
+      } else {
+        xo_next[0] = xo_next[1] = make_uint4(0, 0, 0, 0);
+      }
+    };
+    prefetch(unit);
+
     int local = 0;
-    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++local) {
-      const int m0 = (tile % m_tiles) * BM;
+    uint32_t sc = 0;   // chunks stored by this warp (selects the staging buffer)
+    for (int tile = unit; tile < num_tiles; tile += units, ++local) {
+      const int m0 = (tile % m_tiles) * C::TILE_M + static_cast<int>(rank) * BM;
       const int n0 = (tile / m_tiles) * BN;
       const int buf = tc_out ? 0 : (local & 1);
       const uint32_t aph = tc_out ? (local & 1) : ((local >> 1) & 1);
       const int row = m0 + q * 32 + lane;
 
-      // Per-tile column data (w_scale, W_O tile as fp32) and this row's X_O values.
+      // Stage this tile's column data in shared memory; keep the row data in registers.
+      __half2 xo2[kCcMax / 2];
+      const float rs = rs_next;
       if (!OUT_I32) {
-        const int n = n0 + et;
-        sw_s[et] = (n < N) ? w_scale[n] : 0.0f;
-        if (cc_out) {
-          for (int j = 0; j < kCcMax; ++j)
-            wo_s[j * BN + et] =
-                (n < N && j < count) ? __half2float(W_O[static_cast<size_t>(n) * ld + j]) : 0.0f;
-        }
-      }
-      float xo[kCcMax];
-      float rs = 0.0f;
-      if (!OUT_I32) {
-        if (row < M) rs = x_scale[row] * (1.0f / 16129.0f);
+        if (et < BN) {
+          sw_s[et] = sw_next;
+          if (cc_out) {
+            const __half* h = reinterpret_cast<const __half*>(wo_next);
 #pragma unroll
-        for (int j = 0; j < kCcMax; ++j)
-          xo[j] = (cc_out && row < M && j < count)
-                      ? __half2float(X_O[static_cast<size_t>(row) * ld + j])
-                      : 0.0f;
+            for (int j = 0; j < kCcMax; ++j) wo_s[j * BN + et] = h[j];
+          }
+        }
+        const __half2* h2 = reinterpret_cast<const __half2*>(xo_next);
+#pragma unroll
+        for (int j = 0; j < kCcMax / 2; ++j) xo2[j] = h2[j];
       }
       epi_sync();
+      prefetch(tile + units);
 
-      const bool ok = mbar_wait(&acc_full[buf], aph);
+      // Warp-uniform, so that a timed-out wait can never split the warp before
+      // the warp-collective TMEM loads below.
+      const bool ok = __all_sync(0xffffffffu, mbar_wait(&acc_full[buf], aph));
       if (!ok) {
         record_error(status, kStatusTimeout);
         *abort_flag = 1;
       }
       tc_fence_after();
       const uint32_t lane_base = tmem + (static_cast<uint32_t>(q * 32) << 16);
+      // The chunk loop is instantiated separately for the two outlier modes so that
+      // each keeps only its own registers live.
+      auto chunks = [&](auto tc_tag) {
+        constexpr bool TC = decltype(tc_tag)::value;
 #pragma unroll 1
-      for (int c = half * 128; c < half * 128 + 128 && ok; c += 32) {
-        __syncwarp();
-        uint32_t acc[32];
-        uint32_t oacc[32];
-        tmem_ld_32x32b_x32(lane_base + buf * BN + c, acc);
-        if (tc_out) tmem_ld_32x32b_x32(lane_base + BN + c, oacc);
-        tmem_ld_wait();
-        const int col0 = n0 + c;
-        if (row < M && col0 < N) {
-          if constexpr (OUT_I32) {
-            int32_t* orow = reinterpret_cast<int32_t*>(out) + static_cast<size_t>(row) * N;
-            if (vec_ok && col0 + 32 <= N) {
+        for (int c = col_lo; c < col_lo + BN / 4 && ok; c += 16, ++sc) {
+          if (!OUT_I32 && y_tma) {
+            // The staging buffer of this chunk was last drained two stores ago.
+            if (lane == 0) bulk_wait_group_read<1>();
+          }
+          __syncwarp();
+          // tcgen05.ld is warp-collective: issued by all 32 lanes, outside any
+          // per-row condition (tc_out and ok are uniform across the warp).
+          uint32_t acc[16];
+          uint32_t oacc[TC ? 16 : 1];
+          tmem_ld_32x32b_x16(lane_base + buf * BN + c, acc);
+          if constexpr (TC) tmem_ld_32x32b_x16(lane_base + BN + c, oacc);
+          tmem_ld_wait();
+          const int col0 = n0 + c;
+          if (row < M && col0 < N) {
+            if constexpr (OUT_I32) {
+              int32_t* orow = reinterpret_cast<int32_t*>(out) + static_cast<size_t>(row) * N;
+              if (vec_ok && col0 + 16 <= N) {
 #pragma unroll
-              for (int j = 0; j < 32; j += 4)
-                *reinterpret_cast<uint4*>(orow + col0 + j) =
-                    make_uint4(acc[j], acc[j + 1], acc[j + 2], acc[j + 3]);
+                for (int j = 0; j < 16; j += 4)
+                  *reinterpret_cast<uint4*>(orow + col0 + j) =
+                      make_uint4(acc[j], acc[j + 1], acc[j + 2], acc[j + 3]);
+              } else {
+#pragma unroll
+                for (int j = 0; j < 16; ++j)
+                  if (col0 + j < N) orow[col0 + j] = static_cast<int32_t>(acc[j]);
+              }
             } else {
+              float y[16];
+              const float4* sw4 = reinterpret_cast<const float4*>(sw_s + c);
 #pragma unroll
-              for (int j = 0; j < 32; ++j)
-                if (col0 + j < N) orow[col0 + j] = static_cast<int32_t>(acc[j]);
-            }
-          } else {
-            float y[32];
+              for (int j = 0; j < 4; ++j) {
+                const float4 w = sw4[j];
+                y[4 * j + 0] = static_cast<float>(static_cast<int32_t>(acc[4 * j + 0])) * (rs * w.x);
+                y[4 * j + 1] = static_cast<float>(static_cast<int32_t>(acc[4 * j + 1])) * (rs * w.y);
+                y[4 * j + 2] = static_cast<float>(static_cast<int32_t>(acc[4 * j + 2])) * (rs * w.z);
+                y[4 * j + 3] = static_cast<float>(static_cast<int32_t>(acc[4 * j + 3])) * (rs * w.w);
+              }
+              if constexpr (TC) {
 #pragma unroll
-            for (int j = 0; j < 32; ++j)
-              y[j] = static_cast<float>(static_cast<int32_t>(acc[j])) * (rs * sw_s[c + j]);
-            if (tc_out) {
+                for (int j = 0; j < 16; ++j) y[j] += __uint_as_float(oacc[j]);
+              } else if (cc_out) {
+                float o[16];
 #pragma unroll
-              for (int j = 0; j < 32; ++j) y[j] += __uint_as_float(oacc[j]);
-            } else if (cc_out) {
-              float o[32];
+                for (int j = 0; j < 16; ++j) o[j] = 0.0f;
 #pragma unroll
-              for (int j = 0; j < 32; ++j) o[j] = 0.0f;
+                for (int t = 0; t < kCcMax; ++t) {
+                  if (t < count) {
+                    const float xt = (t & 1) ? __high2float(xo2[t >> 1]) : __low2float(xo2[t >> 1]);
+                    const uint4* w8 = reinterpret_cast<const uint4*>(wo_s + t * BN + c);
 #pragma unroll
-              for (int t = 0; t < kCcMax; ++t) {
-                if (t < count) {
-                  const float4* w4 = reinterpret_cast<const float4*>(wo_s + t * BN + c);
+                    for (int j = 0; j < 2; ++j) {
+                      const uint4 wv = w8[j];
+                      const __half2* w2 = reinterpret_cast<const __half2*>(&wv);
 #pragma unroll
-                  for (int j = 0; j < 8; ++j) {
-                    const float4 w = w4[j];
-                    o[4 * j + 0] = fmaf(xo[t], w.x, o[4 * j + 0]);
-                    o[4 * j + 1] = fmaf(xo[t], w.y, o[4 * j + 1]);
-                    o[4 * j + 2] = fmaf(xo[t], w.z, o[4 * j + 2]);
-                    o[4 * j + 3] = fmaf(xo[t], w.w, o[4 * j + 3]);
+                      for (int i = 0; i < 4; ++i) {
+                        const float2 w = __half22float2(w2[i]);
+                        o[8 * j + 2 * i] = fmaf(xt, w.x, o[8 * j + 2 * i]);
+                        o[8 * j + 2 * i + 1] = fmaf(xt, w.y, o[8 * j + 2 * i + 1]);
+                      }
+                    }
                   }
                 }
-              }
 #pragma unroll
-              for (int j = 0; j < 32; ++j) y[j] += o[j];
+                for (int j = 0; j < 16; ++j) y[j] += o[j];
+              }
+              __half* orow = reinterpret_cast<__half*>(out) + static_cast<size_t>(row) * N;
+              if (y_tma) {
+                // Row `lane` of this warp's 32 x 16 staging block, 16-byte chunks
+                // XOR-swizzled by bit 2 of the row (the TMA 32-byte swizzle).
+                uint8_t* buf_row = stg + ((warp - 2) * 2 + (sc & 1)) * STG_BUF_BYTES + lane * 32;
+                const int sw = (lane >> 2) & 1;
+#pragma unroll
+                for (int j = 0; j < 16; j += 8) {
+                  uint4 v;
+                  __half2* h = reinterpret_cast<__half2*>(&v);
+                  h[0] = __floats2half2_rn(y[j], y[j + 1]);
+                  h[1] = __floats2half2_rn(y[j + 2], y[j + 3]);
+                  h[2] = __floats2half2_rn(y[j + 4], y[j + 5]);
+                  h[3] = __floats2half2_rn(y[j + 6], y[j + 7]);
+                  *reinterpret_cast<uint4*>(buf_row + (((j >> 3) ^ sw) << 4)) = v;
+                }
+              } else if (vec_ok && col0 + 16 <= N) {
+#pragma unroll
+                for (int j = 0; j < 16; j += 8) {
+                  uint4 v;
+                  __half2* h = reinterpret_cast<__half2*>(&v);
+                  h[0] = __floats2half2_rn(y[j], y[j + 1]);
+                  h[1] = __floats2half2_rn(y[j + 2], y[j + 3]);
+                  h[2] = __floats2half2_rn(y[j + 4], y[j + 5]);
+                  h[3] = __floats2half2_rn(y[j + 6], y[j + 7]);
+                  *reinterpret_cast<uint4*>(orow + col0 + j) = v;
+                }
+              } else {
+#pragma unroll
+                for (int j = 0; j < 16; ++j)
+                  if (col0 + j < N) orow[col0 + j] = __float2half_rn(y[j]);
+              }
             }
-            __half* orow = reinterpret_cast<__half*>(out) + static_cast<size_t>(row) * N;
-            if (vec_ok && col0 + 32 <= N) {
-#pragma unroll
-              for (int j = 0; j < 32; j += 8) {
-                uint4 v;
-                __half2* h = reinterpret_cast<__half2*>(&v);
-                h[0] = __floats2half2_rn(y[j], y[j + 1]);
-                h[1] = __floats2half2_rn(y[j + 2], y[j + 3]);
-                h[2] = __floats2half2_rn(y[j + 4], y[j + 5]);
-                h[3] = __floats2half2_rn(y[j + 6], y[j + 7]);
-                *reinterpret_cast<uint4*>(orow + col0 + j) = v;
-              }
-            } else {
-#pragma unroll
-              for (int j = 0; j < 32; ++j)
-                if (col0 + j < N) orow[col0 + j] = __float2half_rn(y[j]);
+          }
+          if (!OUT_I32 && y_tma) {
+            // Rows >= M are staged too (as anything) and clipped by the TMA store.
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0 && col0 < N) {
+              tma_store_2d(&tmY, stg + ((warp - 2) * 2 + (sc & 1)) * STG_BUF_BYTES, col0,
+                           m0 + q * 32);
+              bulk_commit_group();
             }
           }
         }
-      }
+      };
+      if (tc_out)
+        chunks(std::true_type{});
+      else
+        chunks(std::false_type{});
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&acc_empty[buf]);
+      if (lane == 0) {
+        if constexpr (PAIR)
+          mbar_arrive_cluster(cluster_addr(&acc_empty[buf], 0));
+        else
+          mbar_arrive(&acc_empty[buf]);
+      }
       epi_sync();   // the tile's sw_s / wo_s are no longer read
       if (!ok || *abort_flag) break;
     }
+    if (!OUT_I32 && y_tma && lane == 0) bulk_wait_group_all();
   }
 
   tc_fence_before();
   __syncthreads();
+  if constexpr (PAIR) cluster_sync();   // the peer may still read our shared memory
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, TMEM_COLS);
+    if constexpr (PAIR)
+      tmem_dealloc_pair(tmem, TMEM_COLS);
+    else
+      tmem_dealloc(tmem, TMEM_COLS);
   }
 }
 
@@ -364,68 +514,100 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-// Row-major [rows][cols] matrix, box of box_rows x (128 bytes), 128-byte swizzle.
+// Row-major [rows][cols] matrix, box of box_rows x box_bytes (one swizzle span).
 bool make_tmap(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int elem_bytes,
-               uint64_t cols, uint64_t rows, uint32_t box_rows) {
+               uint64_t cols, uint64_t rows, uint32_t box_rows, uint32_t box_bytes = 128,
+               CUtensorMapSwizzle swz = CU_TENSOR_MAP_SWIZZLE_128B) {
   auto fn = encode_fn();
   if (!fn) return false;
   const cuuint64_t dims[2] = {cols, rows};
   const cuuint64_t strides[1] = {cols * static_cast<uint64_t>(elem_bytes)};
-  const cuuint32_t box[2] = {static_cast<cuuint32_t>(128 / elem_bytes), box_rows};
+  const cuuint32_t box[2] = {static_cast<cuuint32_t>(box_bytes / elem_bytes), box_rows};
   const cuuint32_t estr[2] = {1, 1};
   return fn(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-            CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <bool OUT_I32>
+int sm_count(int dev) {
+  static int cached[64] = {};
+  if (dev >= 0 && dev < 64 && cached[dev]) return cached[dev];
+  int n = 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n < 2) n = 2;
+  if (dev >= 0 && dev < 64) cached[dev] = n;
+  return n;
+}
+
+template <bool OUT_I32, bool PAIR>
 cudaError_t launch(const GemmArgs& a, cudaStream_t s) {
-  CUtensorMap maps[4];
+  using C = Cfg<PAIR>;
+  CUtensorMap maps[5];
   std::memset(maps, 0, sizeof(maps));
   if (!make_tmap(&maps[0], a.Xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.K, a.M, BM) ||
-      !make_tmap(&maps[1], a.Wq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.K, a.N, BN))
+      !make_tmap(&maps[1], a.Wq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.K, a.N, C::B_ROWS))
     return cudaErrorInvalidValue;
   if (!OUT_I32 && a.X_O && a.W_O) {
     if (!make_tmap(&maps[2], a.X_O, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, a.ld, a.M, BM) ||
-        !make_tmap(&maps[3], a.W_O, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, a.ld, a.N, BN))
+        !make_tmap(&maps[3], a.W_O, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, a.ld, a.N, C::B_ROWS))
       return cudaErrorInvalidValue;
   } else {
     maps[2] = maps[0];
     maps[3] = maps[1];
   }
-  auto kern = gemm_i8_persistent_kernel<OUT_I32>;
+  // fp16 Y leaves through TMA stores when its row stride allows (N % 8 == 0).
+  int y_tma = 0;
+  if (!OUT_I32 && a.N % 8 == 0 &&
+      make_tmap(&maps[4], a.out, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, a.N, a.M, 32, 32,
+                CU_TENSOR_MAP_SWIZZLE_32B))
+    y_tma = 1;
+  if (!y_tma) maps[4] = maps[0];
+  auto kern = gemm_i8_persistent_kernel<OUT_I32, PAIR>;
   static bool attr_set[64] = {};  // per instantiation and device
-  static int sm_count[64] = {};
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev >= 64 || !attr_set[dev]) {
-    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
     if (e != cudaSuccess) return e;
-    int sms = 0;
-    e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    if (e != cudaSuccess) return e;
-    if (dev < 64) {
-      attr_set[dev] = true;
-      sm_count[dev] = sms;
-    }
+    if (dev < 64) attr_set[dev] = true;
   }
-  const int sms = dev < 64 ? sm_count[dev] : 148;
-  const int m_tiles = (a.M + BM - 1) / BM;
+  const int sms = sm_count(dev);
+  const int m_tiles = (a.M + C::TILE_M - 1) / C::TILE_M;
   const int n_tiles = (a.N + BN - 1) / BN;
   const int tiles = m_tiles * n_tiles;
-  const int grid = tiles < sms ? tiles : sms;
-  kern<<<grid, kThreads, SMEM_BYTES, s>>>(maps[0], maps[1], maps[2], maps[3], a.x_scale,
-                                          a.w_scale, OUT_I32 ? nullptr : a.n_outliers, a.X_O,
-                                          a.W_O, a.ld, a.out, a.M, a.N, a.K, a.status);
-  return cudaGetLastError();
+  const int max_units = PAIR ? sms / 2 : sms;
+  const int units = tiles < max_units ? tiles : max_units;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(PAIR ? 2 * units : units);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = C::SMEM_BYTES;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  if (PAIR) {
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+  }
+  e = cudaLaunchKernelEx(&cfg, kern, maps[0], maps[1], maps[2], maps[3], maps[4], y_tma,
+                         a.x_scale, a.w_scale,
+                         OUT_I32 ? nullptr : a.n_outliers, a.X_O, a.W_O, a.ld, a.out, a.M, a.N,
+                         a.K, a.status);
+  if (e != cudaSuccess) (void)cudaGetLastError();   // do not leave it for the next launch
+  return e;
 }
 
 }  // namespace
 
-cudaError_t launch_gemm_mixed(const GemmArgs& a, cudaStream_t s) { return launch<false>(a, s); }
+// CTA pairs whenever there is more than one 128-row block of output rows.
+cudaError_t launch_gemm_mixed(const GemmArgs& a, cudaStream_t s) {
+  return a.M > BM ? launch<false, true>(a, s) : launch<false, false>(a, s);
+}
 
-cudaError_t launch_gemm_i32(const GemmArgs& a, cudaStream_t s) { return launch<true>(a, s); }
+cudaError_t launch_gemm_i32(const GemmArgs& a, cudaStream_t s) {
+  return a.M > BM ? launch<true, true>(a, s) : launch<true, false>(a, s);
+}
 
 }  // namespace i8mm
