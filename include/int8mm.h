@@ -192,6 +192,32 @@ int int8_debug_gemm_i32(const int8_t* Xq, const int8_t* Wq, int M, int N, int K,
  */
 int int8_device_status(const void* workspace, i8mm_stream_t stream);
 
+/*
+ * int8_mixed_matmul without a workspace argument, for callers that cannot give
+ * the library device memory: for example code whose host framework owns every
+ * device allocation and offers it no allocator, or code that must not grow its
+ * device memory use while it runs. The paper has no counterpart to this entry
+ * point; it is an interface convenience of this library.
+ *   Arguments and results are those of int8_mixed_matmul.
+ *   Scratch: a fixed device array built into the library,
+ *            I8MM_NOALLOC_SCRATCH_BYTES (64 MiB), which every GPU that loads
+ *            the library holds until the process exits. Nothing is allocated
+ *            or freed by the call.
+ *   Limit:   problems with int8_mixed_matmul_workspace_size(M, N, K) larger
+ *            than I8MM_NOALLOC_SCRATCH_BYTES return I8MM_ERR_WORKSPACE.
+ *   Set-up:  the first call on a device looks up the array's device address
+ *            (with that device current) and caches it; make that first call
+ *            before any stream capture.
+ *   Sharing: all calls on a device use the same array, which keeps the last
+ *            call's contents (each call clears the words it needs first).
+ *            Calls that can overlap on the GPU (several streams or host
+ *            threads) race on the array; the caller must serialise them.
+ */
+#define I8MM_NOALLOC_SCRATCH_BYTES ((size_t)64 << 20)
+int int8_mixed_matmul_noalloc(const void* X, const int8_t* Wq, const float* w_scale,
+                              const void* W_fp16, int M, int N, int K, float threshold,
+                              void* Y, i8mm_stream_t stream);
+
 /* Static string for a status code. */
 const char* int8_status_string(int status);
 
