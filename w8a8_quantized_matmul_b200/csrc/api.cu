@@ -245,6 +245,26 @@ int mixed_matmul_impl(const void* X, const int8_t* Wq, const float* w_scale, con
   const __half* Xh = static_cast<const __half*>(X);
   const __half* Wh = static_cast<const __half*>(W_fp16);
 
+  // Decode shapes: one clustered kernel for the whole call.
+  if (stages == 3 && !ev && decode_supported(M, K)) {
+    DecodeArgs da{};
+    da.X = Xh;
+    da.W = Wh;
+    da.Wq = Wq;
+    da.w_scale = w_scale;
+    da.Y = static_cast<__half*>(Y);
+    da.M = M;
+    da.N = N;
+    da.K = K;
+    da.threshold = threshold;
+    da.bitmap = bitmap;
+    da.n_outliers = count;
+    da.col_idx = idx;
+    da.x_scale = xs;
+    da.Xq = Xq;
+    da.status = status;
+    return cuda_fail("decode_kernel launch", launch_decode(da, stream));
+  }
   if (ev && cudaEventRecord(ev[0], stream) != cudaSuccess) return I8MM_ERR_CUDA;
   if (stages & 1) {
     // 1. count, status, barrier counter and bitmap are contiguous: one memset.

@@ -602,6 +602,12 @@ cudaError_t launch(const GemmArgs& a, cudaStream_t s) {
 }  // namespace
 
 // CTA pairs whenever there is more than one 128-row block of output rows.
+bool make_tmap_2d(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int elem_bytes,
+                  uint64_t cols, uint64_t rows, uint32_t box_rows, uint32_t box_bytes,
+                  CUtensorMapSwizzle swz) {
+  return make_tmap(m, base, dt, elem_bytes, cols, rows, box_rows, box_bytes, swz);
+}
+
 cudaError_t launch_gemm_mixed(const GemmArgs& a, cudaStream_t s) {
   return a.M > BM ? launch<false, true>(a, s) : launch<false, false>(a, s);
 }

@@ -2,6 +2,7 @@
 // and the C-ABI layer of libint8mm.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
@@ -77,5 +78,36 @@ struct GemmArgs {
 
 cudaError_t launch_gemm_mixed(const GemmArgs& a, cudaStream_t s);
 cudaError_t launch_gemm_i32(const GemmArgs& a, cudaStream_t s);
+
+// Row-major [rows][cols] tensor map with a box of box_rows x box_bytes (one
+// swizzle span wide); defined in gemm_sm100.cu.
+bool make_tmap_2d(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int elem_bytes,
+                  uint64_t cols, uint64_t rows, uint32_t box_rows, uint32_t box_bytes,
+                  CUtensorMapSwizzle swz);
+inline bool make_tmap_sw128(CUtensorMap* m, const void* base, CUtensorMapDataType dt,
+                            int elem_bytes, uint64_t cols, uint64_t rows, uint32_t box_rows) {
+  return make_tmap_2d(m, base, dt, elem_bytes, cols, rows, box_rows, 128,
+                      CU_TENSOR_MAP_SWIZZLE_128B);
+}
+
+// Decode-shape path (M <= 16): one clustered kernel (decode.cu).
+struct DecodeArgs {
+  const __half* X;        // [M][K]
+  const __half* W;        // [N][K] fp16 weight (outlier columns are read)
+  const int8_t* Wq;       // [N][K]
+  const float* w_scale;   // [N]
+  __half* Y;              // [M][N]
+  int M, N, K;
+  float threshold;
+  uint32_t* bitmap;       // workspace outputs (written by the first cluster)
+  int32_t* n_outliers;
+  int32_t* col_idx;
+  float* x_scale;
+  int8_t* Xq;
+  int32_t* status;
+};
+
+bool decode_supported(int M, int K);
+cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t s);
 
 }  // namespace i8mm
