@@ -210,6 +210,8 @@ DECODE_CASES = [
     (16, 512, 200, 6, math.inf),
     (16, 512, 200, 6, 0.0),        # every nonzero column is an outlier
     (12, 4096, 1000, 0, 6.0),
+    (16, 4096, 256, 64, 6.0),      # more outliers per CTA than are gathered ahead
+    (5, 1040, 136, 3, 6.0),        # two ranks, the last K-block 16 columns wide
 ]
 
 

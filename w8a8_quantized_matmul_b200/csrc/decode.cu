@@ -6,26 +6,35 @@
 // of the scales, FP16 product over the outlier columns, final sum); tanjunchen
 // "quantization explained part 2" section 1.2 (threshold 6.0).
 //
-// With at most 16 tokens the work is bound by reading Wq once. The grid is
-// made of clusters of S CTAs; a cluster owns 128 output features (rows of Wq)
-// and its CTAs split K, so every CTA streams a 128 x (K/S) slice of Wq:
-//   * the producer TMA-loads the whole slice at kernel start (up to 8 stages of
-//     128 x 128 bytes, no reuse), before anything else;
-//   * all threads bulk-copy the CTA's K-range of every token row of X into
-//     shared memory. Every CTA sees all tokens, so the outlier flags of its
-//     columns are exact locally; each computes per-token maxima over its
-//     non-outlier columns and the cluster exchanges them through distributed
-//     shared memory to form each token's absmax;
-//   * the CTA writes the INT8 codes of its X range straight into the 128-byte
-//     swizzled K-major layout the tensor core reads (16 token rows) and one
-//     thread issues tcgen05.mma kind::i8 with M = 128 weight rows, N = 16 tokens;
-//   * the outlier product of the CTA's own outlier columns is formed on CUDA
-//     cores (fp16 products are exact in fp32);
-//   * INT32 partials (exact, order free) and fp32 outlier partials are summed
-//     across the cluster in a fixed rank order through distributed shared
-//     memory; each CTA finishes 128/S rows and writes Y.
-// Cluster 0 also writes the intermediates the workspace documents (bitmap,
-// count, ascending outlier list, x_scale, Xq). No TMA multicast is used.
+// With at most 16 tokens the work is bound by reading Wq once; everything else
+// is arranged to finish while that stream is in flight. The grid is made of
+// clusters of S CTAs; a cluster owns 128 output features (rows of Wq) and its
+// CTAs split K, so every CTA reads a 128 x (K/S) slice of Wq (at most 8 blocks
+// of 128 x 128 bytes, all requested at kernel start).
+//
+// Warp roles (320 threads):
+//   warp 0     producer: bulk-copies the CTA's K-range of every token row of X
+//              (first, it is small and L2-resident), then TMA-loads the Wq slice
+//   warp 1     TMEM allocator and MMA issuer: tcgen05.mma kind::i8 with
+//              M = 128 weight rows, N = 16 tokens, one K-block as it lands
+//   warps 2-9  X workers, 4 columns per thread, all 16 tokens held in registers:
+//              exact outlier flags of their columns (every token is here),
+//              per-token maxima over the non-outlier columns, and after the
+//              cluster exchange of those maxima the INT8 codes, written straight
+//              into the 128-byte-swizzled K-major B operand of the MMA
+//   warps 4-7  also the epilogue: the fp32 outlier partials of the CTA's own
+//              outlier columns on CUDA cores (fp16 products are exact in fp32),
+//              the INT32 partials from TMEM, and the cross-CTA sum.
+//
+// Cross-CTA traffic uses st.async into the peer's shared memory, counted in
+// bytes on the peer's mbarrier: one 80-byte message per CTA pair with the
+// per-token maxima and the outlier count, then each CTA pushes every row's
+// 16 INT32 + 16 fp32 partials to the CTA that finishes that row, which sums the
+// S partials in rank order and writes Y. A split cluster barrier only publishes
+// the mbarrier initialisation and keeps every CTA alive until its peers have
+// issued their last store into it. Cluster 0 also writes the intermediates the
+// workspace documents (bitmap, count, ascending outlier list, x_scale, Xq).
+// No TMA multicast is used.
 #include <cuda.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
@@ -41,32 +50,43 @@ namespace i8mm {
 
 namespace {
 
-constexpr int kRows = 128;       // Wq rows (output features) per cluster
-constexpr int kKB = 128;         // int8 columns per K-block
-constexpr int kMaxBlocks = 8;    // K-blocks per CTA (all in flight at once)
-constexpr int kTok = 16;         // MMA N: tokens, zero-padded
-constexpr int kThreads = 256;
-constexpr int kWarps = kThreads / 32;
+constexpr int kRows = 128;                    // Wq rows (output features) per cluster = MMA M
+constexpr int kKB = 128;                      // int8 columns per K-block (one swizzle row)
+constexpr int kMaxBlocks = 8;                 // K-blocks per CTA, all in flight at once
+constexpr int kCols = kMaxBlocks * kKB;       // columns per CTA at most
+constexpr int kTok = 16;                      // MMA N: tokens, zero-padded
 constexpr int kMaxCluster = 8;
+constexpr int kXWarps = 8;                    // X workers: 4 columns per thread
+constexpr int kXThreads = kXWarps * 32;
+constexpr int kThreads = 64 + kXThreads;
+constexpr int kMsgWords = 20;                 // exchange message: 16 maxima, count, pad
+constexpr int kRecvRows = kRows + kMaxCluster;   // S * ceil(128 / S) <= 135
+constexpr int kWPrefetch = 8;                 // outlier weights gathered ahead per row
 constexpr int kStatusTimeout = -5;
 
+static_assert(kXThreads * 4 == kCols, "X workers cover the CTA's columns");
+
+// Named barriers (0 is __syncthreads).
+constexpr uint32_t kBarX = 1;       // the X workers
+constexpr uint32_t kBarList = 2;    // warp 2 publishes the local outlier list to warps 4-7
+constexpr uint32_t kBarEpi = 3;     // warps 4-7
+
 struct DecodeSmem {
-  static constexpr int RING = 0;                                   // [8][128][128] i8
-  static constexpr int BOP = RING + kMaxBlocks * kRows * kKB;      // [8][16][128] i8
-  static constexpr int XS = BOP + kMaxBlocks * kTok * kKB;         // [16][1024] f16
-  static constexpr int PI = XS + kTok * kMaxBlocks * kKB * 2;      // [128][16] i32
-  static constexpr int PF = PI + kRows * kTok * 4;                 // [128][16] f32
-  static constexpr int XMAX = PF + kRows * kTok * 4;               // [8 ranks][16] f32
-  static constexpr int XCNT = XMAX + kMaxCluster * kTok * 4;       // [8 ranks] i32
-  static constexpr int BITS = XCNT + kMaxCluster * 4;              // [32] u32
-  static constexpr int LIDX = BITS + 32 * 4;                       // [1024] u16
-  static constexpr int RED = LIDX + kMaxBlocks * kKB * 2;          // [8 warps][16] f32
-  static constexpr int AMAX = RED + kWarps * kTok * 4;             // [16] f32
-  static constexpr int MISC = AMAX + kTok * 4;                     // [4] i32
-  static constexpr int BARS = MISC + 16;                           // full[8], done, xbar
-  static constexpr int TSLOT = BARS + (kMaxBlocks + 2) * 8;
+  static constexpr int RING = 0;                                // [8][128][128] i8 (swizzled)
+  static constexpr int BOP = RING + kMaxBlocks * kRows * kKB;   // [8][16][128] i8 (swizzled)
+  static constexpr int XS = BOP + kMaxBlocks * kTok * kKB;      // [16][kw] f16
+  static constexpr int RECV = XS + kTok * kCols * 2;            // [kRecvRows][8][16 B]
+  static constexpr int MSG = RECV + kRecvRows * 128;            // [8 ranks][20] words
+  static constexpr int BITS = MSG + kMaxCluster * kMsgWords * 4;   // [32] u32
+  static constexpr int LIDX = BITS + 32 * 4;                    // [1024] u16
+  static constexpr int RED = LIDX + kCols * 2;                  // [8 warps][16] f32
+  static constexpr int TOK = RED + kXWarps * kTok * 4;          // amax[16], inv[16] f32
+  static constexpr int WSC = TOK + 2 * kTok * 4;                // [128] f32 w_scale of owned rows
+  static constexpr int MISC = WSC + kRows * 4;                  // lcount, prefix
+  static constexpr int BARS = MISC + 16;                        // full[8] xbar codes done xchg red
+  static constexpr int TSLOT = BARS + (kMaxBlocks + 5) * 8;
   static constexpr int TOTAL = TSLOT + 16;
-  static constexpr int BYTES = TOTAL + 1024;                       // alignment slack
+  static constexpr int BYTES = TOTAL + 1024;                    // alignment slack
 };
 
 __device__ __forceinline__ uint32_t cluster_nctarank() {
@@ -75,21 +95,9 @@ __device__ __forceinline__ uint32_t cluster_nctarank() {
   return r;
 }
 
-__device__ __forceinline__ void st_cluster_f32(uint32_t addr, float v) {
-  asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(addr), "f"(v) : "memory");
-}
-__device__ __forceinline__ void st_cluster_s32(uint32_t addr, int v) {
-  asm volatile("st.shared::cluster.s32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
-}
-__device__ __forceinline__ int ld_cluster_s32(uint32_t addr) {
-  int v;
-  asm volatile("ld.shared::cluster.s32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
-  return v;
-}
-__device__ __forceinline__ float ld_cluster_f32(uint32_t addr) {
-  float v;
-  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
-  return v;
+// Rows finished (owned) by `rank` when 128 rows are dealt out rpr at a time.
+__device__ __forceinline__ int owned_rows(int rank, int rpr) {
+  return max(0, min(rpr, kRows - rank * rpr));
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -101,18 +109,21 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* ring = sm + L::RING;
   uint8_t* bop = sm + L::BOP;
   __half* xs = reinterpret_cast<__half*>(sm + L::XS);
-  int32_t* p_i32 = reinterpret_cast<int32_t*>(sm + L::PI);
-  float* p_f32 = reinterpret_cast<float*>(sm + L::PF);
-  float* xmax = reinterpret_cast<float*>(sm + L::XMAX);
-  int32_t* xcnt = reinterpret_cast<int32_t*>(sm + L::XCNT);
+  uint8_t* recv = sm + L::RECV;
+  uint32_t* msg = reinterpret_cast<uint32_t*>(sm + L::MSG);
   uint32_t* bits = reinterpret_cast<uint32_t*>(sm + L::BITS);
   uint16_t* lidx = reinterpret_cast<uint16_t*>(sm + L::LIDX);
   float* red = reinterpret_cast<float*>(sm + L::RED);
-  float* amax = reinterpret_cast<float*>(sm + L::AMAX);
+  float* amax_s = reinterpret_cast<float*>(sm + L::TOK);
+  float* inv_s = amax_s + kTok;
+  float* wsc = reinterpret_cast<float*>(sm + L::WSC);
   int32_t* misc = reinterpret_cast<int32_t*>(sm + L::MISC);
   uint64_t* full = reinterpret_cast<uint64_t*>(sm + L::BARS);
-  uint64_t* done = full + kMaxBlocks;
-  uint64_t* xbar = done + 1;
+  uint64_t* xbar = full + kMaxBlocks;
+  uint64_t* codes_bar = xbar + 1;
+  uint64_t* done = xbar + 2;
+  uint64_t* xchg = xbar + 3;
+  uint64_t* redbar = xbar + 4;
   uint32_t* tslot = reinterpret_cast<uint32_t*>(sm + L::TSLOT);
 
   const int tid = threadIdx.x;
@@ -126,16 +137,22 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int nkb = (K + kKB - 1) / kKB;
   const int bper = (nkb + S - 1) / S;
   const int kb0 = min(nkb, rank * bper);
-  const int nb = min(nkb, kb0 + bper) - kb0;            // K-blocks of this CTA (0..8)
+  const int nb = min(nkb, kb0 + bper) - kb0;            // K-blocks of this CTA (1..8)
   const int k0 = min(K, kb0 * kKB);
-  const int k1 = min(K, (kb0 + nb) * kKB);
-  const int kw = k1 - k0;                               // columns of this CTA
+  const int kw = min(K, (kb0 + nb) * kKB) - k0;         // columns of this CTA
+  const int rpr = (kRows + S - 1) / S;                  // rows finished per rank
   const bool writer = (tile == 0);                      // cluster 0 writes intermediates
 
   if (tid == 0) {
     for (int b = 0; b < kMaxBlocks; ++b) mbar_init(&full[b], 1);
-    mbar_init(done, 1);
     mbar_init(xbar, 1);
+    mbar_init(codes_bar, kXWarps);
+    mbar_init(done, 1);
+    mbar_init(xchg, 1);
+    mbar_init(redbar, 1);
+    // The peers' stores are counted in bytes; the one local arrival is made now.
+    mbar_arrive_expect_tx(xchg, static_cast<uint32_t>(S * kMsgWords * 4));
+    mbar_arrive_expect_tx(redbar, static_cast<uint32_t>(S * owned_rows(rank, rpr) * 128));
     fence_mbarrier_init();
     tma_prefetch_desc(&tmWq);
     if (blockIdx.x == 0 && a.status) *a.status = 0;
@@ -147,253 +164,338 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  cluster_sync();   // every CTA's barriers and buffers exist before any remote access
+  cluster_arrive_relaxed();   // phase 1: this CTA's barriers are initialised
   const uint32_t tmem = *tslot;
-
-  // ---- weight stream first: the whole slice is requested at once
-  if (warp == 0 && lane == 0) {
-    for (int b = 0; b < nb; ++b) {
-      mbar_arrive_expect_tx(&full[b], kRows * kKB);
-      tma_load_2d(ring + b * kRows * kKB, &tmWq, &full[b], (kb0 + b) * kKB, n0);
-    }
-  }
-  // ---- this CTA's K-range of every token row of X
   bool ok = true;
-  if (kw > 0) {
-    if (tid == 0) {
+
+  if (warp == 0) {
+    // ---------------------------------------------------------------- producer
+    if (lane == 0) {
       mbar_arrive_expect_tx(xbar, static_cast<uint32_t>(M * kw * 2));
       for (int t = 0; t < M; ++t)
         bulk_load(xs + t * kw, a.X + static_cast<size_t>(t) * K + k0,
                   static_cast<uint32_t>(kw * 2), xbar);
+      for (int b = 0; b < nb; ++b) {
+        mbar_arrive_expect_tx(&full[b], kRows * kKB);
+        tma_load_2d(ring + b * kRows * kKB, &tmWq, &full[b], (kb0 + b) * kKB, n0);
+      }
     }
-    if (!mbar_wait(xbar, 0)) ok = false;
-  }
+    __syncwarp();
+    cluster_wait();
+    cluster_arrive();
+  } else if (warp == 1) {
+    // ---------------------------------------------------------------- MMA issuer
+    cluster_wait();
+    ok = __all_sync(0xffffffffu, mbar_wait(codes_bar, 0));
+    constexpr uint32_t idesc = make_idesc(2 /*s32*/, 1 /*signed*/, kRows, kTok);
+    for (int b = 0; b < nb && ok; ++b) {
+      ok = __all_sync(0xffffffffu, mbar_wait(&full[b], 0));
+      if (!ok) break;
+      tc_fence_after();
+      if (lane == 0) {
+        const uint32_t ad = smem_addr(ring + b * kRows * kKB);
+        const uint32_t bd = smem_addr(bop + b * kTok * kKB);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          mma_i8(tmem, sw128_kmajor_desc(ad + 32 * kk), sw128_kmajor_desc(bd + 32 * kk), idesc,
+                 (b | kk) != 0);
+      }
+      __syncwarp();
+    }
+    // Always committed, so the epilogue's wait ends even after a failed wait here.
+    if (lane == 0) mma_commit(done);
+    __syncwarp();
+    cluster_arrive();
+  } else {
+    // ---------------------------------------------------------------- X workers
+    const int xw = warp - 2;                 // 0..7
+    const int xi = tid - 64;                 // 0..255
+    const int c0 = 4 * xi;                   // first of the thread's 4 columns (CTA-local)
+    const bool cv = c0 < kw;                 // kw is a multiple of 16
+    const float thr = a.threshold;
+    const bool epi = (warp >= 4 && warp < 8);
+    const int r = (warp & 3) * 32 + lane;    // epilogue: tile row = TMEM lane
 
-  // ---- outlier flags of the CTA's columns (exact: every token is here) and
-  //      per-token maxima over its non-outlier columns
-  const int nvec = kw >> 3;                              // 16-byte vectors per row
-  float part[kTok];
+    ok = __all_sync(0xffffffffu, mbar_wait(xbar, 0));
+    uint2 h[kTok];
 #pragma unroll
-  for (int t = 0; t < kTok; ++t) part[t] = 0.0f;
-  if (tid < 128) {                                       // 128 vectors cover 1024 columns
-    const int v = tid;
-    uint32_t m8 = 0;
-    if (v < nvec) {
-      float cm[8];
+    for (int t = 0; t < kTok; ++t)
+      h[t] = (cv && t < M) ? *reinterpret_cast<const uint2*>(xs + t * kw + c0) : make_uint2(0u, 0u);
+
+    // Outlier flags of the 4 columns: the max of |x| over all tokens against the threshold.
+    __half2 m01 = __float2half2_rn(0.0f), m23 = m01;
 #pragma unroll
-      for (int i = 0; i < 8; ++i) cm[i] = 0.0f;
-      for (int t = 0; t < M; ++t) {
-        float f[8];
-        unpack8(*reinterpret_cast<const uint4*>(xs + t * kw + v * 8), f);
+    for (int t = 0; t < kTok; ++t) {
+      m01 = __hmax2(m01, habs2_bits(h[t].x));
+      m23 = __hmax2(m23, habs2_bits(h[t].y));
+    }
+    const float2 f01 = __half22float2(m01), f23 = __half22float2(m23);
+    const uint32_t f4 = (f01.x > thr ? 1u : 0u) | (f01.y > thr ? 2u : 0u) |
+                        (f23.x > thr ? 4u : 0u) | (f23.y > thr ? 8u : 0u);
+    const uint32_t keep0 = ((f4 & 1u) ? 0u : 0x0000FFFFu) | ((f4 & 2u) ? 0u : 0xFFFF0000u);
+    const uint32_t keep1 = ((f4 & 4u) ? 0u : 0x0000FFFFu) | ((f4 & 8u) ? 0u : 0xFFFF0000u);
+
+    // Per-token max of |x| over the non-outlier columns, then a reduce-scatter
+    // over the warp: lane l ends with token (l >> 1) & 15.
+    float pm[kTok];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) cm[i] = fmaxf(cm[i], fabsf(f[i]));
+    for (int t = 0; t < kTok; ++t) {
+      const __half2 m = __hmax2(habs2_bits(h[t].x & keep0), habs2_bits(h[t].y & keep1));
+      pm[t] = fmaxf(__low2float(m), __high2float(m));
+    }
+    {
+      const bool u16 = lane & 16, u8 = lane & 8, u4 = lane & 4, u2 = lane & 2;
+      float v8[8], v4[4], v2[2];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const float send = u16 ? pm[i] : pm[i + 8];
+        const float keep = u16 ? pm[i + 8] : pm[i];
+        v8[i] = fmaxf(keep, __shfl_xor_sync(0xffffffffu, send, 16));
       }
 #pragma unroll
-      for (int i = 0; i < 8; ++i) m8 |= (cm[i] > a.threshold ? 1u : 0u) << i;
+      for (int i = 0; i < 4; ++i) {
+        const float send = u8 ? v8[i] : v8[i + 4];
+        const float keep = u8 ? v8[i + 4] : v8[i];
+        v4[i] = fmaxf(keep, __shfl_xor_sync(0xffffffffu, send, 8));
+      }
+#pragma unroll
+      for (int i = 0; i < 2; ++i) {
+        const float send = u4 ? v4[i] : v4[i + 2];
+        const float keep = u4 ? v4[i + 2] : v4[i];
+        v2[i] = fmaxf(keep, __shfl_xor_sync(0xffffffffu, send, 4));
+      }
+      const float send = u2 ? v2[0] : v2[1];
+      const float keep = u2 ? v2[1] : v2[0];
+      float v = fmaxf(keep, __shfl_xor_sync(0xffffffffu, send, 2));
+      v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 1));
+      if (!(lane & 1)) red[xw * kTok + ((lane >> 1) & 15)] = v;
+    }
+    // Bitmap word of 32 columns = 8 threads x 4 flags.
+    {
+      uint32_t word = f4 << (4 * (lane & 7));
+      word |= __shfl_xor_sync(0xffffffffu, word, 1);
+      word |= __shfl_xor_sync(0xffffffffu, word, 2);
+      word |= __shfl_xor_sync(0xffffffffu, word, 4);
+      if ((lane & 7) == 0) bits[xi >> 3] = word;
+    }
+    named_bar_sync(kBarX, kXThreads);
+
+    if (xw == 0) {
+      // Local outlier list (ascending) and count; then the message to every rank.
+      const int words = (kw + 31) >> 5;
+      const uint32_t bw = (lane < words) ? bits[lane] : 0u;
+      const int c = __popc(bw);
+      int incl = c;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int t = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += t;
+      }
+      uint32_t bb = bw;
+      int p = incl - c;
+      while (bb) {
+        const int j = __ffs(bb) - 1;
+        bb &= bb - 1;
+        lidx[p++] = static_cast<uint16_t>(lane * 32 + j);
+      }
+      const int lcount = __shfl_sync(0xffffffffu, incl, 31);
+      if (lane == 0) misc[0] = lcount;
+      __syncwarp();
+      named_bar_arrive(kBarList, 32 + 128);
+      cluster_wait();   // every CTA's barriers are initialised
+      for (int i = lane; i < S * 5; i += 32) {
+        const int dst = i / 5, ch = i - dst * 5;
+        uint32_t v[4] = {0u, 0u, 0u, 0u};
+        if (ch < 4) {
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            float m = 0.0f;
+#pragma unroll
+            for (int w = 0; w < kXWarps; ++w) m = fmaxf(m, red[w * kTok + 4 * ch + j]);
+            v[j] = __float_as_uint(m);
+          }
+        } else {
+          v[0] = static_cast<uint32_t>(lcount);
+        }
+        st_async_v4(cluster_addr(&msg[rank * kMsgWords + 4 * ch], dst), v[0], v[1], v[2], v[3],
+                    cluster_addr(xchg, dst));
+      }
+    } else {
+      cluster_wait();
+    }
+
+    // Epilogue warps: start the gathers of the outlier weights now, they have
+    // the whole exchange and the code pass to land.
+    int lcount = 0;
+    __half wv[kWPrefetch];
+    if (epi) {
+      named_bar_sync(kBarList, 32 + 128);
+      lcount = misc[0];
+      const int n = n0 + r;
+      const __half* wrow = a.W + static_cast<size_t>(min(n, N - 1)) * K + k0;
+#pragma unroll
+      for (int j = 0; j < kWPrefetch; ++j)
+        wv[j] = (j < lcount && n < N) ? wrow[lidx[j]] : __float2half(0.0f);
+      const int owned = owned_rows(rank, rpr);
+      if (r < owned) {
+        const int nr = n0 + rank * rpr + r;
+        wsc[r] = (nr < N) ? a.w_scale[nr] : 0.0f;
+      }
+    }
+
+    // Token absmax over the whole cluster, its inverse, the outlier prefix.
+    ok = __all_sync(0xffffffffu, mbar_wait(xchg, 0)) && ok;
+    if (xw == 0) {
+      if (lane < kTok) {
+        float m = 0.0f;
+        for (int s = 0; s < S; ++s) m = fmaxf(m, __uint_as_float(msg[s * kMsgWords + lane]));
+        amax_s[lane] = m;
+        inv_s[lane] = quant_inv(m);
+        if (writer && rank == 0 && lane < M) a.x_scale[lane] = m;
+      }
+      if (lane == 0) {
+        int prefix = 0, total = 0;
+        for (int s = 0; s < S; ++s) {
+          const int cs = static_cast<int>(msg[s * kMsgWords + 16]);
+          if (s < rank) prefix += cs;
+          total += cs;
+        }
+        misc[1] = prefix;
+        if (writer && rank == 0) *a.n_outliers = total;
+      }
+    }
+    named_bar_sync(kBarX, kXThreads);
+
+    if (writer) {
+      if (xi < ((kw + 31) >> 5)) a.bitmap[(k0 >> 5) + xi] = bits[xi];
+      const int lc = misc[0], prefix = misc[1];
+      for (int i = xi; i < lc; i += kXThreads) a.col_idx[prefix + i] = k0 + lidx[i];
+    }
+
+    // INT8 codes of the 4 columns for every token, into the B operand (and Xq).
+    if (c0 < nb * kKB) {
+      const uint32_t kb = static_cast<uint32_t>(c0) >> 7, kc = static_cast<uint32_t>(c0) & 127u;
+      const uint32_t keepq = keep_bytes(f4);
 #pragma unroll
       for (int t = 0; t < kTok; ++t) {
-        if (t < M) {
-          float f[8];
-          unpack8(*reinterpret_cast<const uint4*>(xs + t * kw + v * 8), f);
-          float pm = 0.0f;
+        uint32_t q = 0u;
+        if (cv && t < M) q = codes4(h[t], amax_s[t], inv_s[t]) & keepq;
+        const uint32_t off = kb * (kTok * kKB) + (t >> 3) * 1024 + (t & 7) * 128 +
+                             ((((kc >> 4) ^ static_cast<uint32_t>(t & 7))) << 4) + (kc & 15u);
+        *reinterpret_cast<uint32_t*>(bop + off) = q;
+        if (writer && cv && t < M)
+          *reinterpret_cast<uint32_t*>(a.Xq + static_cast<size_t>(t) * K + k0 + c0) = q;
+      }
+    }
+    fence_proxy_async_smem();   // the tensor core reads what the generic proxy wrote
+    __syncwarp();
+    if (lane == 0) mbar_arrive(codes_bar);
+
+    if (!epi) {
+      cluster_arrive();
+    } else {
+      // fp32 outlier partials of this row over the CTA's outlier columns.
+      float o[kTok];
 #pragma unroll
-          for (int i = 0; i < 8; ++i)
-            if (!((m8 >> i) & 1u)) pm = fmaxf(pm, fabsf(f[i]));
-          part[t] = pm;
+      for (int t = 0; t < kTok; ++t) o[t] = 0.0f;
+#pragma unroll
+      for (int j = 0; j < kWPrefetch; ++j) {
+        if (j < lcount) {
+          const int col = lidx[j];
+          const float w = __half2float(wv[j]);
+#pragma unroll
+          for (int t = 0; t < kTok; ++t)
+            if (t < M) o[t] = fmaf(__half2float(xs[t * kw + col]), w, o[t]);
+        }
+      }
+      if (lcount > kWPrefetch) {
+        const int n = n0 + r;
+        const __half* wrow = a.W + static_cast<size_t>(min(n, N - 1)) * K + k0;
+        for (int j = kWPrefetch; j < lcount; ++j) {
+          const int col = lidx[j];
+          const float w = (n < N) ? __half2float(wrow[col]) : 0.0f;
+#pragma unroll
+          for (int t = 0; t < kTok; ++t)
+            if (t < M) o[t] = fmaf(__half2float(xs[t * kw + col]), w, o[t]);
+        }
+      }
+
+      // INT32 partials of the row from TMEM.
+      uint32_t acc[kTok];
+      const bool got = __all_sync(0xffffffffu, mbar_wait(done, 0));
+      if (got) {
+        tc_fence_after();
+        tmem_ld_32x32b_x16(tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16), acc);
+        tmem_ld_wait();
+      } else {
+#pragma unroll
+        for (int t = 0; t < kTok; ++t) acc[t] = 0u;
+      }
+      ok = ok && got;
+
+      // Push the row's partials to the rank that finishes it: 8 chunks of 16 B,
+      // chunk c at position c ^ (row & 7) to spread the banks of the final reads.
+      {
+        const int own = r / rpr, rl = r - own * rpr;
+        const uint32_t base = cluster_addr(recv + (rank * rpr + rl) * 128, own);
+        const uint32_t bar = cluster_addr(redbar, own);
+#pragma unroll
+        for (int ch = 0; ch < 8; ++ch) {
+          const uint32_t pos = static_cast<uint32_t>(ch ^ (rl & 7)) << 4;
+          if (ch < 4)
+            st_async_v4(base + pos, acc[4 * ch], acc[4 * ch + 1], acc[4 * ch + 2], acc[4 * ch + 3],
+                        bar);
+          else
+            st_async_v4(base + pos, __float_as_uint(o[4 * (ch - 4)]),
+                        __float_as_uint(o[4 * (ch - 4) + 1]), __float_as_uint(o[4 * (ch - 4) + 2]),
+                        __float_as_uint(o[4 * (ch - 4) + 3]), bar);
+        }
+      }
+      cluster_arrive();
+
+      // Finish the owned rows: sum the S partials in rank order, dequantise, add.
+      ok = __all_sync(0xffffffffu, mbar_wait(redbar, 0)) && ok;
+      named_bar_sync(kBarEpi, 128);   // wsc of all owned rows is written
+      const int owned = owned_rows(rank, rpr);
+      const int32_t* ri = reinterpret_cast<const int32_t*>(recv);
+      const float* rf = reinterpret_cast<const float*>(recv);
+      for (int e = (warp & 3) * 32 + lane; e < owned * kTok; e += 128) {
+        const int t = e / owned;
+        const int rl = e - t * owned;
+        const int n = n0 + rank * rpr + rl;
+        if (t < M && n < N) {
+          const int pi = (((t >> 2) ^ (rl & 7)) << 2) + (t & 3);
+          const int pf = (((4 + (t >> 2)) ^ (rl & 7)) << 2) + (t & 3);
+          int32_t c = 0;
+          float of = 0.0f;
+          for (int s = 0; s < S; ++s) {
+            const int row = (s * rpr + rl) * 32;
+            c += ri[row + pi];
+            of += rf[row + pf];
+          }
+          const float rs = amax_s[t] * (1.0f / 16129.0f);
+          const float y = static_cast<float>(c) * (rs * wsc[rl]) + of;
+          a.Y[static_cast<size_t>(t) * N + n] = __float2half_rn(y);
         }
       }
     }
-    uint32_t word = m8 << (8 * (lane & 3));
-    word |= __shfl_xor_sync(0xffffffffu, word, 1);
-    word |= __shfl_xor_sync(0xffffffffu, word, 2);
-    if ((lane & 3) == 0) bits[v >> 2] = (v < nvec) ? word : 0u;
-  }
-#pragma unroll
-  for (int t = 0; t < kTok; ++t) {
-    const float m = warp_max(part[t]);
-    if (lane == 0) red[warp * kTok + t] = m;
-  }
-  __syncthreads();
-  if (tid < kTok) {
-    float m = 0.0f;
-    for (int w = 0; w < kWarps; ++w) m = fmaxf(m, red[w * kTok + tid]);
-    // Publish to every CTA of the cluster (slot = this CTA's rank).
-    for (int r = 0; r < S; ++r)
-      st_cluster_f32(cluster_addr(&xmax[rank * kTok + tid], r), m);
-  }
-  // Local outlier list in ascending order (one warp, 32 bitmap words at most).
-  if (warp == 0) {
-    const int words = (kw + 31) >> 5;
-    const uint32_t bw = (lane < words) ? bits[lane] : 0u;
-    const int c = __popc(bw);
-    int incl = c;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int t = __shfl_up_sync(0xffffffffu, incl, o);
-      if (lane >= o) incl += t;
-    }
-    uint32_t b = bw;
-    int p = incl - c;
-    while (b) {
-      const int j = __ffs(b) - 1;
-      b &= b - 1;
-      lidx[p++] = static_cast<uint16_t>(lane * 32 + j);
-    }
-    const int total = __shfl_sync(0xffffffffu, incl, 31);
-    if (lane == 0) {
-      misc[0] = total;
-      for (int r = 0; r < S; ++r) st_cluster_s32(cluster_addr(&xcnt[rank], r), total);
-    }
-  }
-  __syncthreads();
-  cluster_sync();   // maxima and counts of every rank have arrived
-
-  // ---- token absmax, global outlier positions, intermediates (cluster 0)
-  const int lcount = misc[0];
-  int prefix = 0, total = 0;
-  for (int r = 0; r < S; ++r) {
-    const int c = xcnt[r];
-    if (r < rank) prefix += c;
-    total += c;
-  }
-  if (tid < kTok) {
-    float m = 0.0f;
-    for (int r = 0; r < S; ++r) m = fmaxf(m, xmax[r * kTok + tid]);
-    amax[tid] = m;
-    if (writer && rank == 0 && tid < M) a.x_scale[tid] = m;
-  }
-  if (writer) {
-    for (int w = tid; w < ((kw + 31) >> 5); w += kThreads) a.bitmap[(k0 >> 5) + w] = bits[w];
-    for (int i = tid; i < lcount; i += kThreads) a.col_idx[prefix + i] = k0 + lidx[i];
-    if (rank == 0 && tid == 0) *a.n_outliers = total;
-  }
-  __syncthreads();
-
-  // ---- INT8 codes of the X range into the swizzled K-major B operand (16 rows)
-  //      and, in cluster 0, into Xq
-  for (int e = tid; e < kTok * nb * 8; e += kThreads) {
-    const int t = e / (nb * 8);
-    const int c = e - t * (nb * 8);                      // 16-byte chunk along K
-    const int b = c >> 3, cc = c & 7;
-    uint4 q = make_uint4(0, 0, 0, 0);
-    const int kc = c * 16;                                // first column of the chunk
-    if (t < M && kc < kw) {
-      const float am = amax[t];
-      const float inv = quant_inv(am);
-      const uint32_t wbits = bits[kc >> 5] >> (kc & 31);  // 16 flag bits of the chunk
-      uint32_t* qw = reinterpret_cast<uint32_t*>(&q);
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        float f[8];
-        unpack8(*reinterpret_cast<const uint4*>(xs + t * kw + kc + h * 8), f);
-        int code[8];
-#pragma unroll
-        for (int i = 0; i < 8; ++i)
-          code[i] = ((wbits >> (h * 8 + i)) & 1u) ? 0 : quant_code_fast(f[i], am, inv);
-        qw[2 * h] = pack4(code[0], code[1], code[2], code[3]);
-        qw[2 * h + 1] = pack4(code[4], code[5], code[6], code[7]);
-      }
-      if (writer)
-        *reinterpret_cast<uint4*>(a.Xq + static_cast<size_t>(t) * K + k0 + kc) = q;
-    }
-    uint8_t* dst = bop + b * (kTok * kKB) + (t >> 3) * 1024 + (t & 7) * 128 + ((cc ^ (t & 7)) << 4);
-    *reinterpret_cast<uint4*>(dst) = q;
-  }
-  fence_proxy_async_smem();   // generic writes above are read by the tensor core
-  __syncthreads();
-
-  // ---- MMA: D[128 weight rows][16 tokens] += Wq_slice . Xq_range^T
-  if (warp == 1 && lane == 0) {
-    constexpr uint32_t idesc = make_idesc(2 /*s32*/, 1 /*signed*/, kRows, kTok);
-    for (int b = 0; b < nb; ++b) {
-      if (!mbar_wait(&full[b], 0)) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
-      const uint32_t ad = smem_addr(ring + b * kRows * kKB);
-      const uint32_t bd = smem_addr(bop + b * kTok * kKB);
-#pragma unroll
-      for (int kk = 0; kk < 4; ++kk)
-        mma_i8(tmem, sw128_kmajor_desc(ad + 32 * kk), sw128_kmajor_desc(bd + 32 * kk), idesc,
-               (b | kk) != 0);
-    }
-    mma_commit(done);
   }
 
-  // ---- fp32 outlier partials of this CTA's outlier columns (CUDA cores)
-  if (tid < kRows) {
-    float o[kTok];
-#pragma unroll
-    for (int t = 0; t < kTok; ++t) o[t] = 0.0f;
-    const int n = n0 + tid;
-    if (n < N) {
-      const __half* wrow = a.W + static_cast<size_t>(n) * K + k0;
-      for (int i = 0; i < lcount; ++i) {
-        const int j = lidx[i];
-        const float w = __half2float(wrow[j]);
-#pragma unroll
-        for (int t = 0; t < kTok; ++t)
-          if (t < M) o[t] = fmaf(__half2float(xs[t * kw + j]), w, o[t]);
-      }
-    }
-#pragma unroll
-    for (int t = 0; t < kTok; ++t) p_f32[tid * kTok + t] = o[t];
-  }
-
-  // ---- INT32 partials from TMEM (warps 4..7: lane quarters 0..3)
-  if (warp >= 4) {
-    const int q = warp & 3;
-    uint32_t acc[16];
-    bool got = true;
-    if (nb > 0) got = __all_sync(0xffffffffu, mbar_wait(done, 0));
-    if (nb > 0 && got) {
-      tc_fence_after();
-      tmem_ld_32x32b_x16(tmem + (static_cast<uint32_t>(q * 32) << 16), acc);
-      tmem_ld_wait();
-    } else {
-#pragma unroll
-      for (int t = 0; t < 16; ++t) acc[t] = 0u;
-    }
-    if (!got) ok = false;
-    const int r = q * 32 + lane;
-#pragma unroll
-    for (int t = 0; t < kTok; ++t) p_i32[r * kTok + t] = static_cast<int32_t>(acc[t]);
-  }
-  if (!ok && a.status) atomicExch(a.status, kStatusTimeout);
+  if (!ok && lane == 0 && a.status) atomicExch(a.status, kStatusTimeout);
   tc_fence_before();
   __syncthreads();
-  cluster_sync();   // every rank's partials are complete
-
-  // ---- sum the partials of all ranks (fixed order) for this CTA's share of rows
-  const int rpr = (kRows + S - 1) / S;
-  for (int e = tid; e < rpr * kTok; e += kThreads) {
-    const int t = e / rpr;
-    const int rl = rank * rpr + (e - t * rpr);
-    const int n = n0 + rl;
-    if (t < M && rl < kRows && n < N) {
-      int32_t c = 0;
-      float o = 0.0f;
-      for (int r = 0; r < S; ++r) {
-        c += ld_cluster_s32(cluster_addr(&p_i32[rl * kTok + t], r));
-        o += ld_cluster_f32(cluster_addr(&p_f32[rl * kTok + t], r));
-      }
-      const float rs = amax[t] * (1.0f / 16129.0f);
-      const float y = static_cast<float>(c) * (rs * a.w_scale[n]) + o;
-      a.Y[static_cast<size_t>(t) * N + n] = __float2half_rn(y);
-    }
-  }
-  __syncthreads();
-  cluster_sync();   // no CTA leaves while a peer may still read its partials
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem, 32);
   }
+  cluster_wait();   // no CTA leaves while a peer may still store into it
 }
 
 }  // namespace
 
-bool decode_supported(int M, int K) { return M >= 1 && M <= kTok && K <= kMaxCluster * kMaxBlocks * kKB; }
+bool decode_supported(int M, int K) {
+  return M >= 1 && M <= kTok && K <= kMaxCluster * kMaxBlocks * kKB;
+}
 
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t s) {
   CUtensorMap tm;

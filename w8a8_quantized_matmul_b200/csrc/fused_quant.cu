@@ -47,8 +47,6 @@ constexpr int kThreads = 512;
 constexpr int kWarps = kThreads / 32;
 constexpr int kMaxGroup = 16;                 // rows per reduction group (and per wave)
 constexpr uint64_t kBarrierLimitNs = 2000000000ull;
-constexpr float kMagic = 12582912.0f;         // 1.5 * 2^23
-constexpr float kTieMargin = 0.5f - 6.2e-5f;
 
 __device__ __forceinline__ int ld_acquire(const int32_t* p) {
   int v;
@@ -60,76 +58,6 @@ __device__ __forceinline__ uint64_t gtimer() {
   uint64_t t;
   asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
   return t;
-}
-
-// Paired IEEE fp32 arithmetic (round to nearest even in each lane).
-__device__ __forceinline__ uint64_t f2pack(float a, float b) {
-  return static_cast<uint64_t>(__float_as_uint(a)) |
-         (static_cast<uint64_t>(__float_as_uint(b)) << 32);
-}
-__device__ __forceinline__ uint64_t mul2(uint64_t a, uint64_t b) {
-  uint64_t r;
-  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
-  return r;
-}
-__device__ __forceinline__ uint64_t add2(uint64_t a, uint64_t b) {
-  uint64_t r;
-  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
-  return r;
-}
-__device__ __forceinline__ uint64_t sub2(uint64_t a, uint64_t b) {
-  uint64_t r;
-  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
-  return r;
-}
-__device__ __forceinline__ float lo(uint64_t v) { return __uint_as_float(static_cast<uint32_t>(v)); }
-__device__ __forceinline__ float hi(uint64_t v) { return __uint_as_float(static_cast<uint32_t>(v >> 32)); }
-
-// |x| of both halves (sign bits cleared) as a half2.
-__device__ __forceinline__ __half2 habs2_bits(uint32_t w) {
-  const uint32_t a = w & 0x7FFF7FFFu;
-  return *reinterpret_cast<const __half2*>(&a);
-}
-
-// 0xFFFF in each half that is NOT an outlier column, for half2 i of an 8-column mask.
-__device__ __forceinline__ uint32_t keep_half2(uint32_t m8, int i) {
-  return (((m8 >> (2 * i)) & 1u) ? 0u : 0x0000FFFFu) | (((m8 >> (2 * i + 1)) & 1u) ? 0u : 0xFFFF0000u);
-}
-
-// 0xFF in each byte of a 4-code word that is NOT an outlier column.
-__device__ __forceinline__ uint32_t keep_bytes(uint32_t m4) {
-  return ((m4 & 1u) ? 0u : 0x000000FFu) | ((m4 & 2u) ? 0u : 0x0000FF00u) |
-         ((m4 & 4u) ? 0u : 0x00FF0000u) | ((m4 & 8u) ? 0u : 0xFF000000u);
-}
-
-// Eight INT8 codes of the vector u (exact; see the file comment).
-__device__ __forceinline__ uint2 codes8(const uint4& u, float amax, float inv) {
-  if (amax == 0.0f) return make_uint2(0u, 0u);
-  const uint32_t* w = reinterpret_cast<const uint32_t*>(&u);
-  const uint64_t inv2 = f2pack(inv, inv);
-  const uint64_t magic2 = f2pack(kMagic, kMagic);
-  uint32_t b[8];
-  float emax = 0.0f;
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&w[i]));
-    const uint64_t y = mul2(f2pack(f.x, f.y), inv2);
-    const uint64_t s = add2(y, magic2);
-    const uint64_t e = sub2(y, sub2(s, magic2));
-    emax = fmaxf(emax, fmaxf(fabsf(lo(e)), fabsf(hi(e))));
-    b[2 * i] = static_cast<uint32_t>(s);
-    b[2 * i + 1] = static_cast<uint32_t>(s >> 32);
-  }
-  if (emax > kTieMargin) {
-    // Within reach of a rounding tie: form the correctly rounded quotient.
-    float f[8];
-    unpack8(u, f);
-#pragma unroll
-    for (int i = 0; i < 8; ++i) b[i] = static_cast<uint32_t>(quant_code(f[i], amax));
-  }
-  const uint32_t w0 = __byte_perm(__byte_perm(b[0], b[1], 0x0040), __byte_perm(b[2], b[3], 0x0040), 0x5410);
-  const uint32_t w1 = __byte_perm(__byte_perm(b[4], b[5], 0x0040), __byte_perm(b[6], b[7], 0x0040), 0x5410);
-  return make_uint2(w0, w1);
 }
 
 }  // namespace
