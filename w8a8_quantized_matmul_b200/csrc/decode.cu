@@ -102,9 +102,11 @@ __device__ __forceinline__ int owned_rows(int rank, int rpr) {
 
 __global__ void __launch_bounds__(kThreads, 1)
     decode_kernel(const __grid_constant__ CUtensorMap tmWq, DecodeArgs a) {
-  extern __shared__ uint8_t dsm_raw[];
-  uint8_t* sm = reinterpret_cast<uint8_t*>(
-      (reinterpret_cast<uintptr_t>(dsm_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  extern __shared__ __align__(1024) uint8_t dsm_raw[];
+  // 1024-byte aligned base (swizzle atoms). Derived by an offset from the
+  // shared array, not through an integer cast, so every pointer below stays in
+  // the shared state space and compiles to shared-memory loads and stores.
+  uint8_t* sm = dsm_raw + ((1024u - (smem_addr(dsm_raw) & 1023u)) & 1023u);
   using L = DecodeSmem;
   uint8_t* ring = sm + L::RING;
   uint8_t* bop = sm + L::BOP;
@@ -154,8 +156,18 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_arrive_expect_tx(xchg, static_cast<uint32_t>(S * kMsgWords * 4));
     mbar_arrive_expect_tx(redbar, static_cast<uint32_t>(S * owned_rows(rank, rpr) * 128));
     fence_mbarrier_init();
-    tma_prefetch_desc(&tmWq);
     if (blockIdx.x == 0 && a.status) *a.status = 0;
+    // Producer: X first (small, L2-resident after the first cluster), then the
+    // whole Wq slice. Issued before the CTA barrier: only this thread has used
+    // the barriers so far.
+    mbar_arrive_expect_tx(xbar, static_cast<uint32_t>(M * kw * 2));
+    for (int t = 0; t < M; ++t)
+      bulk_load(xs + t * kw, a.X + static_cast<size_t>(t) * K + k0, static_cast<uint32_t>(kw * 2),
+                xbar);
+    for (int b = 0; b < nb; ++b) {
+      mbar_arrive_expect_tx(&full[b], kRows * kKB);
+      tma_load_2d(ring + b * kRows * kKB, &tmWq, &full[b], (kb0 + b) * kKB, n0);
+    }
   }
   if (warp == 1) {
     tmem_alloc(tslot, 32);
@@ -169,45 +181,34 @@ __global__ void __launch_bounds__(kThreads, 1)
   bool ok = true;
 
   if (warp == 0) {
-    // ---------------------------------------------------------------- producer
-    if (lane == 0) {
-      mbar_arrive_expect_tx(xbar, static_cast<uint32_t>(M * kw * 2));
-      for (int t = 0; t < M; ++t)
-        bulk_load(xs + t * kw, a.X + static_cast<size_t>(t) * K + k0,
-                  static_cast<uint32_t>(kw * 2), xbar);
-      for (int b = 0; b < nb; ++b) {
-        mbar_arrive_expect_tx(&full[b], kRows * kKB);
-        tma_load_2d(ring + b * kRows * kKB, &tmWq, &full[b], (kb0 + b) * kKB, n0);
-      }
-    }
-    __syncwarp();
+    // ---------------------------------------------------------------- producer (done)
     cluster_wait();
     cluster_arrive();
   } else if (warp == 1) {
     // ---------------------------------------------------------------- MMA issuer
+    // The whole warp runs the loop; one elected lane issues each MMA.
     cluster_wait();
     ok = __all_sync(0xffffffffu, mbar_wait(codes_bar, 0));
     constexpr uint32_t idesc = make_idesc(2 /*s32*/, 1 /*signed*/, kRows, kTok);
+    const uint64_t a0 = sw128_kmajor_desc(smem_addr(ring));
+    const uint64_t b0 = sw128_kmajor_desc(smem_addr(bop));
     for (int b = 0; b < nb && ok; ++b) {
       ok = __all_sync(0xffffffffu, mbar_wait(&full[b], 0));
       if (!ok) break;
       tc_fence_after();
-      if (lane == 0) {
-        const uint32_t ad = smem_addr(ring + b * kRows * kKB);
-        const uint32_t bd = smem_addr(bop + b * kTok * kKB);
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk)
-          mma_i8(tmem, sw128_kmajor_desc(ad + 32 * kk), sw128_kmajor_desc(bd + 32 * kk), idesc,
-                 (b | kk) != 0);
-      }
-      __syncwarp();
+      for (int kk = 0; kk < 4; ++kk)
+        mma_i8_elect(tmem, a0 + static_cast<uint64_t>((b * kRows * kKB + 32 * kk) >> 4),
+                     b0 + static_cast<uint64_t>((b * kTok * kKB + 32 * kk) >> 4), idesc,
+                     (b | kk) != 0);
     }
     // Always committed, so the epilogue's wait ends even after a failed wait here.
-    if (lane == 0) mma_commit(done);
-    __syncwarp();
+    mma_commit_elect(done);
     cluster_arrive();
   } else {
     // ---------------------------------------------------------------- X workers
+    // Loops over tokens stay rolled: this code runs once per launch, and
+    // straight-line code would be bound by instruction fetch.
     const int xw = warp - 2;                 // 0..7
     const int xi = tid - 64;                 // 0..255
     const int c0 = 4 * xi;                   // first of the thread's 4 columns (CTA-local)
@@ -215,61 +216,26 @@ __global__ void __launch_bounds__(kThreads, 1)
     const float thr = a.threshold;
     const bool epi = (warp >= 4 && warp < 8);
     const int r = (warp & 3) * 32 + lane;    // epilogue: tile row = TMEM lane
+    const uint2* xrow = reinterpret_cast<const uint2*>(xs) + xi;   // + t * (kw / 4)
+    const int xstride = kw >> 2;             // uint2 per token row
 
     ok = __all_sync(0xffffffffu, mbar_wait(xbar, 0));
-    uint2 h[kTok];
-#pragma unroll
-    for (int t = 0; t < kTok; ++t)
-      h[t] = (cv && t < M) ? *reinterpret_cast<const uint2*>(xs + t * kw + c0) : make_uint2(0u, 0u);
 
     // Outlier flags of the 4 columns: the max of |x| over all tokens against the threshold.
     __half2 m01 = __float2half2_rn(0.0f), m23 = m01;
-#pragma unroll
-    for (int t = 0; t < kTok; ++t) {
-      m01 = __hmax2(m01, habs2_bits(h[t].x));
-      m23 = __hmax2(m23, habs2_bits(h[t].y));
+    if (cv) {
+#pragma unroll 4
+      for (int t = 0; t < M; ++t) {
+        const uint2 v = xrow[t * xstride];
+        m01 = __hmax2(m01, habs2_bits(v.x));
+        m23 = __hmax2(m23, habs2_bits(v.y));
+      }
     }
     const float2 f01 = __half22float2(m01), f23 = __half22float2(m23);
     const uint32_t f4 = (f01.x > thr ? 1u : 0u) | (f01.y > thr ? 2u : 0u) |
                         (f23.x > thr ? 4u : 0u) | (f23.y > thr ? 8u : 0u);
     const uint32_t keep0 = ((f4 & 1u) ? 0u : 0x0000FFFFu) | ((f4 & 2u) ? 0u : 0xFFFF0000u);
     const uint32_t keep1 = ((f4 & 4u) ? 0u : 0x0000FFFFu) | ((f4 & 8u) ? 0u : 0xFFFF0000u);
-
-    // Per-token max of |x| over the non-outlier columns, then a reduce-scatter
-    // over the warp: lane l ends with token (l >> 1) & 15.
-    float pm[kTok];
-#pragma unroll
-    for (int t = 0; t < kTok; ++t) {
-      const __half2 m = __hmax2(habs2_bits(h[t].x & keep0), habs2_bits(h[t].y & keep1));
-      pm[t] = fmaxf(__low2float(m), __high2float(m));
-    }
-    {
-      const bool u16 = lane & 16, u8 = lane & 8, u4 = lane & 4, u2 = lane & 2;
-      float v8[8], v4[4], v2[2];
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const float send = u16 ? pm[i] : pm[i + 8];
-        const float keep = u16 ? pm[i + 8] : pm[i];
-        v8[i] = fmaxf(keep, __shfl_xor_sync(0xffffffffu, send, 16));
-      }
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const float send = u8 ? v8[i] : v8[i + 4];
-        const float keep = u8 ? v8[i + 4] : v8[i];
-        v4[i] = fmaxf(keep, __shfl_xor_sync(0xffffffffu, send, 8));
-      }
-#pragma unroll
-      for (int i = 0; i < 2; ++i) {
-        const float send = u4 ? v4[i] : v4[i + 2];
-        const float keep = u4 ? v4[i + 2] : v4[i];
-        v2[i] = fmaxf(keep, __shfl_xor_sync(0xffffffffu, send, 4));
-      }
-      const float send = u2 ? v2[0] : v2[1];
-      const float keep = u2 ? v2[1] : v2[0];
-      float v = fmaxf(keep, __shfl_xor_sync(0xffffffffu, send, 2));
-      v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 1));
-      if (!(lane & 1)) red[xw * kTok + ((lane >> 1) & 15)] = v;
-    }
     // Bitmap word of 32 columns = 8 threads x 4 flags.
     {
       uint32_t word = f4 << (4 * (lane & 7));
@@ -277,6 +243,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       word |= __shfl_xor_sync(0xffffffffu, word, 2);
       word |= __shfl_xor_sync(0xffffffffu, word, 4);
       if ((lane & 7) == 0) bits[xi >> 3] = word;
+    }
+    // Per-token max of |x| over the non-outlier columns: per thread, then over
+    // the warp (non-negative floats order like their bit patterns).
+#pragma unroll 2
+    for (int t = 0; t < M; ++t) {
+      const uint2 v = cv ? xrow[t * xstride] : make_uint2(0u, 0u);
+      const __half2 m = __hmax2(habs2_bits(v.x & keep0), habs2_bits(v.y & keep1));
+      const float pm = fmaxf(__low2float(m), __high2float(m));
+      const uint32_t wm = __reduce_max_sync(0xffffffffu, __float_as_uint(pm));
+      if (lane == 0) red[xw * kTok + t] = __uint_as_float(wm);
     }
     named_bar_sync(kBarX, kXThreads);
 
@@ -299,23 +275,27 @@ __global__ void __launch_bounds__(kThreads, 1)
         lidx[p++] = static_cast<uint16_t>(lane * 32 + j);
       }
       const int lcount = __shfl_sync(0xffffffffu, incl, 31);
+      // CTA maxima of the tokens (0 for the padding tokens).
+      float cm = 0.0f;
+      if (lane < M) {
+        for (int w = 0; w < kXWarps; ++w) cm = fmaxf(cm, red[w * kTok + lane]);
+      }
       if (lane == 0) misc[0] = lcount;
+      __syncwarp();
+      // Lane l alone read red[w][l]; its CTA maximum replaces red[0][l].
+      if (lane < kTok) red[lane] = cm;
       __syncwarp();
       named_bar_arrive(kBarList, 32 + 128);
       cluster_wait();   // every CTA's barriers are initialised
       for (int i = lane; i < S * 5; i += 32) {
         const int dst = i / 5, ch = i - dst * 5;
-        uint32_t v[4] = {0u, 0u, 0u, 0u};
+        uint32_t v[4] = {static_cast<uint32_t>(lcount), 0u, 0u, 0u};
         if (ch < 4) {
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            float m = 0.0f;
-#pragma unroll
-            for (int w = 0; w < kXWarps; ++w) m = fmaxf(m, red[w * kTok + 4 * ch + j]);
-            v[j] = __float_as_uint(m);
-          }
-        } else {
-          v[0] = static_cast<uint32_t>(lcount);
+          const float4 m4 = *reinterpret_cast<const float4*>(red + 4 * ch);
+          v[0] = __float_as_uint(m4.x);
+          v[1] = __float_as_uint(m4.y);
+          v[2] = __float_as_uint(m4.z);
+          v[3] = __float_as_uint(m4.w);
         }
         st_async_v4(cluster_addr(&msg[rank * kMsgWords + 4 * ch], dst), v[0], v[1], v[2], v[3],
                     cluster_addr(xchg, dst));
@@ -348,16 +328,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (xw == 0) {
       if (lane < kTok) {
         float m = 0.0f;
-        for (int s = 0; s < S; ++s) m = fmaxf(m, __uint_as_float(msg[s * kMsgWords + lane]));
+        for (int s2 = 0; s2 < S; ++s2) m = fmaxf(m, __uint_as_float(msg[s2 * kMsgWords + lane]));
         amax_s[lane] = m;
         inv_s[lane] = quant_inv(m);
         if (writer && rank == 0 && lane < M) a.x_scale[lane] = m;
       }
       if (lane == 0) {
         int prefix = 0, total = 0;
-        for (int s = 0; s < S; ++s) {
-          const int cs = static_cast<int>(msg[s * kMsgWords + 16]);
-          if (s < rank) prefix += cs;
+        for (int s2 = 0; s2 < S; ++s2) {
+          const int cs = static_cast<int>(msg[s2 * kMsgWords + 16]);
+          if (s2 < rank) prefix += cs;
           total += cs;
         }
         misc[1] = prefix;
@@ -374,17 +354,19 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     // INT8 codes of the 4 columns for every token, into the B operand (and Xq).
     if (c0 < nb * kKB) {
-      const uint32_t kb = static_cast<uint32_t>(c0) >> 7, kc = static_cast<uint32_t>(c0) & 127u;
+      const uint32_t kc = static_cast<uint32_t>(c0) & 127u;
+      uint8_t* dst = bop + (c0 >> 7) * (kTok * kKB) + (kc & 15u);
       const uint32_t keepq = keep_bytes(f4);
-#pragma unroll
+      int8_t* xq = a.Xq + k0 + c0;
+#pragma unroll 2
       for (int t = 0; t < kTok; ++t) {
         uint32_t q = 0u;
-        if (cv && t < M) q = codes4(h[t], amax_s[t], inv_s[t]) & keepq;
-        const uint32_t off = kb * (kTok * kKB) + (t >> 3) * 1024 + (t & 7) * 128 +
-                             ((((kc >> 4) ^ static_cast<uint32_t>(t & 7))) << 4) + (kc & 15u);
-        *reinterpret_cast<uint32_t*>(bop + off) = q;
-        if (writer && cv && t < M)
-          *reinterpret_cast<uint32_t*>(a.Xq + static_cast<size_t>(t) * K + k0 + c0) = q;
+        if (cv && t < M) {
+          q = codes4(xrow[t * xstride], amax_s[t], inv_s[t]) & keepq;
+          if (writer) *reinterpret_cast<uint32_t*>(xq + static_cast<size_t>(t) * K) = q;
+        }
+        const uint32_t off = (t >> 3) * 1024 + (t & 7) * 128 + (((kc >> 4) ^ (t & 7)) << 4);
+        *reinterpret_cast<uint32_t*>(dst + off) = q;
       }
     }
     fence_proxy_async_smem();   // the tensor core reads what the generic proxy wrote
@@ -398,26 +380,20 @@ __global__ void __launch_bounds__(kThreads, 1)
       float o[kTok];
 #pragma unroll
       for (int t = 0; t < kTok; ++t) o[t] = 0.0f;
+      const int n = n0 + r;
+      const __half* wrow = a.W + static_cast<size_t>(min(n, N - 1)) * K + k0;
+#pragma unroll 1
+      for (int j = 0; j < lcount; ++j) {
+        const int col = lidx[j];
+        __half wh = __float2half(0.0f);
 #pragma unroll
-      for (int j = 0; j < kWPrefetch; ++j) {
-        if (j < lcount) {
-          const int col = lidx[j];
-          const float w = __half2float(wv[j]);
+        for (int i = 0; i < kWPrefetch; ++i)
+          if (i == j) wh = wv[i];
+        if (j >= kWPrefetch && n < N) wh = wrow[col];
+        const float w = __half2float(wh);
 #pragma unroll
-          for (int t = 0; t < kTok; ++t)
-            if (t < M) o[t] = fmaf(__half2float(xs[t * kw + col]), w, o[t]);
-        }
-      }
-      if (lcount > kWPrefetch) {
-        const int n = n0 + r;
-        const __half* wrow = a.W + static_cast<size_t>(min(n, N - 1)) * K + k0;
-        for (int j = kWPrefetch; j < lcount; ++j) {
-          const int col = lidx[j];
-          const float w = (n < N) ? __half2float(wrow[col]) : 0.0f;
-#pragma unroll
-          for (int t = 0; t < kTok; ++t)
-            if (t < M) o[t] = fmaf(__half2float(xs[t * kw + col]), w, o[t]);
-        }
+        for (int t = 0; t < kTok; ++t)
+          if (t < M) o[t] = fmaf(__half2float(xs[t * kw + col]), w, o[t]);
       }
 
       // INT32 partials of the row from TMEM.
@@ -459,23 +435,24 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int owned = owned_rows(rank, rpr);
       const int32_t* ri = reinterpret_cast<const int32_t*>(recv);
       const float* rf = reinterpret_cast<const float*>(recv);
+#pragma unroll 1
       for (int e = (warp & 3) * 32 + lane; e < owned * kTok; e += 128) {
         const int t = e / owned;
         const int rl = e - t * owned;
-        const int n = n0 + rank * rpr + rl;
-        if (t < M && n < N) {
+        const int nn = n0 + rank * rpr + rl;
+        if (t < M && nn < N) {
           const int pi = (((t >> 2) ^ (rl & 7)) << 2) + (t & 3);
           const int pf = (((4 + (t >> 2)) ^ (rl & 7)) << 2) + (t & 3);
           int32_t c = 0;
           float of = 0.0f;
-          for (int s = 0; s < S; ++s) {
-            const int row = (s * rpr + rl) * 32;
+          for (int s2 = 0; s2 < S; ++s2) {
+            const int row = (s2 * rpr + rl) * 32;
             c += ri[row + pi];
             of += rf[row + pf];
           }
           const float rs = amax_s[t] * (1.0f / 16129.0f);
           const float y = static_cast<float>(c) * (rs * wsc[rl]) + of;
-          a.Y[static_cast<size_t>(t) * N + n] = __float2half_rn(y);
+          a.Y[static_cast<size_t>(t) * N + nn] = __float2half_rn(y);
         }
       }
     }

@@ -109,9 +109,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                               int32_t* status) {
   using C = Cfg<PAIR>;
   constexpr int STAGES = C::STAGES;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  // 1024-byte aligned base (swizzle atoms). Derived by an offset from the
+  // shared array, not through an integer cast, so every pointer below stays in
+  // the shared state space and compiles to shared-memory loads and stores.
+  uint8_t* smem = smem_raw + ((1024u - (smem_addr(smem_raw) & 1023u)) & 1023u);
   uint8_t* stg = smem + C::RING_BYTES;                                          // staging
   __half* wo_s = reinterpret_cast<__half*>(stg + C::STG_BYTES);                // [kCcMax][BN]
   float* sw_s = reinterpret_cast<float*>(stg + C::STG_BYTES + C::WO_BYTES);     // [BN]

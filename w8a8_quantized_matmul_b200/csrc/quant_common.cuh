@@ -185,33 +185,32 @@ __device__ __forceinline__ uint2 codes8(const uint4& u, float amax, float inv) {
   return make_uint2(w0, w1);
 }
 
+// Exact codes of four fp16 values (the tie fallback of codes4), kept out of line
+// so the common path stays short.
+static __device__ __noinline__ uint32_t codes4_exact(uint32_t w0, uint32_t w1, float amax) {
+  const float2 f0 = __half22float2(*reinterpret_cast<const __half2*>(&w0));
+  const float2 f1 = __half22float2(*reinterpret_cast<const __half2*>(&w1));
+  return pack4(quant_code(f0.x, amax), quant_code(f0.y, amax), quant_code(f1.x, amax),
+               quant_code(f1.y, amax));
+}
+
 // Four INT8 codes of the fp16 values in h (two half2 words), same rule as codes8.
 __device__ __forceinline__ uint32_t codes4(const uint2& h, float amax, float inv) {
   if (amax == 0.0f) return 0u;
   const uint64_t inv2 = f2pack(inv, inv);
   const uint64_t magic2 = f2pack(kMagic, kMagic);
-  const uint32_t w[2] = {h.x, h.y};
-  uint32_t b[4];
-  float emax = 0.0f;
-#pragma unroll
-  for (int i = 0; i < 2; ++i) {
-    const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&w[i]));
-    const uint64_t y = mul2(f2pack(f.x, f.y), inv2);
-    const uint64_t s = add2(y, magic2);
-    const uint64_t e = sub2(y, sub2(s, magic2));
-    emax = fmaxf(emax, fmaxf(fabsf(lo(e)), fabsf(hi(e))));
-    b[2 * i] = static_cast<uint32_t>(s);
-    b[2 * i + 1] = static_cast<uint32_t>(s >> 32);
-  }
-  if (emax > kTieMargin) {
-#pragma unroll
-    for (int i = 0; i < 2; ++i) {
-      const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&w[i]));
-      b[2 * i] = static_cast<uint32_t>(quant_code(f.x, amax));
-      b[2 * i + 1] = static_cast<uint32_t>(quant_code(f.y, amax));
-    }
-  }
-  return __byte_perm(__byte_perm(b[0], b[1], 0x0040), __byte_perm(b[2], b[3], 0x0040), 0x5410);
+  const float2 f0 = __half22float2(*reinterpret_cast<const __half2*>(&h.x));
+  const float2 f1 = __half22float2(*reinterpret_cast<const __half2*>(&h.y));
+  const uint64_t y0 = mul2(f2pack(f0.x, f0.y), inv2);
+  const uint64_t y1 = mul2(f2pack(f1.x, f1.y), inv2);
+  const uint64_t s0 = add2(y0, magic2);
+  const uint64_t s1 = add2(y1, magic2);
+  const uint64_t e0 = sub2(y0, sub2(s0, magic2));
+  const uint64_t e1 = sub2(y1, sub2(s1, magic2));
+  const float emax = fmaxf(fmaxf(fabsf(lo(e0)), fabsf(hi(e0))), fmaxf(fabsf(lo(e1)), fabsf(hi(e1))));
+  if (emax > kTieMargin) return codes4_exact(h.x, h.y, amax);
+  const uint32_t b0 = static_cast<uint32_t>(s0), b1 = static_cast<uint32_t>(s0 >> 32);
+  const uint32_t b2 = static_cast<uint32_t>(s1), b3 = static_cast<uint32_t>(s1 >> 32);
+  return __byte_perm(__byte_perm(b0, b1, 0x0040), __byte_perm(b2, b3, 0x0040), 0x5410);
 }
-
 }  // namespace i8mm
