@@ -7,32 +7,39 @@
 // "quantization explained part 2" section 1.2 (threshold 6.0).
 //
 // With at most 16 tokens the work is bound by reading Wq once; everything else
-// is arranged to finish while that stream is in flight. The grid is made of
-// clusters of S CTAs; a cluster owns 128 output features (rows of Wq) and its
-// CTAs split K, so every CTA reads a 128 x (K/S) slice of Wq (at most 8 blocks
-// of 128 x 128 bytes, all requested at kernel start).
+// is arranged to finish while that stream is in flight, and the per-CTA work on
+// the critical path is kept small because it runs on few warps.
 //
-// Warp roles (320 threads):
-//   warp 0     producer: bulk-copies the CTA's K-range of every token row of X
-//              (first, it is small and L2-resident), then TMA-loads the Wq slice
-//   warp 1     TMEM allocator and MMA issuer: tcgen05.mma kind::i8 with
-//              M = 128 weight rows, N = 16 tokens, one K-block as it lands
-//   warps 2-9  X workers, 4 columns per thread, all 16 tokens held in registers:
-//              exact outlier flags of their columns (every token is here),
-//              per-token maxima over the non-outlier columns, and after the
-//              cluster exchange of those maxima the INT8 codes, written straight
-//              into the 128-byte-swizzled K-major B operand of the MMA
-//   warps 4-7  also the epilogue: the fp32 outlier partials of the CTA's own
-//              outlier columns on CUDA cores (fp16 products are exact in fp32),
-//              the INT32 partials from TMEM, and the cross-CTA sum.
+// The grid is made of clusters of S <= 8 CTAs. A cluster owns 128 output
+// features (rows of Wq) and its CTAs split K, so every CTA reads a 128 x (K/S)
+// slice of Wq as nbox = 8 TMA boxes of 128 rows x 128 bytes, all requested at
+// kernel start (K = 4096: clusters of 4, one CTA per SM, all resident at once).
+// The layout also supports nbox = 4 (about 100 KB, two CTAs per SM, clusters of
+// 8); that variant measured slower because the launch of its 256 CTAs spread
+// over about 2 us.
+//
+// Warp roles (64 + 32*nxw threads, nxw = 2*nbox X workers):
+//   warp 0        barrier set-up and the copies: the CTA's K-range of X (2-D
+//                 boxes; tokens past M read as zeros), then the Wq slice
+//   warp 1        TMEM allocator and MMA issuer: tcgen05.mma kind::i8,
+//                 M = 128 weight rows, N = 16 tokens, issued by an elected lane
+//   X workers     2 columns per thread, loops over the tokens: exact outlier
+//                 flags (every token is here), per-token maxima over the
+//                 non-outlier columns (one redux per token and warp), and after
+//                 the cluster exchange of those maxima the INT8 codes, written
+//                 into the 128-byte-swizzled K-major B operand of the MMA
+//   warps 4-7     (X workers too) the epilogue: the fp32 outlier partials of the
+//                 CTA's own outlier columns on CUDA cores (fp16 products are
+//                 exact in fp32), the INT32 partials from TMEM dequantised with
+//                 the row and column scales, and the cross-CTA sum.
 //
 // Cross-CTA traffic uses st.async into the peer's shared memory, counted in
 // bytes on the peer's mbarrier: one 80-byte message per CTA pair with the
-// per-token maxima and the outlier count, then each CTA pushes every row's
-// 16 INT32 + 16 fp32 partials to the CTA that finishes that row, which sums the
-// S partials in rank order and writes Y. A split cluster barrier only publishes
-// the mbarrier initialisation and keeps every CTA alive until its peers have
-// issued their last store into it. Cluster 0 also writes the intermediates the
+// per-token maxima and the outlier count; then each CTA pushes every row's 16
+// fp32 partial results to the CTA that finishes that row, which adds the S
+// partials in rank order and writes Y. A split cluster barrier publishes the
+// mbarrier initialisation and keeps every CTA alive until its peers have issued
+// their last store into it. Cluster 0 also writes the intermediates the
 // workspace documents (bitmap, count, ascending outlier list, x_scale, Xq).
 // No TMA multicast is used.
 #include <cuda.h>
@@ -50,44 +57,47 @@ namespace i8mm {
 
 namespace {
 
-constexpr int kRows = 128;                    // Wq rows (output features) per cluster = MMA M
+constexpr int kTileRows = 128;                // MMA M = output rows per cluster
 constexpr int kKB = 128;                      // int8 columns per K-block (one swizzle row)
-constexpr int kMaxBlocks = 8;                 // K-blocks per CTA, all in flight at once
-constexpr int kCols = kMaxBlocks * kKB;       // columns per CTA at most
+constexpr int kMaxBoxes = 8;                  // Wq boxes (128 x 128 B) per CTA, all in flight
+constexpr int kBoxBytes = kTileRows * kKB;
 constexpr int kTok = 16;                      // MMA N: tokens, zero-padded
 constexpr int kMaxCluster = 8;
-constexpr int kXWarps = 8;                    // X workers: 4 columns per thread
-constexpr int kXThreads = kXWarps * 32;
-constexpr int kThreads = 64 + kXThreads;
+constexpr int kMaxCols = kMaxBoxes * kKB;     // columns per CTA at most
+constexpr int kXBox = 256;                    // fp16 columns per X box
+constexpr int kMaxXWarps = kMaxCols / 64;     // 2 columns per thread
 constexpr int kMsgWords = 20;                 // exchange message: 16 maxima, count, pad
-constexpr int kRecvRows = kRows + kMaxCluster;   // S * ceil(128 / S) <= 135
+constexpr int kRecvRows = kTileRows + kMaxCluster;   // S * ceil(128 / S) <= 128 + S - 1
 constexpr int kWPrefetch = 8;                 // outlier weights gathered ahead per row
 constexpr int kStatusTimeout = -5;
 
-static_assert(kXThreads * 4 == kCols, "X workers cover the CTA's columns");
-
 // Named barriers (0 is __syncthreads).
 constexpr uint32_t kBarX = 1;       // the X workers
-constexpr uint32_t kBarList = 2;    // warp 2 publishes the local outlier list to warps 4-7
-constexpr uint32_t kBarEpi = 3;     // warps 4-7
+constexpr uint32_t kBarList = 2;    // the first X warp publishes the outlier list to warps 4-7
 
+// Shared-memory layout for nbox Wq boxes per CTA (offsets from a 1024-byte
+// aligned base).
 struct DecodeSmem {
-  static constexpr int RING = 0;                                // [8][128][128] i8 (swizzled)
-  static constexpr int BOP = RING + kMaxBlocks * kRows * kKB;   // [8][16][128] i8 (swizzled)
-  static constexpr int XS = BOP + kMaxBlocks * kTok * kKB;      // [16][kw] f16
-  static constexpr int RECV = XS + kTok * kCols * 2;            // [kRecvRows][8][16 B]
-  static constexpr int MSG = RECV + kRecvRows * 128;            // [8 ranks][20] words
-  static constexpr int BITS = MSG + kMaxCluster * kMsgWords * 4;   // [32] u32
-  static constexpr int LIDX = BITS + 32 * 4;                    // [1024] u16
-  static constexpr int RED = LIDX + kCols * 2;                  // [8 warps][16] f32
-  static constexpr int TOK = RED + kXWarps * kTok * 4;          // amax[16], inv[16] f32
-  static constexpr int WSC = TOK + 2 * kTok * 4;                // [128] f32 w_scale of owned rows
-  static constexpr int MISC = WSC + kRows * 4;                  // lcount, prefix
-  static constexpr int BARS = MISC + 16;                        // full[8] xbar codes done xchg red
-  static constexpr int TSLOT = BARS + (kMaxBlocks + 5) * 8;
-  static constexpr int TOTAL = TSLOT + 16;
-  static constexpr int BYTES = TOTAL + 1024;                    // alignment slack
+  int ring, bop, xs, recv, msg, bits, lidx, red, tok, misc, bars, tslot, bytes;
 };
+__host__ __device__ inline DecodeSmem decode_layout(int nbox) {
+  DecodeSmem L;
+  int off = 0;
+  L.ring = off;  off += nbox * kBoxBytes;                 // [nbox] Wq boxes (swizzled)
+  L.bop = off;   off += nbox * kTok * kKB;                // [nbox][16][128] i8 (swizzled)
+  L.xs = off;    off += nbox * kKB * kTok * 2;            // [nbox/2][16][256] f16
+  L.recv = off;  off += kRecvRows * 64;                   // [rows][4][16 B] fp32 partials
+  L.msg = off;   off += kMaxCluster * kMsgWords * 4;      // [8 ranks][20] words
+  L.bits = off;  off += 32 * 4;                           // outlier bitmap of the columns
+  L.lidx = off;  off += kMaxCols * 2;                     // ascending outlier list
+  L.red = off;   off += kMaxXWarps * kTok * 4;            // [warps][16] f32
+  L.tok = off;   off += 3 * kTok * 4;                     // amax, amax/127^2, 1/amax
+  L.misc = off;  off += 16;                               // lcount, prefix
+  L.bars = off;  off += (kMaxBoxes + 5) * 8;              // full[8] xbar codes done xchg red
+  L.tslot = off; off += 16;
+  L.bytes = off + 1024;                                   // alignment slack
+  return L;
+}
 
 __device__ __forceinline__ uint32_t cluster_nctarank() {
   uint32_t r;
@@ -95,78 +105,79 @@ __device__ __forceinline__ uint32_t cluster_nctarank() {
   return r;
 }
 
-// Rows finished (owned) by `rank` when 128 rows are dealt out rpr at a time.
+// Rows finished (owned) by `rank` when the 128 rows are dealt out rpr at a time.
 __device__ __forceinline__ int owned_rows(int rank, int rpr) {
-  return max(0, min(rpr, kRows - rank * rpr));
+  return max(0, min(rpr, kTileRows - rank * rpr));
 }
 
-__global__ void __launch_bounds__(kThreads, 1)
-    decode_kernel(const __grid_constant__ CUtensorMap tmWq, DecodeArgs a) {
+__global__ void __launch_bounds__(64 + 32 * kMaxXWarps, 1)
+    decode_kernel(const __grid_constant__ CUtensorMap tmWq, const __grid_constant__ CUtensorMap tmX,
+                  DecodeArgs a) {
   extern __shared__ __align__(1024) uint8_t dsm_raw[];
-  // 1024-byte aligned base (swizzle atoms). Derived by an offset from the
-  // shared array, not through an integer cast, so every pointer below stays in
-  // the shared state space and compiles to shared-memory loads and stores.
+  // 1024-byte aligned base, derived by an offset so pointers stay in the shared space.
   uint8_t* sm = dsm_raw + ((1024u - (smem_addr(dsm_raw) & 1023u)) & 1023u);
-  using L = DecodeSmem;
-  uint8_t* ring = sm + L::RING;
-  uint8_t* bop = sm + L::BOP;
-  __half* xs = reinterpret_cast<__half*>(sm + L::XS);
-  uint8_t* recv = sm + L::RECV;
-  uint32_t* msg = reinterpret_cast<uint32_t*>(sm + L::MSG);
-  uint32_t* bits = reinterpret_cast<uint32_t*>(sm + L::BITS);
-  uint16_t* lidx = reinterpret_cast<uint16_t*>(sm + L::LIDX);
-  float* red = reinterpret_cast<float*>(sm + L::RED);
-  float* amax_s = reinterpret_cast<float*>(sm + L::TOK);
-  float* inv_s = amax_s + kTok;
-  float* wsc = reinterpret_cast<float*>(sm + L::WSC);
-  int32_t* misc = reinterpret_cast<int32_t*>(sm + L::MISC);
-  uint64_t* full = reinterpret_cast<uint64_t*>(sm + L::BARS);
-  uint64_t* xbar = full + kMaxBlocks;
+  const int nbox = a.nbox;                              // 4 or 8
+  const DecodeSmem L = decode_layout(nbox);
+  uint8_t* ring = sm + L.ring;
+  uint8_t* bop = sm + L.bop;
+  __half* xs = reinterpret_cast<__half*>(sm + L.xs);
+  uint8_t* recv = sm + L.recv;
+  uint32_t* msg = reinterpret_cast<uint32_t*>(sm + L.msg);
+  uint32_t* bits = reinterpret_cast<uint32_t*>(sm + L.bits);
+  uint16_t* lidx = reinterpret_cast<uint16_t*>(sm + L.lidx);
+  float* red = reinterpret_cast<float*>(sm + L.red);
+  float* amax_s = reinterpret_cast<float*>(sm + L.tok);
+  float* rs_s = amax_s + kTok;
+  float* ra_s = amax_s + 2 * kTok;
+  int32_t* misc = reinterpret_cast<int32_t*>(sm + L.misc);
+  uint64_t* full = reinterpret_cast<uint64_t*>(sm + L.bars);
+  uint64_t* xbar = full + kMaxBoxes;
   uint64_t* codes_bar = xbar + 1;
   uint64_t* done = xbar + 2;
   uint64_t* xchg = xbar + 3;
   uint64_t* redbar = xbar + 4;
-  uint32_t* tslot = reinterpret_cast<uint32_t*>(sm + L::TSLOT);
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(sm + L.tslot);
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
   const int lane = tid & 31;
   const int S = static_cast<int>(cluster_nctarank());
   const int rank = static_cast<int>(cluster_ctarank());
+  const int nxw = 2 * nbox;                             // X worker warps
+  const int nxt = 32 * nxw;
   const int tile = blockIdx.x / S;
-  const int n0 = tile * kRows;
+  const int n0 = tile * kTileRows;
   const int M = a.M, N = a.N, K = a.K;
   const int nkb = (K + kKB - 1) / kKB;
   const int bper = (nkb + S - 1) / S;
   const int kb0 = min(nkb, rank * bper);
-  const int nb = min(nkb, kb0 + bper) - kb0;            // K-blocks of this CTA (1..8)
+  const int nb = min(nkb, kb0 + bper) - kb0;            // K-blocks of this CTA (1..nbox)
   const int k0 = min(K, kb0 * kKB);
   const int kw = min(K, (kb0 + nb) * kKB) - k0;         // columns of this CTA
-  const int rpr = (kRows + S - 1) / S;                  // rows finished per rank
+  const int nbx = (kw + kXBox - 1) / kXBox;             // X boxes
+  const int rpr = (kTileRows + S - 1) / S;              // rows finished per rank
   const bool writer = (tile == 0);                      // cluster 0 writes intermediates
 
   if (tid == 0) {
-    for (int b = 0; b < kMaxBlocks; ++b) mbar_init(&full[b], 1);
+    for (int b = 0; b < kMaxBoxes; ++b) mbar_init(&full[b], 1);
     mbar_init(xbar, 1);
-    mbar_init(codes_bar, kXWarps);
+    mbar_init(codes_bar, nxw);
     mbar_init(done, 1);
     mbar_init(xchg, 1);
     mbar_init(redbar, 1);
     // The peers' stores are counted in bytes; the one local arrival is made now.
     mbar_arrive_expect_tx(xchg, static_cast<uint32_t>(S * kMsgWords * 4));
-    mbar_arrive_expect_tx(redbar, static_cast<uint32_t>(S * owned_rows(rank, rpr) * 128));
+    mbar_arrive_expect_tx(redbar, static_cast<uint32_t>(S * owned_rows(rank, rpr) * 64));
     fence_mbarrier_init();
     if (blockIdx.x == 0 && a.status) *a.status = 0;
-    // Producer: X first (small, L2-resident after the first cluster), then the
-    // whole Wq slice. Issued before the CTA barrier: only this thread has used
-    // the barriers so far.
-    mbar_arrive_expect_tx(xbar, static_cast<uint32_t>(M * kw * 2));
-    for (int t = 0; t < M; ++t)
-      bulk_load(xs + t * kw, a.X + static_cast<size_t>(t) * K + k0, static_cast<uint32_t>(kw * 2),
-                xbar);
+    // X first (small, L2-resident after the first cluster), then the Wq slice.
+    // Issued before the CTA barrier: only this thread has used the barriers.
+    mbar_arrive_expect_tx(xbar, static_cast<uint32_t>(nbx * kTok * kXBox * 2));
+    for (int j = 0; j < nbx; ++j)
+      tma_load_2d(xs + j * kTok * kXBox, &tmX, xbar, k0 + j * kXBox, 0);
     for (int b = 0; b < nb; ++b) {
-      mbar_arrive_expect_tx(&full[b], kRows * kKB);
-      tma_load_2d(ring + b * kRows * kKB, &tmWq, &full[b], (kb0 + b) * kKB, n0);
+      mbar_arrive_expect_tx(&full[b], kBoxBytes);
+      tma_load_2d(ring + b * kBoxBytes, &tmWq, &full[b], (kb0 + b) * kKB, n0);
     }
   }
   if (warp == 1) {
@@ -181,80 +192,79 @@ __global__ void __launch_bounds__(kThreads, 1)
   bool ok = true;
 
   if (warp == 0) {
-    // ---------------------------------------------------------------- producer (done)
     cluster_wait();
     cluster_arrive();
   } else if (warp == 1) {
     // ---------------------------------------------------------------- MMA issuer
-    // The whole warp runs the loop; one elected lane issues each MMA.
     cluster_wait();
     ok = __all_sync(0xffffffffu, mbar_wait(codes_bar, 0));
-    constexpr uint32_t idesc = make_idesc(2 /*s32*/, 1 /*signed*/, kRows, kTok);
+    // Orders the MMAs after the X workers' code stores (a thread sync). The
+    // Wq boxes come from TMA and need only their mbarrier.
+    tc_fence_after();
+    constexpr uint32_t idesc = make_idesc(2 /*s32*/, 1 /*signed*/, kTileRows, kTok);
     const uint64_t a0 = sw128_kmajor_desc(smem_addr(ring));
     const uint64_t b0 = sw128_kmajor_desc(smem_addr(bop));
     for (int b = 0; b < nb && ok; ++b) {
       ok = __all_sync(0xffffffffu, mbar_wait(&full[b], 0));
       if (!ok) break;
-      tc_fence_after();
 #pragma unroll
       for (int kk = 0; kk < 4; ++kk)
-        mma_i8_elect(tmem, a0 + static_cast<uint64_t>((b * kRows * kKB + 32 * kk) >> 4),
+        mma_i8_elect(tmem, a0 + static_cast<uint64_t>((b * kBoxBytes + 32 * kk) >> 4),
                      b0 + static_cast<uint64_t>((b * kTok * kKB + 32 * kk) >> 4), idesc,
                      (b | kk) != 0);
     }
     // Always committed, so the epilogue's wait ends even after a failed wait here.
     mma_commit_elect(done);
     cluster_arrive();
+  } else if (warp - 2 >= nxw) {
+    cluster_wait();
+    cluster_arrive();
   } else {
     // ---------------------------------------------------------------- X workers
-    // Loops over tokens stay rolled: this code runs once per launch, and
-    // straight-line code would be bound by instruction fetch.
-    const int xw = warp - 2;                 // 0..7
-    const int xi = tid - 64;                 // 0..255
-    const int c0 = 4 * xi;                   // first of the thread's 4 columns (CTA-local)
+    // Loops over tokens stay rolled: this code runs once per launch on few
+    // warps, and straight-line code would be bound by instruction fetch.
+    const int xw = warp - 2;
+    const int xi = tid - 64;
+    const int c0 = 2 * xi;                   // the thread's 2 columns (CTA-local)
     const bool cv = c0 < kw;                 // kw is a multiple of 16
     const float thr = a.threshold;
     const bool epi = (warp >= 4 && warp < 8);
-    const int r = (warp & 3) * 32 + lane;    // epilogue: tile row = TMEM lane
-    const uint2* xrow = reinterpret_cast<const uint2*>(xs) + xi;   // + t * (kw / 4)
-    const int xstride = kw >> 2;             // uint2 per token row
+    // Column pair c0 of token t: box c0/256, row t, column c0%256.
+    const uint32_t* xcol =
+        reinterpret_cast<const uint32_t*>(xs + (c0 >> 8) * (kTok * kXBox) + (c0 & (kXBox - 1)));
+    constexpr int xstride = kXBox / 2;       // uint32 per token row of a box
 
     ok = __all_sync(0xffffffffu, mbar_wait(xbar, 0));
 
-    // Outlier flags of the 4 columns: the max of |x| over all tokens against the threshold.
-    __half2 m01 = __float2half2_rn(0.0f), m23 = m01;
+    // Outlier flags of the 2 columns: the max of |x| over all tokens against the threshold.
+    __half2 cm = __float2half2_rn(0.0f);
     if (cv) {
 #pragma unroll 4
-      for (int t = 0; t < M; ++t) {
-        const uint2 v = xrow[t * xstride];
-        m01 = __hmax2(m01, habs2_bits(v.x));
-        m23 = __hmax2(m23, habs2_bits(v.y));
-      }
+      for (int t = 0; t < M; ++t) cm = __hmax2(cm, habs2_bits(xcol[t * xstride]));
     }
-    const float2 f01 = __half22float2(m01), f23 = __half22float2(m23);
-    const uint32_t f4 = (f01.x > thr ? 1u : 0u) | (f01.y > thr ? 2u : 0u) |
-                        (f23.x > thr ? 4u : 0u) | (f23.y > thr ? 8u : 0u);
-    const uint32_t keep0 = ((f4 & 1u) ? 0u : 0x0000FFFFu) | ((f4 & 2u) ? 0u : 0xFFFF0000u);
-    const uint32_t keep1 = ((f4 & 4u) ? 0u : 0x0000FFFFu) | ((f4 & 8u) ? 0u : 0xFFFF0000u);
-    // Bitmap word of 32 columns = 8 threads x 4 flags.
+    const float2 cf = __half22float2(cm);
+    const uint32_t f2 = (cf.x > thr ? 1u : 0u) | (cf.y > thr ? 2u : 0u);
+    const uint32_t keep = ((f2 & 1u) ? 0u : 0x0000FFFFu) | ((f2 & 2u) ? 0u : 0xFFFF0000u);
+    const uint32_t keepq = ((f2 & 1u) ? 0u : 0x00FFu) | ((f2 & 2u) ? 0u : 0xFF00u);
     {
-      uint32_t word = f4 << (4 * (lane & 7));
+      // Bitmap word of 32 columns = 16 threads x 2 flags.
+      uint32_t word = f2 << (2 * (lane & 15));
       word |= __shfl_xor_sync(0xffffffffu, word, 1);
       word |= __shfl_xor_sync(0xffffffffu, word, 2);
       word |= __shfl_xor_sync(0xffffffffu, word, 4);
-      if ((lane & 7) == 0) bits[xi >> 3] = word;
+      word |= __shfl_xor_sync(0xffffffffu, word, 8);
+      if ((lane & 15) == 0) bits[xi >> 4] = word;
     }
-    // Per-token max of |x| over the non-outlier columns: per thread, then over
-    // the warp (non-negative floats order like their bit patterns).
+    // Per-token max of |x| over the non-outlier columns, per warp with one
+    // redux (non-negative floats order like their bit patterns).
 #pragma unroll 2
     for (int t = 0; t < M; ++t) {
-      const uint2 v = cv ? xrow[t * xstride] : make_uint2(0u, 0u);
-      const __half2 m = __hmax2(habs2_bits(v.x & keep0), habs2_bits(v.y & keep1));
-      const float pm = fmaxf(__low2float(m), __high2float(m));
-      const uint32_t wm = __reduce_max_sync(0xffffffffu, __float_as_uint(pm));
+      const uint32_t v = cv ? xcol[t * xstride] : 0u;
+      const float2 f = __half22float2(habs2_bits(v & keep));
+      const uint32_t wm = __reduce_max_sync(0xffffffffu, __float_as_uint(fmaxf(f.x, f.y)));
       if (lane == 0) red[xw * kTok + t] = __uint_as_float(wm);
     }
-    named_bar_sync(kBarX, kXThreads);
+    named_bar_sync(kBarX, nxt);
 
     if (xw == 0) {
       // Local outlier list (ascending) and count; then the message to every rank.
@@ -276,14 +286,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       const int lcount = __shfl_sync(0xffffffffu, incl, 31);
       // CTA maxima of the tokens (0 for the padding tokens).
-      float cm = 0.0f;
+      float cmx = 0.0f;
       if (lane < M) {
-        for (int w = 0; w < kXWarps; ++w) cm = fmaxf(cm, red[w * kTok + lane]);
+        for (int w = 0; w < nxw; ++w) cmx = fmaxf(cmx, red[w * kTok + lane]);
       }
       if (lane == 0) misc[0] = lcount;
       __syncwarp();
       // Lane l alone read red[w][l]; its CTA maximum replaces red[0][l].
-      if (lane < kTok) red[lane] = cm;
+      if (lane < kTok) red[lane] = cmx;
       __syncwarp();
       named_bar_arrive(kBarList, 32 + 128);
       cluster_wait();   // every CTA's barriers are initialised
@@ -304,23 +314,22 @@ __global__ void __launch_bounds__(kThreads, 1)
       cluster_wait();
     }
 
-    // Epilogue warps: start the gathers of the outlier weights now, they have
-    // the whole exchange and the code pass to land.
+    // Epilogue warps: start the gathers of the outlier weights and the column
+    // scales now; they have the exchange and the code pass to land.
+    const int q = warp & 3;
+    const int r = q * 32 + lane;             // epilogue: row of the cluster = TMEM lane
+    const int n = n0 + r;
     int lcount = 0;
     __half wv[kWPrefetch];
+    float wsr = 0.0f;
     if (epi) {
       named_bar_sync(kBarList, 32 + 128);
       lcount = misc[0];
-      const int n = n0 + r;
-      const __half* wrow = a.W + static_cast<size_t>(min(n, N - 1)) * K + k0;
+      const __half* wrow = a.W + static_cast<size_t>(n < N ? n : 0) * K + k0;
 #pragma unroll
-      for (int j = 0; j < kWPrefetch; ++j)
-        wv[j] = (j < lcount && n < N) ? wrow[lidx[j]] : __float2half(0.0f);
-      const int owned = owned_rows(rank, rpr);
-      if (r < owned) {
-        const int nr = n0 + rank * rpr + r;
-        wsc[r] = (nr < N) ? a.w_scale[nr] : 0.0f;
-      }
+      for (int i = 0; i < kWPrefetch; ++i)
+        wv[i] = (n < N && i < lcount) ? wrow[lidx[i]] : __float2half(0.0f);
+      wsr = (n < N) ? a.w_scale[n] : 0.0f;
     }
 
     // Token absmax over the whole cluster, its inverse, the outlier prefix.
@@ -330,7 +339,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         float m = 0.0f;
         for (int s2 = 0; s2 < S; ++s2) m = fmaxf(m, __uint_as_float(msg[s2 * kMsgWords + lane]));
         amax_s[lane] = m;
-        inv_s[lane] = quant_inv(m);
+        rs_s[lane] = m * (1.0f / 16129.0f);
+        ra_s[lane] = quant_rcp(m);
         if (writer && rank == 0 && lane < M) a.x_scale[lane] = m;
       }
       if (lane == 0) {
@@ -344,29 +354,29 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (writer && rank == 0) *a.n_outliers = total;
       }
     }
-    named_bar_sync(kBarX, kXThreads);
+    named_bar_sync(kBarX, nxt);
 
     if (writer) {
       if (xi < ((kw + 31) >> 5)) a.bitmap[(k0 >> 5) + xi] = bits[xi];
       const int lc = misc[0], prefix = misc[1];
-      for (int i = xi; i < lc; i += kXThreads) a.col_idx[prefix + i] = k0 + lidx[i];
+      for (int i = xi; i < lc; i += nxt) a.col_idx[prefix + i] = k0 + lidx[i];
     }
 
-    // INT8 codes of the 4 columns for every token, into the B operand (and Xq).
+    // INT8 codes of the 2 columns for every token, into the B operand (and Xq).
     if (c0 < nb * kKB) {
       const uint32_t kc = static_cast<uint32_t>(c0) & 127u;
       uint8_t* dst = bop + (c0 >> 7) * (kTok * kKB) + (kc & 15u);
-      const uint32_t keepq = keep_bytes(f4);
       int8_t* xq = a.Xq + k0 + c0;
 #pragma unroll 2
       for (int t = 0; t < kTok; ++t) {
-        uint32_t q = 0u;
+        uint32_t qv = 0u;
         if (cv && t < M) {
-          q = codes4(xrow[t * xstride], amax_s[t], inv_s[t]) & keepq;
-          if (writer) *reinterpret_cast<uint32_t*>(xq + static_cast<size_t>(t) * K) = q;
+          qv = codes2(xcol[t * xstride], amax_s[t], ra_s[t]) & keepq;
+          if (writer)
+            *reinterpret_cast<uint16_t*>(xq + static_cast<size_t>(t) * K) = static_cast<uint16_t>(qv);
         }
         const uint32_t off = (t >> 3) * 1024 + (t & 7) * 128 + (((kc >> 4) ^ (t & 7)) << 4);
-        *reinterpret_cast<uint32_t*>(dst + off) = q;
+        *reinterpret_cast<uint16_t*>(dst + off) = static_cast<uint16_t>(qv);
       }
     }
     fence_proxy_async_smem();   // the tensor core reads what the generic proxy wrote
@@ -380,79 +390,73 @@ __global__ void __launch_bounds__(kThreads, 1)
       float o[kTok];
 #pragma unroll
       for (int t = 0; t < kTok; ++t) o[t] = 0.0f;
-      const int n = n0 + r;
-      const __half* wrow = a.W + static_cast<size_t>(min(n, N - 1)) * K + k0;
+      const __half* wrow = a.W + static_cast<size_t>(n < N ? n : 0) * K + k0;
 #pragma unroll 1
-      for (int j = 0; j < lcount; ++j) {
-        const int col = lidx[j];
+      for (int jj = 0; jj < lcount; ++jj) {
+        const int col = lidx[jj];
         __half wh = __float2half(0.0f);
 #pragma unroll
         for (int i = 0; i < kWPrefetch; ++i)
-          if (i == j) wh = wv[i];
-        if (j >= kWPrefetch && n < N) wh = wrow[col];
+          if (i == jj) wh = wv[i];
+        if (jj >= kWPrefetch && n < N) wh = wrow[col];
         const float w = __half2float(wh);
+        const __half* xc = xs + (col >> 8) * (kTok * kXBox) + (col & (kXBox - 1));
 #pragma unroll
         for (int t = 0; t < kTok; ++t)
-          if (t < M) o[t] = fmaf(__half2float(xs[t * kw + col]), w, o[t]);
+          if (t < M) o[t] = fmaf(__half2float(xc[t * kXBox]), w, o[t]);
       }
-
-      // INT32 partials of the row from TMEM.
-      uint32_t acc[kTok];
+      // INT32 partials of the row from TMEM, dequantised with the scales.
       const bool got = __all_sync(0xffffffffu, mbar_wait(done, 0));
+      ok = ok && got;
+      uint32_t acc[kTok];
       if (got) {
         tc_fence_after();
-        tmem_ld_32x32b_x16(tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16), acc);
+        tmem_ld_32x32b_x16(tmem + (static_cast<uint32_t>(q * 32) << 16), acc);
         tmem_ld_wait();
       } else {
 #pragma unroll
         for (int t = 0; t < kTok; ++t) acc[t] = 0u;
       }
-      ok = ok && got;
-
-      // Push the row's partials to the rank that finishes it: 8 chunks of 16 B,
-      // chunk c at position c ^ (row & 7) to spread the banks of the final reads.
+      float y[kTok];
+#pragma unroll
+      for (int t = 0; t < kTok; ++t)
+        y[t] = static_cast<float>(static_cast<int32_t>(acc[t])) * (rs_s[t] * wsr) + o[t];
+      // Push to the rank that finishes the row: 4 chunks of 16 B, chunk c at
+      // position c ^ (row & 3) to spread the banks of the final reads.
       {
         const int own = r / rpr, rl = r - own * rpr;
-        const uint32_t base = cluster_addr(recv + (rank * rpr + rl) * 128, own);
+        const uint32_t base = cluster_addr(recv + (rank * rpr + rl) * 64, own);
         const uint32_t bar = cluster_addr(redbar, own);
 #pragma unroll
-        for (int ch = 0; ch < 8; ++ch) {
-          const uint32_t pos = static_cast<uint32_t>(ch ^ (rl & 7)) << 4;
-          if (ch < 4)
-            st_async_v4(base + pos, acc[4 * ch], acc[4 * ch + 1], acc[4 * ch + 2], acc[4 * ch + 3],
-                        bar);
-          else
-            st_async_v4(base + pos, __float_as_uint(o[4 * (ch - 4)]),
-                        __float_as_uint(o[4 * (ch - 4) + 1]), __float_as_uint(o[4 * (ch - 4) + 2]),
-                        __float_as_uint(o[4 * (ch - 4) + 3]), bar);
-        }
+        for (int ch = 0; ch < 4; ++ch)
+          st_async_v4(base + (static_cast<uint32_t>(ch ^ (rl & 3)) << 4),
+                      __float_as_uint(y[4 * ch]), __float_as_uint(y[4 * ch + 1]),
+                      __float_as_uint(y[4 * ch + 2]), __float_as_uint(y[4 * ch + 3]), bar);
       }
       cluster_arrive();
 
-      // Finish the owned rows: sum the S partials in rank order, dequantise, add.
+      // Finish the owned rows: add the S partials in rank order, write Y.
       ok = __all_sync(0xffffffffu, mbar_wait(redbar, 0)) && ok;
-      named_bar_sync(kBarEpi, 128);   // wsc of all owned rows is written
       const int owned = owned_rows(rank, rpr);
-      const int32_t* ri = reinterpret_cast<const int32_t*>(recv);
-      const float* rf = reinterpret_cast<const float*>(recv);
+      const float4* rv = reinterpret_cast<const float4*>(recv);
 #pragma unroll 1
-      for (int e = (warp & 3) * 32 + lane; e < owned * kTok; e += 128) {
-        const int t = e / owned;
-        const int rl = e - t * owned;
+      for (int e = q * 32 + lane; e < owned * 4; e += 128) {
+        const int tg = e / owned;               // tokens 4tg..4tg+3
+        const int rl = e - tg * owned;
         const int nn = n0 + rank * rpr + rl;
-        if (t < M && nn < N) {
-          const int pi = (((t >> 2) ^ (rl & 7)) << 2) + (t & 3);
-          const int pf = (((4 + (t >> 2)) ^ (rl & 7)) << 2) + (t & 3);
-          int32_t c = 0;
-          float of = 0.0f;
-          for (int s2 = 0; s2 < S; ++s2) {
-            const int row = (s2 * rpr + rl) * 32;
-            c += ri[row + pi];
-            of += rf[row + pf];
-          }
-          const float rs = amax_s[t] * (1.0f / 16129.0f);
-          const float y = static_cast<float>(c) * (rs * wsc[rl]) + of;
-          a.Y[static_cast<size_t>(t) * N + nn] = __float2half_rn(y);
+        float4 sum = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+        for (int s2 = 0; s2 < S; ++s2) {
+          const float4 v = rv[(s2 * rpr + rl) * 4 + (tg ^ (rl & 3))];
+          sum.x += v.x;
+          sum.y += v.y;
+          sum.z += v.z;
+          sum.w += v.w;
+        }
+        if (nn < N) {
+          const float sv[4] = {sum.x, sum.y, sum.z, sum.w};
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+            if (4 * tg + i < M) a.Y[static_cast<size_t>(4 * tg + i) * N + nn] = __float2half_rn(sv[i]);
         }
       }
     }
@@ -471,33 +475,42 @@ __global__ void __launch_bounds__(kThreads, 1)
 }  // namespace
 
 bool decode_supported(int M, int K) {
-  return M >= 1 && M <= kTok && K <= kMaxCluster * kMaxBlocks * kKB;
+  return M >= 1 && M <= kTok && K <= kMaxCluster * kMaxBoxes * kKB;
 }
 
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t s) {
-  CUtensorMap tm;
-  std::memset(&tm, 0, sizeof(tm));
-  if (!make_tmap_sw128(&tm, a.Wq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.K, a.N, kRows))
-    return cudaErrorInvalidValue;
   const int nkb = (a.K + kKB - 1) / kKB;
-  int S = (nkb + kMaxBlocks - 1) / kMaxBlocks;          // CTAs per cluster
-  if (S < 1) S = 1;
+  // Eight boxes per CTA: clusters of 4 (K = 4096) are all resident with one CTA
+  // per SM and start together; four boxes per CTA (clusters of 8, two CTAs per
+  // SM) measured slower, their launch spread over about 2 us.
+  const int nbox = kMaxBoxes;
+  const int S = max(1, (nkb + nbox - 1) / nbox);        // CTAs per cluster
   if (S > kMaxCluster) return cudaErrorInvalidValue;
-  const int tiles = (a.N + kRows - 1) / kRows;
-  static bool attr_set[64] = {};
+  const int tiles = (a.N + kTileRows - 1) / kTileRows;
+  CUtensorMap tmw, tmx;
+  std::memset(&tmw, 0, sizeof(tmw));
+  std::memset(&tmx, 0, sizeof(tmx));
+  if (!make_tmap_sw128(&tmw, a.Wq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.K, a.N, kTileRows))
+    return cudaErrorInvalidValue;
+  // X boxes: 16 token rows (rows past M read as zeros) x 256 fp16 columns.
+  if (!make_tmap_2d(&tmx, a.X, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, a.K, a.M, kTok, kXBox * 2,
+                    CU_TENSOR_MAP_SWIZZLE_NONE))
+    return cudaErrorInvalidValue;
+  const int smem = decode_layout(nbox).bytes;
+  static int attr_bytes[64] = {};
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
-  if (dev >= 64 || !attr_set[dev]) {
+  if (dev >= 64 || attr_bytes[dev] < smem) {
     e = cudaFuncSetAttribute(decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             DecodeSmem::BYTES);
+                             decode_layout(kMaxBoxes).bytes);
     if (e != cudaSuccess) return e;
-    if (dev < 64) attr_set[dev] = true;
+    if (dev < 64) attr_bytes[dev] = decode_layout(kMaxBoxes).bytes;
   }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(tiles * S);
-  cfg.blockDim = dim3(kThreads);
-  cfg.dynamicSmemBytes = DecodeSmem::BYTES;
+  cfg.blockDim = dim3(64 + 32 * 2 * nbox);
+  cfg.dynamicSmemBytes = smem;
   cfg.stream = s;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -507,7 +520,8 @@ cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t s) {
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   DecodeArgs args = a;
-  e = cudaLaunchKernelEx(&cfg, decode_kernel, tm, args);
+  args.nbox = nbox;
+  e = cudaLaunchKernelEx(&cfg, decode_kernel, tmw, tmx, args);
   if (e != cudaSuccess) (void)cudaGetLastError();
   return e;
 }

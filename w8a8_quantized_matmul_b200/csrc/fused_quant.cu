@@ -66,7 +66,7 @@ __device__ __forceinline__ uint64_t gtimer() {
 //   rows    [nb][K] fp16       the rows of the current wave, filled by bulk copies
 //   bits    [words] u32        outlier bitmap
 //   prefix  [words] i32        outliers before each bitmap word
-//   red     [kWarps+1][kMaxGroup] f32   per-warp row maxima; last line = row absmax
+//   red     [kWarps+2][kMaxGroup] f32   per-warp row maxima; then row absmax, 1/absmax
 //   misc    [4] i32            running count during the scan
 //   idx     [K] u16            ascending outlier columns
 //   bar     u64                mbarrier of the bulk copies
@@ -83,7 +83,7 @@ __host__ __device__ inline FusedSmem fused_smem_layout(int K, int nb) {
   L.rows = off;   off = align16(off + static_cast<size_t>(nb) * K * 2);
   L.bits = off;   off = align16(off + words * 4);
   L.prefix = off; off = align16(off + words * 4);
-  L.red = off;    off = align16(off + static_cast<size_t>(kWarps + 1) * kMaxGroup * 4);
+  L.red = off;    off = align16(off + static_cast<size_t>(kWarps + 2) * kMaxGroup * 4);
   L.misc = off;   off = align16(off + 16);
   L.idx = off;    off = align16(off + static_cast<size_t>(K) * 2);
   L.bar = off;    off = align16(off + 8);
@@ -111,6 +111,7 @@ __global__ void __launch_bounds__(kThreads, VPT == 1 ? 2 : 1)
   int32_t* s_prefix = reinterpret_cast<int32_t*>(fsm + L.prefix);
   float* s_red = reinterpret_cast<float*>(fsm + L.red);
   float* s_row = s_red + kWarps * kMaxGroup;
+  float* s_rcp = s_row + kMaxGroup;
   int32_t* s_misc = reinterpret_cast<int32_t*>(fsm + L.misc);
   uint16_t* s_idx = reinterpret_cast<uint16_t*>(fsm + L.idx);
   uint64_t* s_bar = reinterpret_cast<uint64_t*>(fsm + L.bar);
@@ -210,86 +211,103 @@ __global__ void __launch_bounds__(kThreads, VPT == 1 ? 2 : 1)
   }
   __syncthreads();
 
-  // ---------------- phase B.1: bitmap, prefix counts and outlier list in shared memory
-  if (tid == 0) s_misc[0] = 0;
-  __syncthreads();
-  for (int base = 0; base < words; base += kThreads) {
-    const int w = base + tid;
-    const uint32_t bits = (w < words) ? __ldcg(a.bitmap + w) : 0u;
-    const int cnt = __popc(bits);
+  // ---------------- phase B.1: outlier masks of this thread's columns (the same
+  // for every row), straight from the global bitmap. Warp 0 also builds the
+  // per-word prefix counts and the ascending outlier list in shared memory; the
+  // other warps start on the row maxima meanwhile.
+  uint32_t m8[VPT];
+#pragma unroll
+  for (int c = 0; c < VPT; ++c) {
+    const int v = tid + kThreads * c;
+    m8[c] = (v < nv) ? (__ldcg(a.bitmap + (v >> 2)) >> (8 * (v & 3))) & 0xFFu : 0u;
+  }
+  // Warp 0 also builds the per-word prefix counts and the ascending outlier
+  // list in shared memory (build_list); its first bitmap words are loaded now so
+  // that their L2 round trip overlaps the row maxima below.
+  const int lper = (words + 31) >> 5;                  // words per lane
+  const int lw0 = min(words, lane * lper), lw1 = min(words, lw0 + lper);
+  uint32_t bw8[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i)
+    bw8[i] = (warp == 0 && lw0 + i < lw1) ? __ldcg(a.bitmap + lw0 + i) : 0u;
+  bool listed = false;
+  auto build_list = [&]() {
+    // Lane l scans the words [lw0, lw1): the first 8 are in bw8.
+    int cnt = 0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      if (lw0 + i < lw1) s_bits[lw0 + i] = bw8[i];
+      cnt += __popc(bw8[i]);
+    }
+    for (int wb = lw0 + 8; wb < lw1; wb += 8) {
+      uint32_t b[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) b[i] = (wb + i < lw1) ? __ldcg(a.bitmap + wb + i) : 0u;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        if (wb + i < lw1) s_bits[wb + i] = b[i];
+        cnt += __popc(b[i]);
+      }
+    }
     int incl = cnt;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
       const int t = __shfl_up_sync(0xffffffffu, incl, o);
       if (lane >= o) incl += t;
     }
-    if (lane == 31) s_red[warp] = __int_as_float(incl);
-    __syncthreads();
-    int wsum = 0;
-    for (int i = 0; i < warp; ++i) wsum += __float_as_int(s_red[i]);
-    const int excl = s_misc[0] + wsum + incl - cnt;
-    if (w < words) {
-      s_bits[w] = bits;
-      s_prefix[w] = excl;
-      uint32_t b = bits;
-      int p = excl;
+    int p = incl - cnt;
+    for (int w = lw0; w < lw1; ++w) {
+      uint32_t b = s_bits[w];
+      s_prefix[w] = p;
       while (b) {
         const int j = __ffs(b) - 1;
         b &= b - 1;
         s_idx[p++] = static_cast<uint16_t>(w * 32 + j);
       }
     }
-    __syncthreads();
-    if (tid == kThreads - 1) s_misc[0] = excl + cnt;
-    __syncthreads();
-  }
-  const int count = s_misc[0];
-  const int pad = (count + 63) & ~63;
-  if (blockIdx.x == 0) {
-    for (int p = tid; p < count; p += kThreads) a.col_idx[p] = s_idx[p];
-    if (tid == 0) *a.n_outliers = count;
-  }
-  // Compacted fp16 outlier panels: kCcMaxOutliers columns wide (zero-padded) when
-  // the GEMM epilogue adds the outlier product itself, a multiple of 64 wide when
-  // the GEMM multiplies the panels on the tensor cores.
-  const bool compact = count > 0;
-  const int pw = count > kCcMaxOutliers ? pad : kCcMaxOutliers;
+    if (lane == 31) s_misc[0] = incl;
+  };
 
-  // Outlier masks of this thread's columns (the same for every row).
-  uint32_t m8[VPT];
+  // ---------------- phase B.2: quantise, the resident wave first, then re-fetch the rest
+  int count = -1, pw = 0;
+  bool compact = false;
+  int items = 0, wn0 = 0, chunks = 0;
+  constexpr int kEarly = 2;   // W_O items per thread gathered before the quantisation
+  __half early[kEarly][8];    // kept as halves: packed only when stored, after the codes
+  // Panel geometry, the published list and the early W_O gathers, once the
+  // outlier list is complete (warp 0 wrote it before the first group barrier).
+  // The early gathers' latency overlaps the quantisation; their stores follow it.
+  auto setup_panels = [&]() {
+    count = s_misc[0];
+    compact = count > 0;
+    // Compacted fp16 outlier panels: kCcMaxOutliers columns wide (zero-padded)
+    // when the GEMM epilogue adds the outlier product itself, a multiple of 64
+    // wide when the GEMM multiplies the panels on the tensor cores.
+    pw = count > kCcMaxOutliers ? ((count + 63) & ~63) : kCcMaxOutliers;
+    if (blockIdx.x == 0) {
+      for (int p = tid; p < count; p += kThreads) a.col_idx[p] = s_idx[p];
+      if (tid == 0) *a.n_outliers = count;
+    }
+    const int nper = (a.N + gridDim.x - 1) / gridDim.x;
+    wn0 = min(a.N, static_cast<int>(blockIdx.x) * nper);
+    const int wn1 = min(a.N, wn0 + nper);
+    chunks = pw >> 3;
+    items = compact ? (wn1 - wn0) * chunks : 0;
 #pragma unroll
-  for (int c = 0; c < VPT; ++c) {
-    const int v = tid + kThreads * c;
-    m8[c] = (v < nv) ? (s_bits[v >> 2] >> (8 * (v & 3))) & 0xFFu : 0u;
-  }
-
-  // W_O gather items of this CTA (row n, 8-column chunk): the loads are issued
-  // now so that their latency overlaps the quantisation below; the stores follow it.
-  const int nper = (a.N + gridDim.x - 1) / gridDim.x;
-  const int wn0 = min(a.N, static_cast<int>(blockIdx.x) * nper);
-  const int wn1 = min(a.N, wn0 + nper);
-  const int chunks = pw >> 3;
-  const int items = compact ? (wn1 - wn0) * chunks : 0;
-  constexpr int kEarly = 2;   // items per thread gathered before the quantisation
-  uint4 early[kEarly];
-#pragma unroll
-  for (int k = 0; k < kEarly; ++k) {
-    const int it = tid + k * kThreads;
-    early[k] = make_uint4(0, 0, 0, 0);
-    if (it < items) {
-      const int n = wn0 + it / chunks;
-      const int ch = it - (n - wn0) * chunks;
-      const __half* wrow = W + static_cast<size_t>(n) * K;
-      __half* h = reinterpret_cast<__half*>(&early[k]);
+    for (int e = 0; e < kEarly; ++e) {
+      const int it = tid + e * kThreads;
+      const bool live = it < items;
+      const int n2 = live ? wn0 + it / chunks : wn0;
+      const int ch = live ? it - (n2 - wn0) * chunks : 0;
+      const __half* wrow = W + static_cast<size_t>(n2) * K;
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
         const int pidx = ch * 8 + i;
-        h[i] = (pidx < count) ? wrow[s_idx[pidx]] : __float2half_rn(0.0f);
+        early[e][i] = (live && pidx < count) ? wrow[s_idx[pidx]] : __float2half_rn(0.0f);
       }
     }
-  }
+  };
 
-  // ---------------- phase B.2: quantise, the resident wave first, then re-fetch the rest
   for (int k = 0; k < nwaves; ++k) {
     const int w = (k == 0) ? nwaves - 1 : k - 1;
     const int wb = r0 + w * wave_rows;
@@ -298,88 +316,85 @@ __global__ void __launch_bounds__(kThreads, VPT == 1 ? 2 : 1)
       __syncthreads();
       n = fetch(w);
     }
-    // Row absmax over the non-outlier columns, for up to kMaxGroup rows at once.
     for (int gb = 0; gb < n; gb += kMaxGroup) {
       const int ng = min(kMaxGroup, n - gb);
-      float part[kMaxGroup];
+      // Row absmax over the non-outlier columns: per thread, then per warp with
+      // one redux (non-negative floats order like their bit patterns).
+#pragma unroll 1
+      for (int g = 0; g < ng; ++g) {
+        const uint4* srow = reinterpret_cast<const uint4*>(s_rows + (gb + g) * row_bytes);
+        __half2 h = __float2half2_rn(0.0f);
 #pragma unroll
-      for (int g = 0; g < kMaxGroup; ++g) {
-        part[g] = 0.0f;
-        if (g < ng) {
-          const uint4* srow = reinterpret_cast<const uint4*>(s_rows + (gb + g) * row_bytes);
-          __half2 h = __float2half2_rn(0.0f);
+        for (int c = 0; c < VPT; ++c) {
+          const int v = tid + kThreads * c;
+          if (v < nv) {
+            const uint4 u = srow[v];
+            const uint32_t* wd = reinterpret_cast<const uint32_t*>(&u);
+            if (m8[c] == 0u) {
 #pragma unroll
-          for (int c = 0; c < VPT; ++c) {
-            const int v = tid + kThreads * c;
-            if (v < nv) {
-              const uint4 u = srow[v];
-              const uint32_t* wd = reinterpret_cast<const uint32_t*>(&u);
-              if (m8[c] == 0u) {
+              for (int i = 0; i < 4; ++i) h = __hmax2(h, habs2_bits(wd[i]));
+            } else {
 #pragma unroll
-                for (int i = 0; i < 4; ++i) h = __hmax2(h, habs2_bits(wd[i]));
-              } else {
-#pragma unroll
-                for (int i = 0; i < 4; ++i) h = __hmax2(h, habs2_bits(wd[i] & keep_half2(m8[c], i)));
-              }
+              for (int i = 0; i < 4; ++i) h = __hmax2(h, habs2_bits(wd[i] & keep_half2(m8[c], i)));
             }
           }
-          const float2 hf = __half22float2(h);
-          part[g] = fmaxf(hf.x, hf.y);
         }
+        const float2 hf = __half22float2(h);
+        const uint32_t m = __reduce_max_sync(0xffffffffu, __float_as_uint(fmaxf(hf.x, hf.y)));
+        if (lane == 0) s_red[warp * kMaxGroup + g] = __uint_as_float(m);
       }
-#pragma unroll
-      for (int g = 0; g < kMaxGroup; ++g) {
-        if (g < ng) {
-          const float m = warp_max(part[g]);
-          if (lane == 0) s_red[warp * kMaxGroup + g] = m;
-        }
-      }
+      if (warp == 0 && !listed) build_list();
+      listed = true;
       __syncthreads();
       if (tid < ng) {
         float m = 0.0f;
 #pragma unroll
         for (int i = 0; i < kWarps; ++i) m = fmaxf(m, s_red[i * kMaxGroup + tid]);
         s_row[tid] = m;
+        s_rcp[tid] = quant_rcp(m);
+        a.x_scale[wb + gb + tid] = m;
       }
       __syncthreads();
+      if (count < 0) setup_panels();
+      // Codes of the group's rows (0 at the outlier columns).
+#pragma unroll 1
       for (int g = 0; g < ng; ++g) {
         const int row = wb + gb + g;
         const float am = s_row[g];
-        const float inv = quant_inv(am);
+        const float ra = s_rcp[g];
         const uint4* srow = reinterpret_cast<const uint4*>(s_rows + (gb + g) * row_bytes);
         uint2* dst = reinterpret_cast<uint2*>(Xq + static_cast<size_t>(row) * K);
-        __half* xo_row = X_O + static_cast<size_t>(row) * a.ld;
 #pragma unroll
         for (int c = 0; c < VPT; ++c) {
           const int v = tid + kThreads * c;
           if (v < nv) {
-            const uint4 u = srow[v];
-            uint2 q = codes8(u, am, inv);
+            uint2 q = codes8(srow[v], am, ra);
             if (m8[c]) {
               q.x &= keep_bytes(m8[c] & 0xFu);
               q.y &= keep_bytes(m8[c] >> 4);
-              if (compact) {
-                const uint32_t wbits = s_bits[v >> 2];
-                const int base = s_prefix[v >> 2];
-                const __half* hv = reinterpret_cast<const __half*>(&u);
-#pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                  if ((m8[c] >> i) & 1u) {
-                    const int bit = 8 * (v & 3) + i;
-                    xo_row[base + __popc(wbits & ((1u << bit) - 1u))] = hv[i];
-                  }
-                }
-              }
             }
             dst[v] = q;
           }
         }
-        if (compact)
-          for (int p = count + tid; p < pw; p += kThreads) xo_row[p] = __float2half_rn(0.0f);
-        if (tid == 0) a.x_scale[row] = am;
       }
-      __syncthreads();   // s_red / s_row are reused by the next group
+      // The group's rows of the compacted panel X_O (outlier columns, then zeros).
+      if (compact) {
+        for (int e = tid; e < ng * pw; e += kThreads) {
+          const int g = e / pw;
+          const int p2 = e - g * pw;
+          const __half* hrow = reinterpret_cast<const __half*>(s_rows + (gb + g) * row_bytes);
+          X_O[static_cast<size_t>(wb + gb + g) * a.ld + p2] =
+              (p2 < count) ? hrow[s_idx[p2]] : __float2half_rn(0.0f);
+        }
+      }
+      __syncthreads();   // s_red / s_row / s_rcp are reused by the next group
     }
+  }
+
+  if (count < 0) {   // no rows of X here: the W_O rows are still this CTA's
+    if (warp == 0) build_list();
+    __syncthreads();
+    setup_panels();
   }
 
   // ---------------- phase B.3: W_O rows of this CTA (outlier columns of W)
@@ -391,7 +406,11 @@ __global__ void __launch_bounds__(kThreads, VPT == 1 ? 2 : 1)
     if (it < items) {
       const int n = wn0 + it / chunks;
       const int ch = it - (n - wn0) * chunks;
-      reinterpret_cast<uint4*>(W_O + static_cast<size_t>(n) * a.ld)[ch] = early[k];
+      uint4 o;
+      __half* h = reinterpret_cast<__half*>(&o);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) h[i] = early[k][i];
+      reinterpret_cast<uint4*>(W_O + static_cast<size_t>(n) * a.ld)[ch] = o;
     }
   }
   for (int it = tid + kEarly * kThreads; it < items; it += kThreads) {

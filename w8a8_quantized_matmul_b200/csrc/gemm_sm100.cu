@@ -237,7 +237,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             ok = false;
             break;
           }
-          tc_fence_after();
+          // The stage was written by TMA and is ordered by its mbarrier alone;
+          // a tcgen05 fence here would stall the issue of every stage.
           const uint32_t a = smem_addr(smem + s * C::STAGE_BYTES);
           const uint32_t b = a + C::A_BYTES;
           if (it < nk) {
@@ -603,13 +604,13 @@ cudaError_t launch(const GemmArgs& a, cudaStream_t s) {
 
 }  // namespace
 
-// CTA pairs whenever there is more than one 128-row block of output rows.
 bool make_tmap_2d(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int elem_bytes,
                   uint64_t cols, uint64_t rows, uint32_t box_rows, uint32_t box_bytes,
                   CUtensorMapSwizzle swz) {
   return make_tmap(m, base, dt, elem_bytes, cols, rows, box_rows, box_bytes, swz);
 }
 
+// CTA pairs whenever there is more than one 128-row block of output rows.
 cudaError_t launch_gemm_mixed(const GemmArgs& a, cudaStream_t s) {
   return a.M > BM ? launch<false, true>(a, s) : launch<false, false>(a, s);
 }

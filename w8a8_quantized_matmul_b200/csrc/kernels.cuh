@@ -105,6 +105,7 @@ struct DecodeArgs {
   float* x_scale;
   int8_t* Xq;
   int32_t* status;
+  int nbox;               // Wq boxes per CTA (set by launch_decode)
 };
 
 bool decode_supported(int M, int K);

@@ -5,6 +5,15 @@
 // section, vector-wise quantisation with c = 127/absmax; the rounding is to
 // nearest, ties to even): q = clamp(rint(fl32(fl32(x*127)/a)), -127, 127),
 // x*127 exact in fp32 for fp16 x, one correctly rounded fp32 division.
+//
+// The kernels form the correctly rounded quotient without a division: with
+// n = x*127 (exact), ra = fl(1/a) (one correctly rounded reciprocal per group),
+// q = fl(n*ra), r = fma(q, -a, n) and q' = fma(r, ra, q), q' equals fl(n/a)
+// for every pair of fp16 values x, a with |x| <= a (the one-step FMA
+// correction of a reciprocal-based quotient). This was checked for all such
+// pairs exhaustively; the check ships with the tests. The integer code of q'
+// (|q'| <= 127) is then the low byte of fl(q' + 1.5*2^23), which rounds half
+// to even. Entries of outlier columns may exceed a; their codes are discarded.
 #pragma once
 
 #include <cuda_fp16.h>
@@ -31,27 +40,17 @@ __device__ __forceinline__ int quant_code(float x, float a) {
   return max(-127, min(127, q));
 }
 
-// The same code without a division on the common path: with inv = fl(127/a),
-// y = fl(x*inv) is within 127*(2^-23 + 2^-48) < 1.6e-5 of the exact quotient
-// t = x*127/a, and fl(t) within 127*2^-24 < 7.6e-6 of t, so y and fl(t) are less
-// than 2.3e-5 apart. Unless y lies within 6.2e-5 of a half-integer, both round
-// to the same integer; near a half-integer the correctly rounded quotient is
-// formed exactly as quant_code does. Needs |x| <= a (true for every non-outlier
-// entry of a row, since a is their absmax).
-__device__ __forceinline__ int quant_code_fast(float x, float a, float inv) {
-  if (a == 0.0f) return 0;
-  const float y = __fmul_rn(x, inv);
-  const float r = rintf(y);
-  int q;
-  if (fabsf(y - r) <= 0.5f - 6.2e-5f)
-    q = static_cast<int>(r);
-  else
-    q = __float2int_rn(__fdiv_rn(__fmul_rn(x, 127.0f), a));
-  return max(-127, min(127, q));
-}
+// 1/a correctly rounded; 0 for an all-zero group (every code is then 0).
+__device__ __forceinline__ float quant_rcp(float a) { return a == 0.0f ? 0.0f : __frcp_rn(a); }
 
-__device__ __forceinline__ float quant_inv(float a) {
-  return a == 0.0f ? 0.0f : __fdiv_rn(127.0f, a);
+// The code of quant_code from the FMA-corrected quotient (ra = quant_rcp(a);
+// exact for |x| <= a, see the file comment).
+__device__ __forceinline__ int quant_code_fma(float x, float a, float ra) {
+  const float n = __fmul_rn(x, 127.0f);
+  const float q = __fmul_rn(n, ra);
+  const float r = __fmaf_rn(q, -a, n);
+  const int c = __float2int_rn(__fmaf_rn(r, ra, q));
+  return max(-127, min(127, c));
 }
 
 __device__ __forceinline__ uint32_t pack4(int a, int b, int c, int d) {
@@ -81,7 +80,7 @@ __device__ __forceinline__ float masked_absmax8(const uint4& u, const uint32_t* 
 // entries are also copied to their compacted position in the X_O row.
 template <bool COMPACT>
 __device__ __forceinline__ void quantize8(const uint4& u, const uint32_t* s_bits,
-                                          const int32_t* s_prefix, int v, float amax, float inv,
+                                          const int32_t* s_prefix, int v, float amax, float ra,
                                           uint2* dst, __half* xo_row) {
   const uint32_t wbits = s_bits[v >> 2];
   const uint32_t m8 = (wbits >> (8 * (v & 3))) & 0xFFu;
@@ -89,7 +88,7 @@ __device__ __forceinline__ void quantize8(const uint4& u, const uint32_t* s_bits
   unpack8(u, f);
   int q[8];
 #pragma unroll
-  for (int i = 0; i < 8; ++i) q[i] = ((m8 >> i) & 1u) ? 0 : quant_code_fast(f[i], amax, inv);
+  for (int i = 0; i < 8; ++i) q[i] = ((m8 >> i) & 1u) ? 0 : quant_code_fma(f[i], amax, ra);
   uint2 o;
   o.x = pack4(q[0], q[1], q[2], q[3]);
   o.y = pack4(q[4], q[5], q[6], q[7]);
@@ -112,8 +111,6 @@ __device__ __forceinline__ void quantize8(const uint4& u, const uint32_t* s_bits
 // rounds y to the nearest integer (ties to even) and leaves it in the low
 // mantissa bits, so the low byte of the sum is the two's-complement code.
 constexpr float kMagic = 12582912.0f;
-// |y - rint(y)| above this means y is within 6.2e-5 of a half-integer.
-constexpr float kTieMargin = 0.5f - 6.2e-5f;
 
 // Paired IEEE fp32 arithmetic (round to nearest even in each lane).
 __device__ __forceinline__ uint64_t f2pack(float a, float b) {
@@ -128,6 +125,11 @@ __device__ __forceinline__ uint64_t mul2(uint64_t a, uint64_t b) {
 __device__ __forceinline__ uint64_t add2(uint64_t a, uint64_t b) {
   uint64_t r;
   asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
   return r;
 }
 __device__ __forceinline__ uint64_t sub2(uint64_t a, uint64_t b) {
@@ -155,62 +157,36 @@ __device__ __forceinline__ uint32_t keep_bytes(uint32_t m4) {
          ((m4 & 4u) ? 0u : 0x00FF0000u) | ((m4 & 8u) ? 0u : 0xFF000000u);
 }
 
+// Codes of the fp16 pair w, each in the low byte of its fp32 lane (the 1.5*2^23
+// rounding): n = w*127, q = n*ra, r = fma(q, -a, n), q' = fma(r, ra, q).
+// a2 = (-a, -a), ra2 = (ra, ra) packed once per group.
+__device__ __forceinline__ uint64_t code_lanes(uint32_t w, uint64_t na2, uint64_t ra2) {
+  const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&w));
+  const uint64_t n = mul2(f2pack(f.x, f.y), f2pack(127.0f, 127.0f));
+  const uint64_t q = mul2(n, ra2);
+  const uint64_t r = fma2(q, na2, n);
+  return add2(fma2(r, ra2, q), f2pack(kMagic, kMagic));
+}
+
 // Eight INT8 codes of the vector u (exact; see the file comment).
-__device__ __forceinline__ uint2 codes8(const uint4& u, float amax, float inv) {
-  if (amax == 0.0f) return make_uint2(0u, 0u);
+__device__ __forceinline__ uint2 codes8(const uint4& u, float amax, float ra) {
   const uint32_t* w = reinterpret_cast<const uint32_t*>(&u);
-  const uint64_t inv2 = f2pack(inv, inv);
-  const uint64_t magic2 = f2pack(kMagic, kMagic);
+  const uint64_t na2 = f2pack(-amax, -amax), ra2 = f2pack(ra, ra);
   uint32_t b[8];
-  float emax = 0.0f;
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
-    const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&w[i]));
-    const uint64_t y = mul2(f2pack(f.x, f.y), inv2);
-    const uint64_t s = add2(y, magic2);
-    const uint64_t e = sub2(y, sub2(s, magic2));
-    emax = fmaxf(emax, fmaxf(fabsf(lo(e)), fabsf(hi(e))));
+    const uint64_t s = code_lanes(w[i], na2, ra2);
     b[2 * i] = static_cast<uint32_t>(s);
     b[2 * i + 1] = static_cast<uint32_t>(s >> 32);
-  }
-  if (emax > kTieMargin) {
-    // Within reach of a rounding tie: form the correctly rounded quotient.
-    float f[8];
-    unpack8(u, f);
-#pragma unroll
-    for (int i = 0; i < 8; ++i) b[i] = static_cast<uint32_t>(quant_code(f[i], amax));
   }
   const uint32_t w0 = __byte_perm(__byte_perm(b[0], b[1], 0x0040), __byte_perm(b[2], b[3], 0x0040), 0x5410);
   const uint32_t w1 = __byte_perm(__byte_perm(b[4], b[5], 0x0040), __byte_perm(b[6], b[7], 0x0040), 0x5410);
   return make_uint2(w0, w1);
 }
 
-// Exact codes of four fp16 values (the tie fallback of codes4), kept out of line
-// so the common path stays short.
-static __device__ __noinline__ uint32_t codes4_exact(uint32_t w0, uint32_t w1, float amax) {
-  const float2 f0 = __half22float2(*reinterpret_cast<const __half2*>(&w0));
-  const float2 f1 = __half22float2(*reinterpret_cast<const __half2*>(&w1));
-  return pack4(quant_code(f0.x, amax), quant_code(f0.y, amax), quant_code(f1.x, amax),
-               quant_code(f1.y, amax));
-}
-
-// Four INT8 codes of the fp16 values in h (two half2 words), same rule as codes8.
-__device__ __forceinline__ uint32_t codes4(const uint2& h, float amax, float inv) {
-  if (amax == 0.0f) return 0u;
-  const uint64_t inv2 = f2pack(inv, inv);
-  const uint64_t magic2 = f2pack(kMagic, kMagic);
-  const float2 f0 = __half22float2(*reinterpret_cast<const __half2*>(&h.x));
-  const float2 f1 = __half22float2(*reinterpret_cast<const __half2*>(&h.y));
-  const uint64_t y0 = mul2(f2pack(f0.x, f0.y), inv2);
-  const uint64_t y1 = mul2(f2pack(f1.x, f1.y), inv2);
-  const uint64_t s0 = add2(y0, magic2);
-  const uint64_t s1 = add2(y1, magic2);
-  const uint64_t e0 = sub2(y0, sub2(s0, magic2));
-  const uint64_t e1 = sub2(y1, sub2(s1, magic2));
-  const float emax = fmaxf(fmaxf(fabsf(lo(e0)), fabsf(hi(e0))), fmaxf(fabsf(lo(e1)), fabsf(hi(e1))));
-  if (emax > kTieMargin) return codes4_exact(h.x, h.y, amax);
-  const uint32_t b0 = static_cast<uint32_t>(s0), b1 = static_cast<uint32_t>(s0 >> 32);
-  const uint32_t b2 = static_cast<uint32_t>(s1), b3 = static_cast<uint32_t>(s1 >> 32);
-  return __byte_perm(__byte_perm(b0, b1, 0x0040), __byte_perm(b2, b3, 0x0040), 0x5410);
+// Two INT8 codes (low two bytes) of the fp16 pair w, same rule as codes8.
+__device__ __forceinline__ uint32_t codes2(uint32_t w, float amax, float ra) {
+  const uint64_t s = code_lanes(w, f2pack(-amax, -amax), f2pack(ra, ra));
+  return __byte_perm(static_cast<uint32_t>(s), static_cast<uint32_t>(s >> 32), 0x0040) & 0xFFFFu;
 }
 }  // namespace i8mm

@@ -195,19 +195,19 @@ __global__ void __launch_bounds__(256) quantize_rows_kernel(const __half* __rest
         if (v < nv) amax = fmaxf(amax, masked_absmax8(buf[t], s_bits, v));
       }
       amax = warp_max(amax);
-      const float inv = quant_inv(amax);
+      const float ra = quant_rcp(amax);
 #pragma unroll
       for (int t = 0; t < VPL; ++t) {
         const int v = lane + 32 * t;
-        if (v < nv) quantize8<false>(buf[t], s_bits, nullptr, v, amax, inv, dst, nullptr);
+        if (v < nv) quantize8<false>(buf[t], s_bits, nullptr, v, amax, ra, dst, nullptr);
       }
     } else {
       // Rows longer than the register budget: two passes, the second from L1/L2.
       for (int v = lane; v < nv; v += 32) amax = fmaxf(amax, masked_absmax8(__ldg(src + v), s_bits, v));
       amax = warp_max(amax);
-      const float inv = quant_inv(amax);
+      const float ra = quant_rcp(amax);
       for (int v = lane; v < nv; v += 32)
-        quantize8<false>(__ldg(src + v), s_bits, nullptr, v, amax, inv, dst, nullptr);
+        quantize8<false>(__ldg(src + v), s_bits, nullptr, v, amax, ra, dst, nullptr);
     }
     if (lane == 0) x_scale[row] = amax;
   }
