@@ -161,6 +161,25 @@ int int8_mixed_matmul_profiled(const void* X, const int8_t* Wq, const float* w_s
                                void* Y, void* workspace, size_t workspace_bytes,
                                i8mm_stream_t stream, void* const* events);
 
+// Token-sharded (data-parallel over tokens) form of int8_mixed_matmul, one call
+// per rank on that rank's rows of X. AIInfra "05Quantization01", LLM.int8()
+// section: the outlier feature dimensions are those where any token of the
+// batch exceeds the threshold, so ranks holding parts of one batch must agree
+// on one set. Each rank runs int8_find_outlier_cols on its own rows, the ranks
+// gather their bitmaps (one collective, ceil(K/32) words per rank), and each
+// calls this with all of them: the outlier set is their bitwise OR, and the
+// rest (per-token quantisation, INT8 product, outlier product, sum) is exactly
+// int8_mixed_matmul restricted to the rank's rows. Concatenating the ranks' Y
+// gives, element for element, the Y of one int8_mixed_matmul over the whole batch.
+//   X        device fp16 [M][K], this rank's tokens (M may be 0)
+//   bitmaps  device u32 [n_bitmaps][ceil(K/32)], read only; 4-byte aligned
+//   other arguments, layout, workspace and errors as int8_mixed_matmul; the
+//   workspace's bitmap holds the OR afterwards. Always runs the prefill kernels.
+int int8_mixed_matmul_sharded(const void* X, const int8_t* Wq, const float* w_scale,
+                              const void* W_fp16, int M, int N, int K, const uint32_t* bitmaps,
+                              int n_bitmaps, void* Y, void* workspace, size_t workspace_bytes,
+                              i8mm_stream_t stream);
+
 /*
  * Measurement hook: one stage of int8_mixed_matmul on its own, so that each
  * kernel can be timed back to back.

@@ -192,18 +192,38 @@ def outlier_gemm(X: np.ndarray, W: np.ndarray, idx: np.ndarray) -> np.ndarray:
 # ---------------------------------------------------------------------------
 # Full decomposition ([AIInfra]: C_f16 = C_outlier + C_normal).
 # ---------------------------------------------------------------------------
+def mask_to_bitmap(mask: np.ndarray):
+    """(bitmap uint32[ceil(K/32)], count, idx) of a boolean column mask."""
+    mask = np.asarray(mask, dtype=bool)
+    K = mask.size
+    bitmap = np.zeros((K + 31) // 32, dtype=np.uint32)
+    idx = np.nonzero(mask)[0].astype(np.int32)
+    for j in idx:
+        bitmap[j // 32] |= np.uint32(1) << np.uint32(j % 32)
+    return bitmap, int(idx.size), idx
+
+
 def llm_int8_matmul(X: np.ndarray, W: np.ndarray, threshold: float = 6.0,
-                    Wq: np.ndarray | None = None, w_scale: np.ndarray | None = None):
+                    Wq: np.ndarray | None = None, w_scale: np.ndarray | None = None,
+                    outlier_mask: np.ndarray | None = None):
     """All steps of the path; returns a dict with Y (fp16 [M, N]) and every intermediate.
 
     `W` is the fp16 weight [N, K]; it supplies the outlier columns of the
     FP16 product. `Wq`/`w_scale` default to quantize_weight_rows(W).
+    `outlier_mask` (bool [K]) replaces the detection step with a given outlier
+    set: the set of a batch whose tokens are split over several processes
+    ([AIInfra]: O is a property of the batch's activations, so every part of
+    the batch uses the same O); the threshold is then unused.
     """
     X = np.asarray(X)
     W = np.asarray(W)
     if Wq is None or w_scale is None:
         Wq, w_scale = quantize_weight_rows(W)
-    mask, bitmap, count, idx = find_outlier_cols(X, threshold)
+    if outlier_mask is None:
+        mask, bitmap, count, idx = find_outlier_cols(X, threshold)
+    else:
+        mask = np.asarray(outlier_mask, dtype=bool)
+        bitmap, count, idx = mask_to_bitmap(mask)
     Xq, x_scale = quantize_act_rows(X, mask)
     C = int32_gemm(Xq, Wq)
     Cn = dequantize(C, x_scale, w_scale)

@@ -1,0 +1,86 @@
+"""Token-sharded path across processes, on the CPU with the gloo backend.
+
+The exchange logic of w8a8_quantized_matmul_b200.sharded (local detection, one
+all-gather of the bitmaps, quantisation and product with their OR) runs with
+the CPU oracle standing in for the two kernels. The concatenated rows of Y must
+equal the oracle's Y over the whole batch exactly, and the OR of the gathered
+bitmaps must equal the whole batch's bitmap ([AIInfra] "05Quantization01",
+LLM.int8() section: the outlier set belongs to the batch).
+"""
+import os
+import socket
+
+import numpy as np
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+import oracle
+import synth
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _find(X_local, threshold):
+    _, bitmap, _, _ = oracle.find_outlier_cols(X_local.numpy(), threshold)
+    return torch.from_numpy(bitmap.view(np.int32).copy())
+
+
+def _apply(X_local, Wq, w_scale, W, bitmaps, Y=None, workspace=None):
+    words = bitmaps.numpy().view(np.uint32)
+    orw = np.bitwise_or.reduce(words, axis=0)
+    K = X_local.shape[1]
+    mask = ((orw[np.arange(K) // 32] >> (np.arange(K) % 32).astype(np.uint32)) & 1).astype(bool)
+    out = oracle.llm_int8_matmul(X_local.numpy(), W.numpy(), Wq=Wq.numpy(), w_scale=w_scale.numpy(),
+                                 outlier_mask=mask)
+    return torch.from_numpy(out["Y"]), torch.from_numpy(orw.view(np.int32).copy())
+
+
+def _worker(rank, world, port, bounds, case, q):
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    import datetime
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=60))
+    try:
+        from w8a8_quantized_matmul_b200.sharded import token_sharded_mixed_matmul
+        M, K, N, n_out, seed = case
+        X, W, _ = synth.random_case(M, K, N, n_out, seed=seed)
+        Wq, w_scale = oracle.quantize_weight_rows(W)
+        r0, r1 = bounds[rank], bounds[rank + 1]
+        Xl = torch.from_numpy(np.ascontiguousarray(X[r0:r1]))
+        Y, orw = token_sharded_mixed_matmul(Xl, torch.from_numpy(Wq), torch.from_numpy(w_scale),
+                                           torch.from_numpy(W), 6.0, find=_find, apply=_apply)
+        q.put((rank, Y.numpy(), orw.numpy()))
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world,split", [(2, [0, 37, 96]), (3, [0, 0, 50, 96]), (2, [0, 96, 96])])
+def test_token_sharded_matches_whole_batch(world, split):
+    case = (96, 320, 72, 4, 11)
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_worker, args=(r, world, port, split, case, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    results = {}
+    for _ in range(world):
+        rank, Y, orw = q.get(timeout=120)
+        results[rank] = (Y, orw)
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    M, K, N, n_out, seed = case
+    X, W, _ = synth.random_case(M, K, N, n_out, seed=seed)
+    ref = oracle.llm_int8_matmul(X, W)
+    Y = np.concatenate([results[r][0] for r in range(world)], axis=0)
+    np.testing.assert_array_equal(Y, ref["Y"])
+    for r in range(world):
+        np.testing.assert_array_equal(results[r][1].view(np.uint32), ref["bitmap"])

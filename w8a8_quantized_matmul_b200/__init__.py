@@ -36,6 +36,7 @@ __all__ = [
     "int8_mixed_matmul",
     "int8_mixed_matmul_profiled",
     "int8_mixed_matmul_stage",
+    "int8_mixed_matmul_sharded",
     "int8_debug_gemm_i32",
     "int8_device_status",
     "Int8mmError",
@@ -172,6 +173,37 @@ def int8_mixed_matmul_stage(stage, X, Wq, w_scale, W_fp16, threshold, Y, workspa
                                          workspace.numel() * workspace.element_size(),
                                          _stream(stream)))
     return Y
+
+
+def int8_mixed_matmul_sharded(X, Wq, w_scale, W_fp16, bitmaps, Y=None, workspace=None,
+                              stream=None):
+    """One rank's part of a token-sharded int8_mixed_matmul.
+
+    X fp16 [M, K] are this rank's tokens; bitmaps int32 [n, ceil(K/32)] are the
+    outlier bitmaps of all ranks' int8_find_outlier_cols (the outlier set is their
+    OR). Returns (Y fp16 [M, N], workspace)."""
+    M, K = X.shape
+    N = Wq.shape[0]
+    _need(X, "X", torch.float16, (M, K))
+    _need(Wq, "Wq", torch.int8, (N, K))
+    _need(w_scale, "w_scale", torch.float32, (N,))
+    _need(W_fp16, "W_fp16", torch.float16, (N, K))
+    words = (K + 31) // 32
+    if bitmaps.dim() != 2:
+        raise ValueError("bitmaps must be [n_ranks, ceil(K/32)]")
+    _need(bitmaps, "bitmaps", torch.int32, (bitmaps.shape[0], words))
+    Y = torch.empty((M, N), dtype=torch.float16, device=X.device) if Y is None else Y
+    _need(Y, "Y", torch.float16, (M, N))
+    need = int8_mixed_matmul_workspace_size(M, N, K)
+    if workspace is None:
+        workspace = torch.empty((max(need, 1),), dtype=torch.uint8, device=X.device)
+    check("int8_mixed_matmul_sharded",
+          load().int8_mixed_matmul_sharded(_ptr(X), _ptr(Wq), _ptr(w_scale), _ptr(W_fp16), M, N,
+                                           K, _ptr(bitmaps), int(bitmaps.shape[0]), _ptr(Y),
+                                           _ptr(workspace),
+                                           workspace.numel() * workspace.element_size(),
+                                           _stream(stream)))
+    return Y, workspace
 
 
 def int8_debug_gemm_i32(Xq, Wq, C=None, stream=None):

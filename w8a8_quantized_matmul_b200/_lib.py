@@ -36,6 +36,8 @@ PROTOTYPES = {
                                         ctypes.POINTER(_vp)]),
     "int8_mixed_matmul_stage": (_i, [_i, _vp, _vp, _vp, _vp, _i, _i, _i, _f, _vp, _vp, _sz, _vp]),
     "int8_mixed_matmul_noalloc": (_i, [_vp, _vp, _vp, _vp, _i, _i, _i, _f, _vp, _vp]),
+    "int8_mixed_matmul_sharded": (_i, [_vp, _vp, _vp, _vp, _i, _i, _i, _vp, _i, _vp, _vp, _sz,
+                                       _vp]),
     "int8_debug_gemm_i32": (_i, [_vp, _vp, _i, _i, _i, _vp, _vp]),
     "int8_device_status": (_i, [_vp, _vp]),
     "int8_status_string": (ctypes.c_char_p, [_i]),

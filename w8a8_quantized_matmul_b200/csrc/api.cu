@@ -213,10 +213,11 @@ int int8_quantize_act_rows(const void* X, int M, int K, const uint32_t* col_bitm
 namespace {
 
 // stages: bit 0 = control-word clear + fused quantisation kernel, bit 1 = GEMM.
+// given / given_n: token-sharded mode (outlier set = OR of the given bitmaps).
 int mixed_matmul_impl(const void* X, const int8_t* Wq, const float* w_scale, const void* W_fp16,
                       int M, int N, int K, float threshold, void* Y, void* workspace,
                       size_t workspace_bytes, cudaStream_t stream, cudaEvent_t const* ev,
-                      int stages = 3) {
+                      int stages = 3, const uint32_t* given = nullptr, int given_n = 0) {
   int st = check_sizes(M, N, K);
   if (st != I8MM_OK) return st;
   if ((st = check_threshold(threshold)) != I8MM_OK) return st;
@@ -246,7 +247,7 @@ int mixed_matmul_impl(const void* X, const int8_t* Wq, const float* w_scale, con
   const __half* Wh = static_cast<const __half*>(W_fp16);
 
   // Decode shapes: one clustered kernel for the whole call.
-  if (stages == 3 && !ev && decode_supported(M, K)) {
+  if (stages == 3 && !ev && !given && decode_supported(M, K)) {
     DecodeArgs da{};
     da.X = Xh;
     da.W = Wh;
@@ -289,6 +290,8 @@ int mixed_matmul_impl(const void* X, const int8_t* Wq, const float* w_scale, con
     fa.W_O = WO;
     fa.ld = L.l.panel_ld;
     fa.status = status;
+    fa.given = given;
+    fa.given_n = given_n;
     e = launch_detect_quantize_compact(fa, stream);
     if (e != cudaSuccess) return cuda_fail("detect_quantize_compact_kernel launch", e);
   }
@@ -335,6 +338,17 @@ int int8_mixed_matmul_stage(int stage, const void* X, const int8_t* Wq, const fl
   if (stage != 1 && stage != 2) return I8MM_ERR_INVALID_ARG;
   return mixed_matmul_impl(X, Wq, w_scale, W_fp16, M, N, K, threshold, Y, workspace,
                            workspace_bytes, stream, nullptr, stage);
+}
+
+int int8_mixed_matmul_sharded(const void* X, const int8_t* Wq, const float* w_scale,
+                              const void* W_fp16, int M, int N, int K, const uint32_t* bitmaps,
+                              int n_bitmaps, void* Y, void* workspace, size_t workspace_bytes,
+                              i8mm_stream_t stream) {
+  if (!bitmaps || n_bitmaps < 1 || n_bitmaps > 65536) return I8MM_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(bitmaps) & 3u) != 0) return I8MM_ERR_ALIGNMENT;
+  // The threshold only enters detection, which the caller has done per rank.
+  return mixed_matmul_impl(X, Wq, w_scale, W_fp16, M, N, K, 0.0f, Y, workspace, workspace_bytes,
+                           stream, nullptr, 3, bitmaps, n_bitmaps);
 }
 
 int int8_mixed_matmul_profiled(const void* X, const int8_t* Wq, const float* w_scale,

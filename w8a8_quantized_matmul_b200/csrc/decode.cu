@@ -141,6 +141,7 @@ __global__ void __launch_bounds__(64 + 32 * kMaxXWarps, 1)
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
   const int lane = tid & 31;
+  griddep_launch_dependents();
   const int S = static_cast<int>(cluster_nctarank());
   const int rank = static_cast<int>(cluster_ctarank());
   const int nxw = 2 * nbox;                             // X worker warps
@@ -169,6 +170,9 @@ __global__ void __launch_bounds__(64 + 32 * kMaxXWarps, 1)
     mbar_arrive_expect_tx(xchg, static_cast<uint32_t>(S * kMsgWords * 4));
     mbar_arrive_expect_tx(redbar, static_cast<uint32_t>(S * owned_rows(rank, rpr) * 64));
     fence_mbarrier_init();
+    // Launched with programmatic stream serialization: the set-up above overlaps
+    // the previous kernel; every global access comes after this wait.
+    griddep_wait();
     if (blockIdx.x == 0 && a.status) *a.status = 0;
     // X first (small, L2-resident after the first cluster), then the Wq slice.
     // Issued before the CTA barrier: only this thread has used the barriers.
@@ -188,6 +192,7 @@ __global__ void __launch_bounds__(64 + 32 * kMaxXWarps, 1)
   __syncthreads();
   tc_fence_after();
   cluster_arrive_relaxed();   // phase 1: this CTA's barriers are initialised
+  if (tid != 0) griddep_wait();
   const uint32_t tmem = *tslot;
   bool ok = true;
 
@@ -512,13 +517,15 @@ cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t s) {
   cfg.blockDim = dim3(64 + 32 * 2 * nbox);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = s;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = S;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   DecodeArgs args = a;
   args.nbox = nbox;
   e = cudaLaunchKernelEx(&cfg, decode_kernel, tmw, tmx, args);

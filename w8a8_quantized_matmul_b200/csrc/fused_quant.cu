@@ -127,6 +127,9 @@ __global__ void __launch_bounds__(kThreads, VPT == 1 ? 2 : 1)
   const int nwaves = (R + nb - 1) / nb;
   const int wave_rows = nwaves ? (R + nwaves - 1) / nwaves : 0;
 
+  // The GEMM that follows may launch now; it waits for this grid's completion
+  // before reading anything written here.
+  griddep_launch_dependents();
   if (tid == 0) {
     mbar_init(s_bar, 1);
     fence_mbarrier_init();
@@ -161,9 +164,11 @@ __global__ void __launch_bounds__(kThreads, VPT == 1 ? 2 : 1)
   for (int c = 0; c < VPT; ++c)
 #pragma unroll
     for (int i = 0; i < 4; ++i) cmax[c][i] = __float2half2_rn(0.0f);
+  const bool given = a.given != nullptr;   // outlier set supplied (token-sharded mode)
   for (int w = 0; w < nwaves; ++w) {
     if (w > 0) __syncthreads();   // everyone is done with the previous wave
     const int n = fetch(w);
+    if (given) continue;
     for (int g = 0; g < n; ++g) {
       const uint4* srow = reinterpret_cast<const uint4*>(s_rows + g * row_bytes);
 #pragma unroll
@@ -191,12 +196,12 @@ __global__ void __launch_bounds__(kThreads, VPT == 1 ? 2 : 1)
     uint32_t word = flags << (8 * (lane & 3));
     word |= __shfl_xor_sync(0xffffffffu, word, 1);
     word |= __shfl_xor_sync(0xffffffffu, word, 2);
-    if ((lane & 3) == 0 && v < nv && word != 0) atomicOr(a.bitmap + (v >> 2), word);
+    if (!given && (lane & 3) == 0 && v < nv && word != 0) atomicOr(a.bitmap + (v >> 2), word);
   }
 
-  // ---------------- grid barrier (bounded)
+  // ---------------- grid barrier (bounded); not needed when the set is given
   __syncthreads();
-  if (tid == 0) {
+  if (tid == 0 && !given) {
     __threadfence();
     atomicAdd(a.sync_ctr, 1);
     const uint64_t t0 = gtimer();
@@ -215,11 +220,18 @@ __global__ void __launch_bounds__(kThreads, VPT == 1 ? 2 : 1)
   // for every row), straight from the global bitmap. Warp 0 also builds the
   // per-word prefix counts and the ascending outlier list in shared memory; the
   // other warps start on the row maxima meanwhile.
+  // Word w of the outlier bitmap: the global bitmap, or the OR of the given ones.
+  auto bitmap_word = [&](int w) -> uint32_t {
+    if (!given) return __ldcg(a.bitmap + w);
+    uint32_t b = 0;
+    for (int r = 0; r < a.given_n; ++r) b |= __ldg(a.given + static_cast<size_t>(r) * words + w);
+    return b;
+  };
   uint32_t m8[VPT];
 #pragma unroll
   for (int c = 0; c < VPT; ++c) {
     const int v = tid + kThreads * c;
-    m8[c] = (v < nv) ? (__ldcg(a.bitmap + (v >> 2)) >> (8 * (v & 3))) & 0xFFu : 0u;
+    m8[c] = (v < nv) ? (bitmap_word(v >> 2) >> (8 * (v & 3))) & 0xFFu : 0u;
   }
   // Warp 0 also builds the per-word prefix counts and the ascending outlier
   // list in shared memory (build_list); its first bitmap words are loaded now so
@@ -229,7 +241,7 @@ __global__ void __launch_bounds__(kThreads, VPT == 1 ? 2 : 1)
   uint32_t bw8[8];
 #pragma unroll
   for (int i = 0; i < 8; ++i)
-    bw8[i] = (warp == 0 && lw0 + i < lw1) ? __ldcg(a.bitmap + lw0 + i) : 0u;
+    bw8[i] = (warp == 0 && lw0 + i < lw1) ? bitmap_word(lw0 + i) : 0u;
   bool listed = false;
   auto build_list = [&]() {
     // Lane l scans the words [lw0, lw1): the first 8 are in bw8.
@@ -242,7 +254,7 @@ __global__ void __launch_bounds__(kThreads, VPT == 1 ? 2 : 1)
     for (int wb = lw0 + 8; wb < lw1; wb += 8) {
       uint32_t b[8];
 #pragma unroll
-      for (int i = 0; i < 8; ++i) b[i] = (wb + i < lw1) ? __ldcg(a.bitmap + wb + i) : 0u;
+      for (int i = 0; i < 8; ++i) b[i] = (wb + i < lw1) ? bitmap_word(wb + i) : 0u;
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
         if (wb + i < lw1) s_bits[wb + i] = b[i];
@@ -266,6 +278,8 @@ __global__ void __launch_bounds__(kThreads, VPT == 1 ? 2 : 1)
       }
     }
     if (lane == 31) s_misc[0] = incl;
+    if (given && blockIdx.x == 0)
+      for (int w = lw0; w < lw1; ++w) a.bitmap[w] = s_bits[w];
   };
 
   // ---------------- phase B.2: quantise, the resident wave first, then re-fetch the rest

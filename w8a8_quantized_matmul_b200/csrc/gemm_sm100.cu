@@ -166,6 +166,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   if constexpr (PAIR) cluster_sync();   // barriers and TMEM of both CTAs are ready
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  // Set-up above overlaps the tail of the previous kernel (the quantisation
+  // kernel); nothing it writes is read before this point.
+  griddep_launch_dependents();
+  griddep_wait();
 
   const int count = (!OUT_I32 && n_outliers) ? *n_outliers : 0;
   const bool tc_out = count > kCcMax;          // outlier product on the tensor cores
@@ -585,15 +589,20 @@ cudaError_t launch(const GemmArgs& a, cudaStream_t s) {
   cfg.blockDim = dim3(kThreads);
   cfg.dynamicSmemBytes = C::SMEM_BYTES;
   cfg.stream = s;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
+  int na = 0;
+  attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[na].val.programmaticStreamSerializationAllowed = 1;
+  ++na;
   if (PAIR) {
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = 2;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    attr[na].id = cudaLaunchAttributeClusterDimension;
+    attr[na].val.clusterDim.x = 2;
+    attr[na].val.clusterDim.y = 1;
+    attr[na].val.clusterDim.z = 1;
+    ++na;
   }
+  cfg.attrs = attr;
+  cfg.numAttrs = na;
   e = cudaLaunchKernelEx(&cfg, kern, maps[0], maps[1], maps[2], maps[3], maps[4], y_tma,
                          a.x_scale, a.w_scale,
                          OUT_I32 ? nullptr : a.n_outliers, a.X_O, a.W_O, a.ld, a.out, a.M, a.N,

@@ -53,6 +53,11 @@ struct FusedArgs {
   __half* W_O;            // out: [N][ld]
   int ld;
   int32_t* status;        // device status word
+  // Token-sharded mode: the outlier set is the OR of given_n bitmaps of
+  // ceil(K/32) words each (one per rank, gathered by the caller); detection and
+  // the grid barrier are skipped and the OR is written to bitmap.
+  const uint32_t* given;
+  int given_n;
 };
 
 cudaError_t launch_detect_quantize_compact(const FusedArgs& a, cudaStream_t s);

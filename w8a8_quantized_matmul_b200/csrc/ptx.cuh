@@ -87,6 +87,19 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
   }
 }
 
+// ---------------------------------------------------------------- dependent launch
+// A kernel launched with programmatic stream serialization may start before the
+// previous kernel in the stream has finished; it must execute griddep_wait()
+// before touching any memory that kernel may write (or read). Every thread that
+// accesses such memory waits itself (or is ordered after one that did).
+__device__ __forceinline__ void griddep_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+// Lets the next kernel of the stream (if launched for it) start its prologue.
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ---------------------------------------------------------------- TMA
 // 2-D tiled bulk copy global -> shared; completion is signalled on `bar`
 // as transaction bytes. (x, y) are element coordinates, x innermost.
