@@ -137,12 +137,12 @@ def time_oracle(w, X, W, Wq, w_scale, budget_s: float, max_rows: int | None = No
 
 
 # --------------------------------------------------------------------------- distributed
-def dist_setup(n_gpus: int):
+def dist_setup(n_gpus: int, want_pg: bool = False):
     import torch
     ws = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
-    if ws > 1:
+    if ws > 1 or (want_pg and "MASTER_ADDR" in os.environ):
         import datetime
         import torch.distributed as dist
         torch.cuda.set_device(local)
@@ -154,8 +154,8 @@ def dist_setup(n_gpus: int):
 
 
 def barrier(ws):
-    if ws > 1:
-        import torch.distributed as dist
+    import torch.distributed as dist
+    if ws > 1 or (dist.is_available() and dist.is_initialized()):
         dist.barrier()
 
 
@@ -193,8 +193,33 @@ class Problem:
     def step(self, i):
         import w8a8_quantized_matmul_b200 as m
         s = self.sets[i % len(self.sets)]
+        if self.sharded:
+            self.sharded_step(s)
+            return
         m.int8_mixed_matmul(s["X"], s["Wq"], s["ws"], s["W"], self.w.threshold, Y=s["Y"],
                             workspace=s["work"])
+
+    sharded = False
+
+    def enable_sharding(self, world):
+        """Token-sharded steps: this rank's tokens, outlier bitmaps all-gathered."""
+        import torch
+        words = (self.w.K + 31) // 32
+        for s in self.sets:
+            s["bm"] = torch.empty((words,), dtype=torch.int32, device="cuda")
+            s["cnt"] = torch.empty((4,), dtype=torch.int32, device="cuda")
+            s["idx"] = torch.empty((self.w.K,), dtype=torch.int32, device="cuda")
+            s["gathered"] = torch.empty((world, words), dtype=torch.int32, device="cuda")
+        self.sharded = True
+
+    def sharded_step(self, s):
+        import torch.distributed as dist
+        import w8a8_quantized_matmul_b200 as m
+        m.int8_find_outlier_cols(s["X"], self.w.threshold, col_bitmap=s["bm"],
+                                 n_outliers=s["cnt"][:1], col_idx=s["idx"])
+        dist.all_gather_into_tensor(s["gathered"], s["bm"])
+        m.int8_mixed_matmul_sharded(s["X"], s["Wq"], s["ws"], s["W"], s["gathered"], Y=s["Y"],
+                                    workspace=s["work"])
 
     def time_stage(self, stage, n, stream):
         """Average device time of one stage launched n times back to back (ms)."""
@@ -250,10 +275,18 @@ def run_ours(args, ws, rank, local):
     props = torch.cuda.get_device_properties(torch.cuda.current_device())
     l2 = getattr(props, "L2_cache_size", 126 * 2 ** 20) or 126 * 2 ** 20
 
+    import torch.distributed as dist
+    sharded = args.dp == "sharded" and dist.is_available() and dist.is_initialized()
     w = synth.WORKLOADS[args.workload]
-    X, W, planted = synth.make_workload(w)
+    if sharded:
+        # this rank's tokens of a batch of ws*M tokens
+        X, W, planted = synth.make_workload_shard(w, rank, ws)
+    else:
+        X, W, planted = synth.make_workload(w)
     n_sets = n_sets_for(w, l2)
     prob = Problem(w, X, W, n_sets)
+    if sharded:
+        prob.enable_sharding(ws)
 
     stream = torch.cuda.current_stream()
     for i in range(args.warmup):
@@ -338,7 +371,9 @@ def run_ours(args, ws, rank, local):
         "data": "synthetic",
         "config": {"workload": w.name, "M": w.M, "K": w.K, "N": w.N, "threshold": w.threshold,
                    "planted_outliers": int(len(planted)), "detected_outliers": count,
-                   "parallelism": f"replicas x{ws}",
+                   "parallelism": (f"token-sharded dp{ws}: {ws}x{w.M} tokens per step, one "
+                                   "all-gather of the ceil(K/32)-word outlier bitmaps" if sharded
+                                   else f"replicas x{ws}"),
                    "l2": f"rotating {n_sets} buffer sets of {prob.bytes_touched() / 1e6:.0f} MB "
                          f"touched per step (> 2x L2 of {l2 / 1e6:.0f} MB)"},
         "roofline": {"kernel": "gemm_i8_persistent_kernel (tcgen05 kind::i8, fp16 outlier epilogue)",
@@ -356,9 +391,12 @@ def run_ours(args, ws, rank, local):
                               "peak_note": f"{peaks_kind} hbm_gbs"},
         "e2e": {"value": round(e2e_value, 3), "unit": "TOPS", "steps": e2e_steps,
                 "h2d_bytes_per_step": 2 * w.M * w.K, "d2h_bytes_per_step": 2 * w.M * w.N},
-        "gpu_launches": 2 * args.steps,
-        "gpu_launches_note": "per step: detect_quantize_compact_kernel and the GEMM kernel "
-                             "(plus one cudaMemsetAsync of the control words)",
+        "gpu_launches": (3 if sharded else 2) * args.steps,
+        "gpu_launches_note": ("per step: detect_outliers_kernel (this rank's tokens), the "
+                              "quantisation kernel with the gathered bitmaps, the GEMM kernel "
+                              "(plus cudaMemsetAsync and the NCCL all-gather)" if sharded else
+                              "per step: detect_quantize_compact_kernel and the GEMM kernel "
+                              "(plus one cudaMemsetAsync of the control words)"),
         "clocks": clk,
     }
     if decode is not None:
@@ -477,6 +515,9 @@ def main():
                     help="seconds of oracle work for the cpu_baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--dp", default="sharded", choices=["sharded", "replicas"],
+                    help="with several ranks: split the tokens of one batch over the ranks "
+                         "(one all-gather of the outlier bitmaps per step) or run full replicas")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -489,14 +530,14 @@ def main():
         print(json.dumps(run_reference(args, ws, rank)), flush=True)
         return
 
-    ws, rank, local = dist_setup(args.gpus)
+    ws, rank, local = dist_setup(args.gpus, want_pg=(args.dp == "sharded"))
     try:
         res = run_ours(args, ws, rank, local)
         if rank == 0:
             print(json.dumps(res), flush=True)
     finally:
-        if ws > 1:
-            import torch.distributed as dist
+        import torch.distributed as dist
+        if dist.is_available() and dist.is_initialized():
             dist.destroy_process_group()
 
 

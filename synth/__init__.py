@@ -132,6 +132,17 @@ def make_workload(w: Workload | str):
     return X, W, cols
 
 
+def make_workload_shard(w: Workload | str, part: int, parts: int):
+    """Rows [part*M, (part+1)*M) of a batch of parts*M tokens drawn like the
+    workload (same weight, same planted columns and signs); with parts = 1 it is
+    make_workload(w). Returns (X shard fp16 [M,K], W fp16 [N,K], planted columns)."""
+    if isinstance(w, str):
+        w = WORKLOADS[w]
+    X, cols = make_activations(parts * w.M, w.K, w.n_outliers, w.lo, w.hi, w.seed)
+    W = make_weight(w.N, w.K, w.w_std, w.seed)
+    return np.ascontiguousarray(X[part * w.M:(part + 1) * w.M]), W, cols
+
+
 def random_case(M: int, K: int, N: int, n_outliers: int, seed: int, lo: float = 6.0,
                 hi: float = 60.0, w_std: float = 0.02, row_fraction: float = OUTLIER_ROW_FRACTION):
     """An arbitrary-shape case with the same statistics (for ragged-shape tests)."""
