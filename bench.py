@@ -253,6 +253,17 @@ def n_sets_for(w, l2_bytes):
 
 CC_MAX_OUTLIERS = 16   # up to this many outlier columns no fp16 panels are written
 
+# DRAM traffic per launch (dram__bytes_read.sum + dram__bytes_write.sum) from one
+# ncu capture of each kernel as it is now; the summaries and commands are in profiles/.
+NCU_TRAFFIC = {
+    "gemm": {"bytes": 78.000128e6 + 35.856896e6,
+             "source": "profiles/gemm_i8_persistent_opt-6.7b-ffn-up-prefill.md"},
+    "quantize": {"bytes": 27.357952e6 + 6.656e3,
+                 "source": "profiles/detect_quantize_compact_opt-6.7b-ffn-up-prefill.md"},
+    "decode": {"bytes": 19.596544e6,
+               "source": "profiles/decode_kernel_decode-16x4096x4096.md"},
+}
+
 
 def quantize_stage_bytes(w, count):
     """Algorithmic bytes of detection + quantisation (+ compaction) per call."""
@@ -379,7 +390,10 @@ def run_ours(args, ws, rank, local):
         "roofline": {"kernel": "gemm_i8_persistent_kernel (tcgen05 kind::i8, fp16 outlier epilogue)",
                      "bound": "tensor", "achieved": round(gemm_tops, 2),
                      "peak": round(int8_peak, 1), "unit": "TOPS",
-                     "frac": round(gemm_tops / int8_peak, 4), "traffic": None,
+                     "frac": round(gemm_tops / int8_peak, 4),
+                     "traffic": (NCU_TRAFFIC["gemm"]["bytes"]
+                                 if w.name == DEFAULT_WORKLOAD else None),
+                     "traffic_source": NCU_TRAFFIC["gemm"]["source"],
                      "peak_note": f"{peaks_kind} bf16 burst {bf16} TFLOP/s x {INT8_OVER_BF16} "
                                   "(dense int8 : bf16 nominal ratio)",
                      "gemm_ms": g_ms,
@@ -388,6 +402,9 @@ def run_ours(args, ws, rank, local):
                               "bound": "hbm", "achieved": round(q_gbs, 1), "peak": hbm,
                               "unit": "GB/s", "frac": round(q_gbs / hbm, 4),
                               "algorithmic_bytes": qbytes, "stage_ms": q_ms,
+                              "traffic": (NCU_TRAFFIC["quantize"]["bytes"]
+                                          if w.name == DEFAULT_WORKLOAD else None),
+                              "traffic_source": NCU_TRAFFIC["quantize"]["source"],
                               "peak_note": f"{peaks_kind} hbm_gbs"},
         "e2e": {"value": round(e2e_value, 3), "unit": "TOPS", "steps": e2e_steps,
                 "h2d_bytes_per_step": 2 * w.M * w.K, "d2h_bytes_per_step": 2 * w.M * w.N},
@@ -463,7 +480,8 @@ def bench_decode(args, stream, l2, hbm):
     gbs = nbytes / (ms / 1e3) / 1e9
     return {"workload": w.name, "M": w.M, "K": w.K, "N": w.N, "us_per_call": round(ms * 1e3, 2),
             "value": round(gbs, 1), "unit": "GB/s", "frac_of_hbm": round(gbs / hbm, 4),
-            "algorithmic_bytes": nbytes, "rotating_sets": n_sets,
+            "algorithmic_bytes": nbytes, "traffic": NCU_TRAFFIC["decode"]["bytes"],
+            "traffic_source": NCU_TRAFFIC["decode"]["source"], "rotating_sets": n_sets,
             "calls_timed": replays * per_graph, "timing": "cuda-graph replay",
             "eager_us_per_call": round(eager_ms * 1e3, 2)}
 
