@@ -15,3 +15,13 @@ from .llm_int8 import (  # noqa: F401
     llm_int8_matmul,
     llm_int8_matmul_at,
 )
+from .llm_int8 import mask_to_bitmap  # noqa: F401,E402
+from .smoothquant import (  # noqa: F401,E402
+    column_absmax,
+    smooth_factors,
+    smooth_weight_rows,
+    smooth_rcp,
+    smooth_act_rows,
+    smoothquant_matmul,
+    per_tensor_quant_dequant,
+)

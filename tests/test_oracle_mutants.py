@@ -44,3 +44,32 @@ def test_pins_catch_planted_mistake(name, tmp_path):
                         "tests/test_oracle_pins.py"], cwd=tmp_path, capture_output=True, text=True,
                        timeout=300)
     assert r.returncode != 0, f"mutant {name} survived the pins:\n{r.stdout[-2000:]}"
+
+
+SQ_MUTANTS = {
+    "sq_x_multiplied_by_s": ("return (np.float32(1.0) / np.asarray(s32, dtype=np.float32)).astype(np.float32)",
+                             "return np.asarray(s32, dtype=np.float32).copy()"),
+    "sq_alpha_swapped": ("s[ok] = a[ok] ** alpha / w[ok] ** (1.0 - alpha)",
+                         "s[ok] = a[ok] ** (1.0 - alpha) / w[ok] ** alpha"),
+    "sq_weight_not_scaled": ("W_hat = np.asarray(W).astype(np.float32) * s32[None, :]",
+                             "W_hat = np.asarray(W).astype(np.float32)"),
+    "sq_dequant_over_127": ("* np.asarray(w_scale, np.float64)[None, :] / float(QMAX_INT8 * QMAX_INT8))",
+                            "* np.asarray(w_scale, np.float64)[None, :] / float(QMAX_INT8))"),
+    "sq_weight_max_over_rows": ("w = np.max(np.abs(np.asarray(W).astype(np.float64)), axis=0)",
+                                "w = np.max(np.abs(np.asarray(W).astype(np.float64))) + 0 * np.asarray(act_absmax)"),
+}
+
+
+@pytest.mark.parametrize("name", sorted(SQ_MUTANTS))
+def test_smoothquant_pins_catch_planted_mistake(name, tmp_path):
+    src = open(os.path.join(ROOT, "oracle", "smoothquant.py")).read()
+    old, new = SQ_MUTANTS[name]
+    assert old in src, f"mutation site for {name} no longer exists"
+    for d in ("oracle", "synth", "tests"):
+        shutil.copytree(os.path.join(ROOT, d), tmp_path / d,
+                        ignore=shutil.ignore_patterns("__pycache__", "test_oracle_mutants.py"))
+    (tmp_path / "oracle" / "smoothquant.py").write_text(src.replace(old, new, 1))
+    r = subprocess.run([sys.executable, "-m", "pytest", "-q", "-x", "-p", "no:cacheprovider",
+                        "tests/test_smoothquant_pins.py"], cwd=tmp_path, capture_output=True,
+                       text=True, timeout=300)
+    assert r.returncode != 0, f"mutant {name} survived the pins:\n{r.stdout[-2000:]}"
