@@ -366,6 +366,11 @@ def run_ours(args, ws, rank, local):
     decode = None
     if args.workload != DECODE_WORKLOAD and not args.no_decode:
         decode = bench_decode(args, stream, l2, hbm)
+    smooth = None
+    if args.workload == DEFAULT_WORKLOAD and not args.no_decode:
+        smooth = bench_smoothquant(args, stream, l2,
+                                   peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+                                   * INT8_OVER_BF16, hbm)
 
     result = {
         "metric": METRIC,
@@ -418,6 +423,8 @@ def run_ours(args, ws, rank, local):
     }
     if decode is not None:
         result["decode"] = decode
+    if smooth is not None:
+        result["smoothquant"] = smooth
     if rank == 0 and not args.no_cpu_baseline:
         import oracle
         Wq_o, ws_o = oracle.quantize_weight_rows(W)
@@ -484,6 +491,52 @@ def bench_decode(args, stream, l2, hbm):
             "traffic_source": NCU_TRAFFIC["decode"]["source"], "rotating_sets": n_sets,
             "calls_timed": replays * per_graph, "timing": "cuda-graph replay",
             "eager_us_per_call": round(eager_ms * 1e3, 2)}
+
+
+def bench_smoothquant(args, stream, l2, int8_peak, hbm):
+    """SmoothQuant W8A8 on the default prefill shape: calibration, smoothing and the
+    weight side once (offline), then the runtime call (smooth + quantise kernel,
+    INT8 GEMM) timed back to back over rotating buffers."""
+    import torch
+    import w8a8_quantized_matmul_b200 as m
+    w = synth.WORKLOADS[DEFAULT_WORKLOAD]
+    X, W, _ = synth.make_workload(w)
+    Xd = torch.from_numpy(X).cuda()
+    Wd = torch.from_numpy(W).cuda()
+    act = m.int8_column_absmax(Xd)             # calibration on this batch, as the pages do
+    wmax = m.int8_column_absmax(Wd)
+    s, r = m.int8_smoothquant_factors(act, wmax, 0.5)
+    Wq, ws = m.int8_smoothquant_weight_rows(Wd, s)
+    n_sets = n_sets_for(w, l2)
+    need = m.int8_smoothquant_workspace_size(w.M, w.N, w.K)
+    sets = [dict(X=Xd if i == 0 else Xd.clone(), Wq=Wq if i == 0 else Wq.clone(),
+                 ws=ws, r=r, Y=torch.empty((w.M, w.N), dtype=torch.float16, device="cuda"),
+                 work=torch.empty((need,), dtype=torch.uint8, device="cuda"))
+            for i in range(n_sets)]
+
+    def step(i):
+        st = sets[i % n_sets]
+        m.int8_smoothquant_matmul(st["X"], st["Wq"], st["ws"], st["r"], Y=st["Y"],
+                                  workspace=st["work"])
+
+    for i in range(max(3, args.warmup)):
+        step(i)
+    steps = max(20, min(args.steps, 500))
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    a.record(stream)
+    for i in range(steps):
+        step(i)
+    b.record(stream)
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b) / steps
+    tops = 2.0 * w.M * w.N * w.K / (ms / 1e3) / 1e12
+    del sets
+    return {"workload": w.name, "alpha": 0.5, "ms_per_call": ms, "value": round(tops, 2),
+            "unit": "TOPS", "frac_of_int8_peak": round(tops / int8_peak, 4), "steps": steps,
+            "rotating_sets": n_sets,
+            "kernels": "smooth_quantize_kernel + gemm_i8_persistent_kernel (no outlier pass)"}
 
 
 # --------------------------------------------------------------------------- reference arm

@@ -161,6 +161,43 @@ int int8_mixed_matmul_profiled(const void* X, const int8_t* Wq, const float* w_s
                                void* Y, void* workspace, size_t workspace_bytes,
                                i8mm_stream_t stream, void* const* events);
 
+// ---------------------------------------------------------------- SmoothQuant W8A8
+// [Tanjunchen] "quantization explained part 2", section 4: per input channel i,
+// X_i / s_i and W_i * s_i with s_i = max|X_i|^alpha / max|W_i|^(1-alpha) leave
+// X.W unchanged (4.2) and make the activations quantisable, so both operands
+// are INT8 (W8A8, no outlier split). s is computed offline from calibration
+// activations (4.4). Here W is [N][K], so W_i is column i; the INT8 scheme after
+// smoothing is per token for X and per output row for W, codes
+// clamp(rint(fl32(fl32(v*127)/absmax)), +-127) of the smoothed fp32 values v.
+
+// colmax[k] = max(colmax[k], max over rows of |X[row][k]|) for an fp16 [rows][K]
+// matrix (running calibration statistic; also the weight's column maxima).
+// colmax: device fp32 [K], 16-byte aligned, initialised by the caller (0 to start).
+int int8_column_absmax(const void* X, int rows, int K, float* colmax, i8mm_stream_t stream);
+
+// s[k] = act_absmax[k]^alpha / w_absmax[k]^(1-alpha) (1 where either is 0) and,
+// if s_rcp is not null, s_rcp[k] = fl32(1/s[k]) (correctly rounded).
+// alpha in [0, 1]. All device fp32 [K].
+int int8_smoothquant_factors(const float* act_absmax, const float* w_absmax, int K, float alpha,
+                             float* s, float* s_rcp, i8mm_stream_t stream);
+
+// Offline weight side: W_hat = fl32(W[n][k] * s[k]), quantised per output row.
+// W fp16 [N][K] -> Wq int8 [N][K], w_scale fp32 [N] (row absmax of W_hat).
+int int8_smoothquant_weight_rows(const void* W, const float* s, int N, int K, int8_t* Wq,
+                                 float* w_scale, i8mm_stream_t stream);
+
+// Bytes of workspace int8_smoothquant_matmul needs (0 for invalid sizes).
+size_t int8_smoothquant_workspace_size(int M, int N, int K);
+
+// Runtime W8A8 path: X_hat = fl32(X[m][k] * s_rcp[k]), per-token absmax codes
+// (Xq and x_scale left in the workspace), INT8 x INT8 -> INT32 on the tensor
+// cores, Y = fp16(C * x_scale * w_scale / 127^2). X fp16 [M][K], Wq/w_scale from
+// int8_smoothquant_weight_rows, s_rcp fp32 [K], Y fp16 [M][N]. Alignment,
+// workspace and error rules as int8_mixed_matmul (256-byte aligned workspace).
+int int8_smoothquant_matmul(const void* X, const int8_t* Wq, const float* w_scale,
+                            const float* s_rcp, int M, int N, int K, void* Y, void* workspace,
+                            size_t workspace_bytes, i8mm_stream_t stream);
+
 // Token-sharded (data-parallel over tokens) form of int8_mixed_matmul, one call
 // per rank on that rank's rows of X. AIInfra "05Quantization01", LLM.int8()
 // section: the outlier feature dimensions are those where any token of the

@@ -1,0 +1,109 @@
+"""SmoothQuant W8A8 CUDA path against the oracle ([Tanjunchen] "quantization
+explained part 2", section 4). Integer outputs (codes) and the column maxima are
+compared bit for bit; the factors (fp32 powers) and Y within tolerance."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+import w8a8_quantized_matmul_b200 as m
+
+pytestmark = pytest.mark.gpu
+
+MAX_REL, MEAN_REL = 1e-2, 1e-3
+
+
+def _y_close(Y, Yref):
+    Y = Y.astype(np.float64)
+    Yref = Yref.astype(np.float64)
+    d = np.abs(Y - Yref)
+    assert d.max() <= MAX_REL * np.abs(Yref).max()
+    assert d.mean() <= MEAN_REL * np.abs(Yref).mean()
+
+
+def test_column_absmax_running():
+    X1, _, _ = synth.random_case(300, 528, 8, 5, seed=41)
+    X2, _, _ = synth.random_case(77, 528, 8, 3, seed=42)
+    cm = m.int8_column_absmax(torch.from_numpy(X1).cuda())
+    cm = m.int8_column_absmax(torch.from_numpy(X2).cuda(), colmax=cm)
+    ref = np.maximum(oracle.column_absmax(X1), oracle.column_absmax(X2))
+    np.testing.assert_array_equal(cm.cpu().numpy(), ref)
+
+
+@pytest.mark.parametrize("alpha", [0.0, 0.5, 0.85, 1.0])
+def test_factors(alpha):
+    X, W, _ = synth.random_case(128, 512, 96, 6, seed=43)
+    W[:, 7] = 0          # an empty weight channel
+    X[:, 9] = 0          # an empty activation channel
+    act = m.int8_column_absmax(torch.from_numpy(X).cuda())
+    wmax = m.int8_column_absmax(torch.from_numpy(W).cuda())
+    s, r = m.int8_smoothquant_factors(act, wmax, alpha)
+    s = s.cpu().numpy()
+    ref = oracle.smooth_factors(oracle.column_absmax(X), W, alpha)
+    np.testing.assert_allclose(s, ref, rtol=4e-7)
+    assert s[7] == 1.0 and s[9] == 1.0
+    np.testing.assert_array_equal(r.cpu().numpy(), np.float32(1.0) / s)
+
+
+CASES = [
+    (64, 512, 256, 4),
+    (300, 1040, 136, 3),
+    (16, 4096, 512, 6),
+    (2048, 4096, 1024, 6),
+    (129, 272, 264, 0),
+]
+
+
+@pytest.mark.parametrize("case", CASES, ids=[f"M{c[0]}-K{c[1]}-N{c[2]}-o{c[3]}" for c in CASES])
+def test_matmul_parity(case):
+    M, K, N, n_out = case
+    X, W, _ = synth.random_case(M, K, N, n_out, seed=M * 7 + K + N)
+    W[:, 3] = 0
+    X[:, 5] = 0
+    s32 = oracle.smooth_factors(oracle.column_absmax(X), W, 0.5).astype(np.float32)
+    r32 = oracle.smooth_rcp(s32)
+    Wq_ref, ws_ref, _ = oracle.smooth_weight_rows(W, s32)
+    ref = oracle.smoothquant_matmul(X, Wq_ref, ws_ref, r32)
+
+    Wd = torch.from_numpy(W).cuda()
+    Wq, ws = m.int8_smoothquant_weight_rows(Wd, torch.from_numpy(s32).cuda())
+    np.testing.assert_array_equal(Wq.cpu().numpy(), Wq_ref)
+    np.testing.assert_array_equal(ws.cpu().numpy(), ws_ref)
+
+    Y, work = m.int8_smoothquant_matmul(torch.from_numpy(X).cuda(), Wq, ws,
+                                        torch.from_numpy(r32).cuda())
+    torch.cuda.synchronize()
+    v = m.smoothquant_workspace_views(work, M, K)
+    assert int(v["status"].item()) == 0
+    np.testing.assert_array_equal(v["x_scale"].cpu().numpy(), ref["x_scale"])
+    np.testing.assert_array_equal(v["Xq"].cpu().numpy(), ref["Xq"])
+    _y_close(Y.cpu().numpy(), ref["Y"])
+
+
+def test_all_gpu_pipeline_beats_plain_int8():
+    """Calibrate, smooth and run entirely on the GPU; the smoothed W8A8 output is
+    closer to the exact product than the unsmoothed one (section 4.5's claim)."""
+    M, K, N = 512, 1024, 256
+    X, W, _ = synth.random_case(M, K, N, 6, seed=77)
+    Xd, Wd = torch.from_numpy(X).cuda(), torch.from_numpy(W).cuda()
+    exact = X.astype(np.float64) @ W.astype(np.float64).T
+    act = m.int8_column_absmax(Xd)
+    wmax = m.int8_column_absmax(Wd)
+    errs = []
+    for alpha in (0.0, 0.5):
+        if alpha == 0.0:
+            s = torch.ones(K, dtype=torch.float32, device="cuda")
+            r = s.clone()
+        else:
+            s, r = m.int8_smoothquant_factors(act, wmax, alpha)
+        Wq, ws = m.int8_smoothquant_weight_rows(Wd, s)
+        Y, _ = m.int8_smoothquant_matmul(Xd, Wq, ws, r)
+        errs.append(np.abs(Y.cpu().numpy().astype(np.float64) - exact).mean())
+    assert errs[1] < 0.7 * errs[0]
+
+
+def test_invalid_arguments():
+    X = torch.zeros((4, 24), dtype=torch.float16, device="cuda")   # K % 16 != 0
+    with pytest.raises(m.Int8mmError):
+        m.int8_column_absmax(X)

@@ -38,6 +38,11 @@ __all__ = [
     "int8_mixed_matmul_stage",
     "int8_mixed_matmul_sharded",
     "int8_debug_gemm_i32",
+    "int8_column_absmax",
+    "int8_smoothquant_factors",
+    "int8_smoothquant_weight_rows",
+    "int8_smoothquant_workspace_size",
+    "int8_smoothquant_matmul",
     "int8_device_status",
     "Int8mmError",
 ]
@@ -204,6 +209,79 @@ def int8_mixed_matmul_sharded(X, Wq, w_scale, W_fp16, bitmaps, Y=None, workspace
                                            workspace.numel() * workspace.element_size(),
                                            _stream(stream)))
     return Y, workspace
+
+
+def int8_column_absmax(X, colmax=None, stream=None):
+    """Running column max |x| of fp16 [rows, K] into fp32 colmax [K] (zeros if None)."""
+    rows, K = X.shape
+    _need(X, "X", torch.float16, (rows, K))
+    colmax = torch.zeros((K,), dtype=torch.float32, device=X.device) if colmax is None else colmax
+    _need(colmax, "colmax", torch.float32, (K,))
+    check("int8_column_absmax",
+          load().int8_column_absmax(_ptr(X), rows, K, _ptr(colmax), _stream(stream)))
+    return colmax
+
+
+def int8_smoothquant_factors(act_absmax, w_absmax, alpha=0.5, s=None, s_rcp=None, stream=None):
+    """SmoothQuant factors s [K] and their reciprocals fl32(1/s) [K]."""
+    K = act_absmax.numel()
+    _need(act_absmax, "act_absmax", torch.float32, (K,))
+    _need(w_absmax, "w_absmax", torch.float32, (K,))
+    s = torch.empty((K,), dtype=torch.float32, device=act_absmax.device) if s is None else s
+    s_rcp = torch.empty_like(s) if s_rcp is None else s_rcp
+    check("int8_smoothquant_factors",
+          load().int8_smoothquant_factors(_ptr(act_absmax), _ptr(w_absmax), K, float(alpha),
+                                          _ptr(s), _ptr(s_rcp), _stream(stream)))
+    return s, s_rcp
+
+
+def int8_smoothquant_weight_rows(W, s, Wq=None, w_scale=None, stream=None):
+    """fp16 W [N, K] and factors s [K] -> (Wq int8 [N, K], w_scale fp32 [N]) of W * s."""
+    N, K = W.shape
+    _need(W, "W", torch.float16, (N, K))
+    _need(s, "s", torch.float32, (K,))
+    Wq = torch.empty((N, K), dtype=torch.int8, device=W.device) if Wq is None else Wq
+    w_scale = torch.empty((N,), dtype=torch.float32, device=W.device) if w_scale is None else w_scale
+    check("int8_smoothquant_weight_rows",
+          load().int8_smoothquant_weight_rows(_ptr(W), _ptr(s), N, K, _ptr(Wq), _ptr(w_scale),
+                                              _stream(stream)))
+    return Wq, w_scale
+
+
+def int8_smoothquant_workspace_size(M: int, N: int, K: int) -> int:
+    return int(load().int8_smoothquant_workspace_size(M, N, K))
+
+
+def int8_smoothquant_matmul(X, Wq, w_scale, s_rcp, Y=None, workspace=None, stream=None):
+    """SmoothQuant W8A8 runtime path; returns (Y fp16 [M, N], workspace)."""
+    M, K = X.shape
+    N = Wq.shape[0]
+    _need(X, "X", torch.float16, (M, K))
+    _need(Wq, "Wq", torch.int8, (N, K))
+    _need(w_scale, "w_scale", torch.float32, (N,))
+    _need(s_rcp, "s_rcp", torch.float32, (K,))
+    Y = torch.empty((M, N), dtype=torch.float16, device=X.device) if Y is None else Y
+    _need(Y, "Y", torch.float16, (M, N))
+    need = int8_smoothquant_workspace_size(M, N, K)
+    if workspace is None:
+        workspace = torch.empty((max(need, 1),), dtype=torch.uint8, device=X.device)
+    check("int8_smoothquant_matmul",
+          load().int8_smoothquant_matmul(_ptr(X), _ptr(Wq), _ptr(w_scale), _ptr(s_rcp), M, N, K,
+                                         _ptr(Y), _ptr(workspace),
+                                         workspace.numel() * workspace.element_size(),
+                                         _stream(stream)))
+    return Y, workspace
+
+
+def smoothquant_workspace_views(workspace: torch.Tensor, M: int, K: int) -> dict:
+    """x_scale fp32 [M] and Xq int8 [M, K] that int8_smoothquant_matmul leaves in its workspace."""
+    def up(x):
+        return (x + 255) // 256 * 256
+    xs_off = up(16)
+    xq_off = up(xs_off + 4 * M)
+    return dict(status=workspace[0:4].view(torch.int32),
+                x_scale=workspace[xs_off:xs_off + 4 * M].view(torch.float32),
+                Xq=workspace[xq_off:xq_off + M * K].view(torch.int8).view(M, K))
 
 
 def int8_debug_gemm_i32(Xq, Wq, C=None, stream=None):
