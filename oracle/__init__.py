@@ -15,7 +15,7 @@ from .llm_int8 import (  # noqa: F401
     llm_int8_matmul,
     llm_int8_matmul_at,
 )
-from .llm_int8 import mask_to_bitmap  # noqa: F401,E402
+from .llm_int8 import mask_to_bitmap, find_topk_cols  # noqa: F401,E402
 from .smoothquant import (  # noqa: F401,E402
     column_absmax,
     smooth_factors,

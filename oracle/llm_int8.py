@@ -127,6 +127,25 @@ def find_outlier_cols(X: np.ndarray, threshold: float):
     return mask, bitmap, int(idx.size), idx
 
 
+def find_topk_cols(X: np.ndarray, k: int) -> np.ndarray:
+    """Mask (bool [K]) of the k columns with the largest max |x| over the rows.
+
+    [AIInfra] LLM.int8() section, training notes: raise the decomposition ratio
+    by computing the top 1% or 2% largest-magnitude feature dimensions in FP16.
+    The magnitude of a column is its max |x| over the rows (the statistic the
+    threshold detection compares); ties go to the lower column index; k is
+    clipped to [0, K].
+    """
+    X32 = np.asarray(X).astype(np.float32)
+    K = X32.shape[1]
+    k = max(0, min(int(k), K))
+    colmax = np.max(np.abs(X32), axis=0) if X32.shape[0] else np.zeros(K, np.float32)
+    order = sorted(range(K), key=lambda j: (-float(colmax[j]), j))
+    mask = np.zeros(K, bool)
+    mask[order[:k]] = True
+    return mask
+
+
 # ---------------------------------------------------------------------------
 # Per-token absmax INT8 quantisation of the non-outlier part ([AIInfra]
 # vector-wise quantisation of each row of X after the outliers are split

@@ -73,3 +73,26 @@ def test_smoothquant_pins_catch_planted_mistake(name, tmp_path):
                         "tests/test_smoothquant_pins.py"], cwd=tmp_path, capture_output=True,
                        text=True, timeout=300)
     assert r.returncode != 0, f"mutant {name} survived the pins:\n{r.stdout[-2000:]}"
+
+
+TOPK_MUTANTS = {
+    "topk_ties_to_higher_index": ("key=lambda j: (-float(colmax[j]), j))", "key=lambda j: (-float(colmax[j]), -j))"),
+    "topk_one_extra_column": ("mask[order[:k]] = True", "mask[order[:k + 1]] = True"),
+    "topk_by_mean_magnitude": ("colmax = np.max(np.abs(X32), axis=0) if X32.shape[0] else np.zeros(K, np.float32)\n    order",
+                               "colmax = np.mean(np.abs(X32), axis=0) if X32.shape[0] else np.zeros(K, np.float32)\n    order"),
+}
+
+
+@pytest.mark.parametrize("name", sorted(TOPK_MUTANTS))
+def test_topk_pins_catch_planted_mistake(name, tmp_path):
+    src = open(os.path.join(ROOT, "oracle", "llm_int8.py")).read()
+    old, new = TOPK_MUTANTS[name]
+    assert old in src, f"mutation site for {name} no longer exists"
+    for d in ("oracle", "synth", "tests"):
+        shutil.copytree(os.path.join(ROOT, d), tmp_path / d,
+                        ignore=shutil.ignore_patterns("__pycache__", "test_oracle_mutants.py"))
+    (tmp_path / "oracle" / "llm_int8.py").write_text(src.replace(old, new, 1))
+    r = subprocess.run([sys.executable, "-m", "pytest", "-q", "-x", "-p", "no:cacheprovider",
+                        "tests/test_topk_pins.py"], cwd=tmp_path, capture_output=True, text=True,
+                       timeout=300)
+    assert r.returncode != 0, f"mutant {name} survived the pins:\n{r.stdout[-2000:]}"
