@@ -161,6 +161,21 @@ int int8_mixed_matmul_profiled(const void* X, const int8_t* Wq, const float* w_s
                                void* Y, void* workspace, size_t workspace_bytes,
                                i8mm_stream_t stream, void* const* events);
 
+// ---------------------------------------------------------------- top-k decomposition
+// [AIInfra] "05Quantization01", LLM.int8() section, training notes: raise the
+// decomposition ratio by computing the top 1% or 2% largest-magnitude feature
+// dimensions in FP16. The outlier set is the k columns of X with the largest
+// max |x| over the M tokens (ties to the lower column index; k >= K selects all
+// columns); the rest of the path is int8_mixed_matmul with that set (per-token
+// absmax codes of the other columns, INT8 product, FP16 product over the set).
+// Arguments, layout and errors as int8_mixed_matmul, except k (>= 0) instead
+// of the threshold and the larger workspace below; the workspace's bitmap,
+// count and list describe the selected set. Always runs the prefill kernels.
+size_t int8_mixed_matmul_topk_workspace_size(int M, int N, int K);
+int int8_mixed_matmul_topk(const void* X, const int8_t* Wq, const float* w_scale,
+                           const void* W_fp16, int M, int N, int K, int k, void* Y,
+                           void* workspace, size_t workspace_bytes, i8mm_stream_t stream);
+
 // ---------------------------------------------------------------- SmoothQuant W8A8
 // [Tanjunchen] "quantization explained part 2", section 4: per input channel i,
 // X_i / s_i and W_i * s_i with s_i = max|X_i|^alpha / max|W_i|^(1-alpha) leave

@@ -39,6 +39,7 @@ __all__ = [
     "int8_mixed_matmul_sharded",
     "int8_debug_gemm_i32",
     "int8_column_absmax",
+    "int8_mixed_matmul_topk",
     "int8_smoothquant_factors",
     "int8_smoothquant_weight_rows",
     "int8_smoothquant_workspace_size",
@@ -208,6 +209,28 @@ def int8_mixed_matmul_sharded(X, Wq, w_scale, W_fp16, bitmaps, Y=None, workspace
                                            _ptr(workspace),
                                            workspace.numel() * workspace.element_size(),
                                            _stream(stream)))
+    return Y, workspace
+
+
+def int8_mixed_matmul_topk(X, Wq, w_scale, W_fp16, k, Y=None, workspace=None, stream=None):
+    """LLM.int8() matmul whose outlier set is the k columns of largest max |x|.
+    Returns (Y fp16 [M, N], workspace); workspace_views() reads the intermediates."""
+    M, K = X.shape
+    N = Wq.shape[0]
+    _need(X, "X", torch.float16, (M, K))
+    _need(Wq, "Wq", torch.int8, (N, K))
+    _need(w_scale, "w_scale", torch.float32, (N,))
+    _need(W_fp16, "W_fp16", torch.float16, (N, K))
+    Y = torch.empty((M, N), dtype=torch.float16, device=X.device) if Y is None else Y
+    _need(Y, "Y", torch.float16, (M, N))
+    need = int(load().int8_mixed_matmul_topk_workspace_size(M, N, K))
+    if workspace is None:
+        workspace = torch.empty((max(need, 1),), dtype=torch.uint8, device=X.device)
+    check("int8_mixed_matmul_topk",
+          load().int8_mixed_matmul_topk(_ptr(X), _ptr(Wq), _ptr(w_scale), _ptr(W_fp16), M, N, K,
+                                        int(k), _ptr(Y), _ptr(workspace),
+                                        workspace.numel() * workspace.element_size(),
+                                        _stream(stream)))
     return Y, workspace
 
 

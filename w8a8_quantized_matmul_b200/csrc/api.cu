@@ -340,6 +340,47 @@ int int8_mixed_matmul_stage(int stage, const void* X, const int8_t* Wq, const fl
                            workspace_bytes, stream, nullptr, stage);
 }
 
+// Extra workspace of the top-k path, after the regular layout: column maxima
+// (fp32 [K]) and the selection bitmap (ceil(K/32) words), each 256-byte aligned.
+size_t int8_mixed_matmul_topk_workspace_size(int M, int N, int K) {
+  Layout L;
+  if (!make_layout(M, N, K, &L)) return 0;
+  const size_t colmax = (L.l.total + 255) & ~static_cast<size_t>(255);
+  const size_t sel = (colmax + static_cast<size_t>(K) * 4 + 255) & ~static_cast<size_t>(255);
+  return (sel + static_cast<size_t>((K + 31) / 32) * 4 + 255) & ~static_cast<size_t>(255);
+}
+
+int int8_mixed_matmul_topk(const void* X, const int8_t* Wq, const float* w_scale,
+                           const void* W_fp16, int M, int N, int K, int k, void* Y,
+                           void* workspace, size_t workspace_bytes, i8mm_stream_t stream) {
+  int st = check_sizes(M, N, K);
+  if (st != I8MM_OK) return st;
+  if (k < 0) return I8MM_ERR_INVALID_ARG;
+  if (M == 0 || N == 0) return I8MM_OK;
+  if (!X || !workspace) return I8MM_ERR_INVALID_ARG;
+  if (!aligned16(X)) return I8MM_ERR_ALIGNMENT;
+  Layout L;
+  make_layout(M, N, K, &L);
+  const size_t need = int8_mixed_matmul_topk_workspace_size(M, N, K);
+  if (workspace_bytes < need) return I8MM_ERR_WORKSPACE;
+  if ((reinterpret_cast<uintptr_t>(workspace) & (kAlign - 1)) != 0) return I8MM_ERR_ALIGNMENT;
+  if ((st = check_device()) != I8MM_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  const size_t colmax_off = (L.l.total + 255) & ~static_cast<size_t>(255);
+  const size_t sel_off = (colmax_off + static_cast<size_t>(K) * 4 + 255) & ~static_cast<size_t>(255);
+  float* colmax = reinterpret_cast<float*>(ws + colmax_off);
+  uint32_t* sel = reinterpret_cast<uint32_t*>(ws + sel_off);
+  cudaError_t e = cudaMemsetAsync(colmax, 0, static_cast<size_t>(K) * 4, s);
+  if (e != cudaSuccess) return cuda_fail("column-max memset", e);
+  e = launch_column_absmax(static_cast<const __half*>(X), M, K, colmax, s);
+  if (e != cudaSuccess) return cuda_fail("column_absmax_kernel launch", e);
+  e = launch_topk_select(colmax, K, k, sel, s);
+  if (e != cudaSuccess) return cuda_fail("topk_select_kernel launch", e);
+  return mixed_matmul_impl(X, Wq, w_scale, W_fp16, M, N, K, 0.0f, Y, workspace, workspace_bytes,
+                           s, nullptr, 3, sel, 1);
+}
+
 int int8_mixed_matmul_sharded(const void* X, const int8_t* Wq, const float* w_scale,
                               const void* W_fp16, int M, int N, int K, const uint32_t* bitmaps,
                               int n_bitmaps, void* Y, void* workspace, size_t workspace_bytes,

@@ -114,6 +114,12 @@ struct DecodeArgs {
 };
 
 bool decode_supported(int M, int K);
+
+// Running column max |x| of an fp16 [rows][K] matrix into fp32 colmax [K]
+// (smoothquant.cu) and the top-k column selection into a bitmap (topk.cu).
+cudaError_t launch_column_absmax(const __half* X, int rows, int K, float* colmax, cudaStream_t s);
+cudaError_t launch_topk_select(const float* colmax, int K, int k, uint32_t* bitmap,
+                               cudaStream_t s);
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t s);
 
 }  // namespace i8mm

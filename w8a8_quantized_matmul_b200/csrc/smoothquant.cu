@@ -176,6 +176,15 @@ int sq_sizes(int M, int N, int K) {
 
 }  // namespace
 
+cudaError_t launch_column_absmax(const __half* X, int rows, int K, float* colmax,
+                                 cudaStream_t s) {
+  const int nv = K / 8;
+  const int row_slice = 64;
+  dim3 grid((nv + kThreads - 1) / kThreads, (rows + row_slice - 1) / row_slice);
+  column_absmax_kernel<<<grid, kThreads, 0, s>>>(X, rows, K, row_slice, colmax);
+  return cudaGetLastError();
+}
+
 }  // namespace i8mm
 
 using namespace i8mm;
@@ -187,12 +196,8 @@ int int8_column_absmax(const void* X, int rows, int K, float* colmax, i8mm_strea
   if (rows == 0) return I8MM_OK;
   if (!X || !colmax) return I8MM_ERR_INVALID_ARG;
   if (!a16(X) || !a16(colmax)) return I8MM_ERR_ALIGNMENT;
-  const int nv = K / 8;
-  const int row_slice = 64;
-  dim3 grid((nv + kThreads - 1) / kThreads, (rows + row_slice - 1) / row_slice);
-  column_absmax_kernel<<<grid, kThreads, 0, static_cast<cudaStream_t>(stream)>>>(
-      static_cast<const __half*>(X), rows, K, row_slice, colmax);
-  return sq_status(cudaGetLastError());
+  return sq_status(launch_column_absmax(static_cast<const __half*>(X), rows, K, colmax,
+                                        static_cast<cudaStream_t>(stream)));
 }
 
 int int8_smoothquant_factors(const float* act_absmax, const float* w_absmax, int K, float alpha,
