@@ -15,7 +15,10 @@ from .llm_int8 import (  # noqa: F401
     llm_int8_matmul,
     llm_int8_matmul_at,
 )
-from .llm_int8 import mask_to_bitmap, find_topk_cols  # noqa: F401,E402
+from .llm_int8 import (  # noqa: F401,E402
+    mask_to_bitmap, find_topk_cols, quantize_act_rows_zp, weight_rowsum, dequantize_zp,
+    ZP_QMIN, ZP_QMAX,
+)
 from .smoothquant import (  # noqa: F401,E402
     column_absmax,
     smooth_factors,

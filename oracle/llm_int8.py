@@ -209,6 +209,58 @@ def outlier_gemm(X: np.ndarray, W: np.ndarray, idx: np.ndarray) -> np.ndarray:
 
 
 # ---------------------------------------------------------------------------
+# Zero-point (asymmetric) per-token quantisation ([Scholia] section 6:
+# q = clip(round(x/s) + z, qmin, qmax), x_hat = s(q - z), z the integer that
+# represents real 0; [AIInfra] LLM.int8() section: zeropoint beats absmax below
+# 6.7B because the outliers are one-sided).
+# ---------------------------------------------------------------------------
+ZP_QMIN, ZP_QMAX = -128, 127
+
+
+def quantize_act_rows_zp(X: np.ndarray, outlier_mask: np.ndarray):
+    """Per-token zero-point INT8 codes of the non-outlier columns.
+
+    Returns (Xq int8 [M, K], step fp32 [M], zero int32 [M]). Per row, over the
+    non-outlier columns: lo = min(0, min x), hi = max(0, max x) (the range keeps
+    real 0 so that it maps to an integer), step = fl32(fl32(hi - lo) / 255),
+    zero = clamp(-128 - rint(fl32(lo / step)), -128, 127), and
+    q = clamp(rint(fl32(x / step)) + zero, -128, 127). At outlier columns q =
+    zero, so (q - zero) is 0 there. A row with no nonzero kept entry gets step 0,
+    zero 0 and all codes 0.
+    """
+    X32 = np.asarray(X).astype(np.float32)
+    keep = ~np.asarray(outlier_mask, dtype=bool)
+    kept = np.where(keep[None, :], X32, np.float32(0))
+    hi = np.maximum(np.max(kept, axis=1), np.float32(0)) if X32.shape[1] else np.zeros(X32.shape[0], np.float32)
+    lo = np.minimum(np.min(kept, axis=1), np.float32(0)) if X32.shape[1] else np.zeros(X32.shape[0], np.float32)
+    step = ((hi - lo).astype(np.float32) / np.float32(255)).astype(np.float32)
+    live = step > 0
+    safe = np.where(live, step, np.float32(1))
+    zero = np.where(live, np.clip(ZP_QMIN - np.rint((lo / safe).astype(np.float32)), ZP_QMIN, ZP_QMAX), 0)
+    zero = zero.astype(np.int32)
+    with np.errstate(divide="ignore", invalid="ignore"):
+        q = np.rint((X32 / safe[:, None]).astype(np.float32)) + zero[:, None]
+    q = np.clip(q, ZP_QMIN, ZP_QMAX)
+    q = np.where(live[:, None], q, 0)
+    q = np.where(keep[None, :], q, zero[:, None])
+    return q.astype(np.int8), step.astype(np.float32), zero
+
+
+def weight_rowsum(Wq: np.ndarray) -> np.ndarray:
+    """sum_k Wq[n, k] (int32 [N]), the zero-point correction's weight factor."""
+    return np.sum(np.asarray(Wq, dtype=np.int64), axis=1).astype(np.int32)
+
+
+def dequantize_zp(C: np.ndarray, zero: np.ndarray, step: np.ndarray, wsum: np.ndarray,
+                  w_scale: np.ndarray) -> np.ndarray:
+    """sum_k step*(q - zero)*w_scale/127*wq = step*w_scale/127*(C - zero*wsum), float64."""
+    Ccor = (np.asarray(C, np.int64) - np.asarray(zero, np.int64)[:, None]
+            * np.asarray(wsum, np.int64)[None, :])
+    return (Ccor.astype(np.float64) * np.asarray(step, np.float64)[:, None]
+            * np.asarray(w_scale, np.float64)[None, :] / float(QMAX_INT8))
+
+
+# ---------------------------------------------------------------------------
 # Full decomposition ([AIInfra]: C_f16 = C_outlier + C_normal).
 # ---------------------------------------------------------------------------
 def mask_to_bitmap(mask: np.ndarray):
@@ -224,7 +276,7 @@ def mask_to_bitmap(mask: np.ndarray):
 
 def llm_int8_matmul(X: np.ndarray, W: np.ndarray, threshold: float = 6.0,
                     Wq: np.ndarray | None = None, w_scale: np.ndarray | None = None,
-                    outlier_mask: np.ndarray | None = None):
+                    outlier_mask: np.ndarray | None = None, zeropoint: bool = False):
     """All steps of the path; returns a dict with Y (fp16 [M, N]) and every intermediate.
 
     `W` is the fp16 weight [N, K]; it supplies the outlier columns of the
@@ -233,6 +285,9 @@ def llm_int8_matmul(X: np.ndarray, W: np.ndarray, threshold: float = 6.0,
     set: the set of a batch whose tokens are split over several processes
     ([AIInfra]: O is a property of the batch's activations, so every part of
     the batch uses the same O); the threshold is then unused.
+    `zeropoint` quantises the non-outlier part of each token with a zero point
+    (quantize_act_rows_zp) instead of the symmetric absmax; x_scale then holds
+    the step and the result also has `zero` and `wsum`.
     """
     X = np.asarray(X)
     W = np.asarray(W)
@@ -243,13 +298,21 @@ def llm_int8_matmul(X: np.ndarray, W: np.ndarray, threshold: float = 6.0,
     else:
         mask = np.asarray(outlier_mask, dtype=bool)
         bitmap, count, idx = mask_to_bitmap(mask)
-    Xq, x_scale = quantize_act_rows(X, mask)
-    C = int32_gemm(Xq, Wq)
-    Cn = dequantize(C, x_scale, w_scale)
+    extra = {}
+    if zeropoint:
+        Xq, x_scale, zero = quantize_act_rows_zp(X, mask)
+        C = int32_gemm(Xq, Wq)
+        wsum = weight_rowsum(Wq)
+        Cn = dequantize_zp(C, zero, x_scale, wsum, w_scale)
+        extra = dict(zero=zero, wsum=wsum)
+    else:
+        Xq, x_scale = quantize_act_rows(X, mask)
+        C = int32_gemm(Xq, Wq)
+        Cn = dequantize(C, x_scale, w_scale)
     Co = outlier_gemm(X, W, idx)
     Y = (Cn + Co).astype(np.float16)
     return dict(Y=Y, mask=mask, bitmap=bitmap, count=count, idx=idx, Xq=Xq,
-                x_scale=x_scale, Wq=Wq, w_scale=w_scale, C=C, C_normal=Cn, C_outlier=Co)
+                x_scale=x_scale, Wq=Wq, w_scale=w_scale, C=C, C_normal=Cn, C_outlier=Co, **extra)
 
 
 def llm_int8_matmul_at(X: np.ndarray, W: np.ndarray, Wq: np.ndarray, w_scale: np.ndarray,

@@ -96,3 +96,30 @@ def test_topk_pins_catch_planted_mistake(name, tmp_path):
                         "tests/test_topk_pins.py"], cwd=tmp_path, capture_output=True, text=True,
                        timeout=300)
     assert r.returncode != 0, f"mutant {name} survived the pins:\n{r.stdout[-2000:]}"
+
+
+ZP_MUTANTS = {
+    "zp_zero_sign_flipped": ("zero = np.where(live, np.clip(ZP_QMIN - np.rint((lo / safe).astype(np.float32)), ZP_QMIN, ZP_QMAX), 0)",
+                             "zero = np.where(live, np.clip(ZP_QMIN + np.rint((lo / safe).astype(np.float32)), ZP_QMIN, ZP_QMAX), 0)"),
+    "zp_range_without_zero": ("lo = np.minimum(np.min(kept, axis=1), np.float32(0))",
+                              "lo = np.min(np.where(keep[None, :], X32, np.float32(np.inf)), axis=1) + 0 * np.float32(0)"),
+    "zp_correction_dropped": ("Ccor = (np.asarray(C, np.int64) - np.asarray(zero, np.int64)[:, None]",
+                              "Ccor = (np.asarray(C, np.int64) - 0 * np.asarray(zero, np.int64)[:, None]"),
+    "zp_step_over_127": ("step = ((hi - lo).astype(np.float32) / np.float32(255)).astype(np.float32)",
+                         "step = ((hi - lo).astype(np.float32) / np.float32(127)).astype(np.float32)"),
+}
+
+
+@pytest.mark.parametrize("name", sorted(ZP_MUTANTS))
+def test_zeropoint_pins_catch_planted_mistake(name, tmp_path):
+    src = open(os.path.join(ROOT, "oracle", "llm_int8.py")).read()
+    old, new = ZP_MUTANTS[name]
+    assert old in src, f"mutation site for {name} no longer exists"
+    for d in ("oracle", "synth", "tests"):
+        shutil.copytree(os.path.join(ROOT, d), tmp_path / d,
+                        ignore=shutil.ignore_patterns("__pycache__", "test_oracle_mutants.py"))
+    (tmp_path / "oracle" / "llm_int8.py").write_text(src.replace(old, new, 1))
+    r = subprocess.run([sys.executable, "-m", "pytest", "-q", "-x", "-p", "no:cacheprovider",
+                        "tests/test_zeropoint_pins.py"], cwd=tmp_path, capture_output=True,
+                       text=True, timeout=300)
+    assert r.returncode != 0, f"mutant {name} survived the pins:\n{r.stdout[-2000:]}"
