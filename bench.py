@@ -428,6 +428,7 @@ def run_ours(args, ws, rank, local):
     if args.workload == DEFAULT_WORKLOAD and not args.no_decode:
         i8p = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]) * INT8_OVER_BF16
         result["topk"] = [bench_topk(args, stream, l2, i8p, f) for f in (0.01, 0.02)]
+        result["zeropoint"] = bench_zeropoint(args, stream, l2, i8p)
     if rank == 0 and not args.no_cpu_baseline:
         import oracle
         Wq_o, ws_o = oracle.quantize_weight_rows(W)
@@ -585,6 +586,51 @@ def bench_topk(args, stream, l2, int8_peak, fraction):
             "steps": steps, "rotating_sets": n_sets,
             "kernels": "column max, top-k select, quantisation with the selected set, GEMM "
                        "(outlier product on the tensor cores for k > 16)"}
+
+
+def bench_zeropoint(args, stream, l2, int8_peak):
+    """The decomposition with zero-point codes on the default prefill shape, timed
+    back to back over rotating buffers (weight row sums computed once, offline)."""
+    import torch
+    import w8a8_quantized_matmul_b200 as m
+    w = synth.WORKLOADS[DEFAULT_WORKLOAD]
+    X, W, _ = synth.make_workload(w)
+    Xd = torch.from_numpy(X).cuda()
+    Wd = torch.from_numpy(W).cuda()
+    Wq, ws = m.int8_quantize_weight_rows(Wd)
+    rsum = m.int8_weight_rowsum(Wq)
+    n_sets = n_sets_for(w, l2)
+    need = int(m.load().int8_mixed_matmul_zp_workspace_size(w.M, w.N, w.K))
+    sets = [dict(X=Xd if i == 0 else Xd.clone(), Wq=Wq if i == 0 else Wq.clone(), ws=ws,
+                 W=Wd if i == 0 else Wd.clone(),
+                 Y=torch.empty((w.M, w.N), dtype=torch.float16, device="cuda"),
+                 work=torch.empty((need,), dtype=torch.uint8, device="cuda"))
+            for i in range(n_sets)]
+
+    def step(i):
+        st = sets[i % n_sets]
+        m.int8_mixed_matmul_zp(st["X"], st["Wq"], st["ws"], rsum, st["W"], w.threshold,
+                               Y=st["Y"], workspace=st["work"])
+
+    for i in range(max(3, args.warmup)):
+        step(i)
+    steps = max(20, min(args.steps, 500))
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    a.record(stream)
+    for i in range(steps):
+        step(i)
+    b.record(stream)
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b) / steps
+    tops = 2.0 * w.M * w.N * w.K / (ms / 1e3) / 1e12
+    del sets
+    return {"workload": w.name, "threshold": w.threshold, "ms_per_call": ms,
+            "value": round(tops, 2), "unit": "TOPS", "frac_of_int8_peak": round(tops / int8_peak, 4),
+            "steps": steps, "rotating_sets": n_sets,
+            "kernels": "detect_quantize_compact_kernel<., zero-point> + "
+                       "gemm_i8_persistent_kernel<., ., zero-point>"}
 
 
 # --------------------------------------------------------------------------- reference arm

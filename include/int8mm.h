@@ -161,6 +161,32 @@ int int8_mixed_matmul_profiled(const void* X, const int8_t* Wq, const float* w_s
                                void* Y, void* workspace, size_t workspace_bytes,
                                i8mm_stream_t stream, void* const* events);
 
+// ---------------------------------------------------------------- zero-point rows
+// [Scholia] "Inference Quantization" notes, section 6: affine codes
+// q = clip(round(x/s) + z, qmin, qmax), x_hat = s(q - z), z the integer that
+// represents real 0; [AIInfra] "05Quantization01", LLM.int8() section: the
+// outliers are one-sided, which is where zeropoint beats absmax. Here the
+// non-outlier part of each token is quantised with a zero point: over its
+// non-outlier columns lo = min(0, min x), hi = max(0, max x), step =
+// fl32(fl32(hi - lo)/255), z = clamp(-128 - rint(fl32(lo/step)), -128, 127),
+// q = clamp(rint(fl32(x/step)) + z, -128, 127), and q = z at outlier columns.
+// The INT8 product then needs sum_k (q - z) Wq[n,k] = C - z * sum_k Wq[n,k], so
+// Y = fp16((C - z*rowsum[n]) * step * w_scale[n] / 127 + X_O.W_O^T).
+
+// rowsum[n] = sum_k Wq[n][k] (int32 [N]), once per weight (offline).
+int int8_weight_rowsum(const int8_t* Wq, int N, int K, int32_t* rowsum, i8mm_stream_t stream);
+
+// The decomposition with zero-point codes. Arguments, layout and errors as
+// int8_mixed_matmul plus w_rowsum (from int8_weight_rowsum, 16-byte aligned)
+// and the larger workspace below. In the workspace x_scale holds the step and
+// an int32 [M] array of zero points follows the regular layout (256-byte
+// aligned). Always runs the prefill kernels.
+size_t int8_mixed_matmul_zp_workspace_size(int M, int N, int K);
+int int8_mixed_matmul_zp(const void* X, const int8_t* Wq, const float* w_scale,
+                         const int32_t* w_rowsum, const void* W_fp16, int M, int N, int K,
+                         float threshold, void* Y, void* workspace, size_t workspace_bytes,
+                         i8mm_stream_t stream);
+
 // ---------------------------------------------------------------- top-k decomposition
 // [AIInfra] "05Quantization01", LLM.int8() section, training notes: raise the
 // decomposition ratio by computing the top 1% or 2% largest-magnitude feature

@@ -40,6 +40,8 @@ __all__ = [
     "int8_debug_gemm_i32",
     "int8_column_absmax",
     "int8_mixed_matmul_topk",
+    "int8_weight_rowsum",
+    "int8_mixed_matmul_zp",
     "int8_smoothquant_factors",
     "int8_smoothquant_weight_rows",
     "int8_smoothquant_workspace_size",
@@ -232,6 +234,46 @@ def int8_mixed_matmul_topk(X, Wq, w_scale, W_fp16, k, Y=None, workspace=None, st
                                         workspace.numel() * workspace.element_size(),
                                         _stream(stream)))
     return Y, workspace
+
+
+def int8_weight_rowsum(Wq, rowsum=None, stream=None):
+    """sum_k Wq[n, k] as int32 [N] (the zero-point correction's weight factor)."""
+    N, K = Wq.shape
+    _need(Wq, "Wq", torch.int8, (N, K))
+    rowsum = torch.empty((N,), dtype=torch.int32, device=Wq.device) if rowsum is None else rowsum
+    check("int8_weight_rowsum",
+          load().int8_weight_rowsum(_ptr(Wq), N, K, _ptr(rowsum), _stream(stream)))
+    return rowsum
+
+
+def int8_mixed_matmul_zp(X, Wq, w_scale, w_rowsum, W_fp16, threshold=6.0, Y=None,
+                         workspace=None, stream=None):
+    """The decomposition with zero-point codes for the non-outlier part.
+    Returns (Y fp16 [M, N], workspace); zero points via zeropoint_views()."""
+    M, K = X.shape
+    N = Wq.shape[0]
+    _need(X, "X", torch.float16, (M, K))
+    _need(Wq, "Wq", torch.int8, (N, K))
+    _need(w_scale, "w_scale", torch.float32, (N,))
+    _need(w_rowsum, "w_rowsum", torch.int32, (N,))
+    _need(W_fp16, "W_fp16", torch.float16, (N, K))
+    Y = torch.empty((M, N), dtype=torch.float16, device=X.device) if Y is None else Y
+    _need(Y, "Y", torch.float16, (M, N))
+    need = int(load().int8_mixed_matmul_zp_workspace_size(M, N, K))
+    if workspace is None:
+        workspace = torch.empty((max(need, 1),), dtype=torch.uint8, device=X.device)
+    check("int8_mixed_matmul_zp",
+          load().int8_mixed_matmul_zp(_ptr(X), _ptr(Wq), _ptr(w_scale), _ptr(w_rowsum),
+                                      _ptr(W_fp16), M, N, K, float(threshold), _ptr(Y),
+                                      _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                      _stream(stream)))
+    return Y, workspace
+
+
+def zeropoint_views(workspace: torch.Tensor, M: int, N: int, K: int) -> torch.Tensor:
+    """The int32 [M] zero points int8_mixed_matmul_zp leaves after the regular layout."""
+    off = (int8_mixed_matmul_workspace_size(M, N, K) + 255) // 256 * 256
+    return workspace[off:off + 4 * M].view(torch.int32)
 
 
 def int8_column_absmax(X, colmax=None, stream=None):

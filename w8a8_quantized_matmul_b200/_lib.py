@@ -40,6 +40,9 @@ PROTOTYPES = {
                                        _vp]),
     "int8_debug_gemm_i32": (_i, [_vp, _vp, _i, _i, _i, _vp, _vp]),
     "int8_column_absmax": (_i, [_vp, _i, _i, _vp, _vp]),
+    "int8_weight_rowsum": (_i, [_vp, _i, _i, _vp, _vp]),
+    "int8_mixed_matmul_zp_workspace_size": (_sz, [_i, _i, _i]),
+    "int8_mixed_matmul_zp": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _f, _vp, _vp, _sz, _vp]),
     "int8_mixed_matmul_topk_workspace_size": (_sz, [_i, _i, _i]),
     "int8_mixed_matmul_topk": (_i, [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _vp, _vp, _sz, _vp]),
     "int8_smoothquant_factors": (_i, [_vp, _vp, _i, _f, _vp, _vp, _vp]),

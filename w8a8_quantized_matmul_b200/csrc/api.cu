@@ -150,6 +150,15 @@ int int8_mixed_matmul_workspace_layout(int M, int N, int K, i8mm_workspace_layou
   return I8MM_OK;
 }
 
+int int8_weight_rowsum(const int8_t* Wq, int N, int K, int32_t* rowsum, i8mm_stream_t stream) {
+  const int st = check_sizes(1, N, K);
+  if (st != I8MM_OK) return st;
+  if (N == 0) return I8MM_OK;
+  if (!Wq || !rowsum) return I8MM_ERR_INVALID_ARG;
+  if (!aligned16(Wq) || !aligned16(rowsum)) return I8MM_ERR_ALIGNMENT;
+  return cuda_status(launch_weight_rowsum(Wq, N, K, rowsum, static_cast<cudaStream_t>(stream)));
+}
+
 int int8_quantize_weight_rows(const void* W, int N, int K, int8_t* Wq, float* w_scale,
                               i8mm_stream_t stream) {
   int st = check_sizes(1, N, K);
@@ -217,7 +226,8 @@ namespace {
 int mixed_matmul_impl(const void* X, const int8_t* Wq, const float* w_scale, const void* W_fp16,
                       int M, int N, int K, float threshold, void* Y, void* workspace,
                       size_t workspace_bytes, cudaStream_t stream, cudaEvent_t const* ev,
-                      int stages = 3, const uint32_t* given = nullptr, int given_n = 0) {
+                      int stages = 3, const uint32_t* given = nullptr, int given_n = 0,
+                      int32_t* x_zero = nullptr, const int32_t* w_rowsum = nullptr) {
   int st = check_sizes(M, N, K);
   if (st != I8MM_OK) return st;
   if ((st = check_threshold(threshold)) != I8MM_OK) return st;
@@ -247,7 +257,7 @@ int mixed_matmul_impl(const void* X, const int8_t* Wq, const float* w_scale, con
   const __half* Wh = static_cast<const __half*>(W_fp16);
 
   // Decode shapes: one clustered kernel for the whole call.
-  if (stages == 3 && !ev && !given && decode_supported(M, K)) {
+  if (stages == 3 && !ev && !given && !x_zero && decode_supported(M, K)) {
     DecodeArgs da{};
     da.X = Xh;
     da.W = Wh;
@@ -292,6 +302,7 @@ int mixed_matmul_impl(const void* X, const int8_t* Wq, const float* w_scale, con
     fa.status = status;
     fa.given = given;
     fa.given_n = given_n;
+    fa.x_zero = x_zero;
     e = launch_detect_quantize_compact(fa, stream);
     if (e != cudaSuccess) return cuda_fail("detect_quantize_compact_kernel launch", e);
   }
@@ -310,6 +321,8 @@ int mixed_matmul_impl(const void* X, const int8_t* Wq, const float* w_scale, con
   g.x_scale = xs;
   g.w_scale = w_scale;
   g.n_outliers = count;
+  g.x_zero = x_zero;
+  g.w_rowsum = w_rowsum;
   g.out = Y;
   g.M = M;
   g.N = N;
@@ -338,6 +351,34 @@ int int8_mixed_matmul_stage(int stage, const void* X, const int8_t* Wq, const fl
   if (stage != 1 && stage != 2) return I8MM_ERR_INVALID_ARG;
   return mixed_matmul_impl(X, Wq, w_scale, W_fp16, M, N, K, threshold, Y, workspace,
                            workspace_bytes, stream, nullptr, stage);
+}
+
+// Extra workspace of the zero-point path, after the regular layout: the
+// per-token zero points (int32 [M]), 256-byte aligned.
+size_t int8_mixed_matmul_zp_workspace_size(int M, int N, int K) {
+  Layout L;
+  if (!make_layout(M, N, K, &L)) return 0;
+  const size_t zoff = (L.l.total + 255) & ~static_cast<size_t>(255);
+  return (zoff + static_cast<size_t>(M) * 4 + 255) & ~static_cast<size_t>(255);
+}
+
+int int8_mixed_matmul_zp(const void* X, const int8_t* Wq, const float* w_scale,
+                         const int32_t* w_rowsum, const void* W_fp16, int M, int N, int K,
+                         float threshold, void* Y, void* workspace, size_t workspace_bytes,
+                         i8mm_stream_t stream) {
+  const int st = check_sizes(M, N, K);
+  if (st != I8MM_OK) return st;
+  if (M == 0 || N == 0) return I8MM_OK;
+  if (!w_rowsum || !workspace) return I8MM_ERR_INVALID_ARG;
+  if (!aligned16(w_rowsum)) return I8MM_ERR_ALIGNMENT;
+  Layout L;
+  make_layout(M, N, K, &L);
+  if (workspace_bytes < int8_mixed_matmul_zp_workspace_size(M, N, K)) return I8MM_ERR_WORKSPACE;
+  int32_t* x_zero = reinterpret_cast<int32_t*>(static_cast<uint8_t*>(workspace) +
+                                               ((L.l.total + 255) & ~static_cast<size_t>(255)));
+  return mixed_matmul_impl(X, Wq, w_scale, W_fp16, M, N, K, threshold, Y, workspace,
+                           workspace_bytes, static_cast<cudaStream_t>(stream), nullptr, 3, nullptr,
+                           0, x_zero, w_rowsum);
 }
 
 // Extra workspace of the top-k path, after the regular layout: column maxima

@@ -66,7 +66,8 @@ __device__ __forceinline__ uint64_t gtimer() {
 //   rows    [nb][K] fp16       the rows of the current wave, filled by bulk copies
 //   bits    [words] u32        outlier bitmap
 //   prefix  [words] i32        outliers before each bitmap word
-//   red     [kWarps+2][kMaxGroup] f32   per-warp row maxima; then row absmax, 1/absmax
+//   red     [2*kWarps+3][kMaxGroup] f32 per-warp row maxima (and, for zero-point codes,
+//                                      of -x); then row absmax or step, 1/absmax, zero point
 //   misc    [4] i32            running count during the scan
 //   idx     [K] u16            ascending outlier columns
 //   bar     u64                mbarrier of the bulk copies
@@ -83,7 +84,7 @@ __host__ __device__ inline FusedSmem fused_smem_layout(int K, int nb) {
   L.rows = off;   off = align16(off + static_cast<size_t>(nb) * K * 2);
   L.bits = off;   off = align16(off + words * 4);
   L.prefix = off; off = align16(off + words * 4);
-  L.red = off;    off = align16(off + static_cast<size_t>(kWarps + 2) * kMaxGroup * 4);
+  L.red = off;    off = align16(off + static_cast<size_t>(2 * kWarps + 3) * kMaxGroup * 4);
   L.misc = off;   off = align16(off + 16);
   L.idx = off;    off = align16(off + static_cast<size_t>(K) * 2);
   L.bar = off;    off = align16(off + 8);
@@ -91,7 +92,7 @@ __host__ __device__ inline FusedSmem fused_smem_layout(int K, int nb) {
   return L;
 }
 
-template <int VPT>
+template <int VPT, bool ZP>
 __global__ void __launch_bounds__(kThreads, VPT == 1 ? 2 : 1)
     detect_quantize_compact_kernel(FusedArgs a, int nb) {
   extern __shared__ __align__(128) uint8_t fsm[];
@@ -112,6 +113,9 @@ __global__ void __launch_bounds__(kThreads, VPT == 1 ? 2 : 1)
   float* s_red = reinterpret_cast<float*>(fsm + L.red);
   float* s_row = s_red + kWarps * kMaxGroup;
   float* s_rcp = s_row + kMaxGroup;
+  float* s_nred = s_rcp + kMaxGroup;                      // [kWarps][kMaxGroup] max of -x
+  int32_t* s_zero = reinterpret_cast<int32_t*>(s_nred + kWarps * kMaxGroup);
+  constexpr bool zp = ZP;   // zero-point codes
   int32_t* s_misc = reinterpret_cast<int32_t*>(fsm + L.misc);
   uint16_t* s_idx = reinterpret_cast<uint16_t*>(fsm + L.idx);
   uint64_t* s_bar = reinterpret_cast<uint64_t*>(fsm + L.bar);
@@ -234,31 +238,30 @@ __global__ void __launch_bounds__(kThreads, VPT == 1 ? 2 : 1)
     m8[c] = (v < nv) ? (bitmap_word(v >> 2) >> (8 * (v & 3))) & 0xFFu : 0u;
   }
   // Warp 0 also builds the per-word prefix counts and the ascending outlier
-  // list in shared memory (build_list); its first bitmap words are loaded now so
-  // that their L2 round trip overlaps the row maxima below.
+  // list in shared memory (build_list); its bitmap words are copied to shared
+  // memory now (cp.async: no registers held) so that their L2 round trip
+  // overlaps the row maxima below.
   const int lper = (words + 31) >> 5;                  // words per lane
   const int lw0 = min(words, lane * lper), lw1 = min(words, lw0 + lper);
-  uint32_t bw8[8];
-#pragma unroll
-  for (int i = 0; i < 8; ++i)
-    bw8[i] = (warp == 0 && lw0 + i < lw1) ? bitmap_word(lw0 + i) : 0u;
+  if (warp == 0 && !given) {
+    for (int w = lw0; w < lw1; ++w)
+      asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_addr(s_bits + w)),
+                   "l"(a.bitmap + w)
+                   : "memory");
+    asm volatile("cp.async.commit_group;" ::: "memory");
+  }
   bool listed = false;
   auto build_list = [&]() {
-    // Lane l scans the words [lw0, lw1): the first 8 are in bw8.
+    // Lane l scans the words [lw0, lw1).
     int cnt = 0;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      if (lw0 + i < lw1) s_bits[lw0 + i] = bw8[i];
-      cnt += __popc(bw8[i]);
-    }
-    for (int wb = lw0 + 8; wb < lw1; wb += 8) {
-      uint32_t b[8];
-#pragma unroll
-      for (int i = 0; i < 8; ++i) b[i] = (wb + i < lw1) ? bitmap_word(wb + i) : 0u;
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        if (wb + i < lw1) s_bits[wb + i] = b[i];
-        cnt += __popc(b[i]);
+    if (!given) {
+      asm volatile("cp.async.wait_all;" ::: "memory");
+      for (int w = lw0; w < lw1; ++w) cnt += __popc(s_bits[w]);
+    } else {
+      for (int w = lw0; w < lw1; ++w) {
+        const uint32_t b = bitmap_word(w);
+        s_bits[w] = b;
+        cnt += __popc(b);
       }
     }
     int incl = cnt;
@@ -333,29 +336,50 @@ __global__ void __launch_bounds__(kThreads, VPT == 1 ? 2 : 1)
     for (int gb = 0; gb < n; gb += kMaxGroup) {
       const int ng = min(kMaxGroup, n - gb);
       // Row absmax over the non-outlier columns: per thread, then per warp with
-      // one redux (non-negative floats order like their bit patterns).
+      // one redux (non-negative floats order like their bit patterns). Zero-point
+      // codes need the largest x and the largest -x instead (both >= 0 with the
+      // outlier columns zeroed, which keeps 0 inside the range).
 #pragma unroll 1
       for (int g = 0; g < ng; ++g) {
         const uint4* srow = reinterpret_cast<const uint4*>(s_rows + (gb + g) * row_bytes);
-        __half2 h = __float2half2_rn(0.0f);
+        __half2 h = __float2half2_rn(0.0f), hn = h;
 #pragma unroll
         for (int c = 0; c < VPT; ++c) {
           const int v = tid + kThreads * c;
           if (v < nv) {
             const uint4 u = srow[v];
             const uint32_t* wd = reinterpret_cast<const uint32_t*>(&u);
-            if (m8[c] == 0u) {
+            if constexpr (!zp) {
+              if (m8[c] == 0u) {
 #pragma unroll
-              for (int i = 0; i < 4; ++i) h = __hmax2(h, habs2_bits(wd[i]));
+                for (int i = 0; i < 4; ++i) h = __hmax2(h, habs2_bits(wd[i]));
+              } else {
+#pragma unroll
+                for (int i = 0; i < 4; ++i) h = __hmax2(h, habs2_bits(wd[i] & keep_half2(m8[c], i)));
+              }
             } else {
 #pragma unroll
-              for (int i = 0; i < 4; ++i) h = __hmax2(h, habs2_bits(wd[i] & keep_half2(m8[c], i)));
+              for (int i = 0; i < 4; ++i) {
+                const uint32_t kw = wd[i] & keep_half2(m8[c], i);
+                const uint32_t nw = kw ^ 0x80008000u;
+                h = __hmax2(h, *reinterpret_cast<const __half2*>(&kw));
+                hn = __hmax2(hn, *reinterpret_cast<const __half2*>(&nw));
+              }
             }
           }
         }
         const float2 hf = __half22float2(h);
-        const uint32_t m = __reduce_max_sync(0xffffffffu, __float_as_uint(fmaxf(hf.x, hf.y)));
-        if (lane == 0) s_red[warp * kMaxGroup + g] = __uint_as_float(m);
+        if constexpr (!zp) {
+          const uint32_t mx = __reduce_max_sync(0xffffffffu, __float_as_uint(fmaxf(hf.x, hf.y)));
+          if (lane == 0) s_red[warp * kMaxGroup + g] = __uint_as_float(mx);
+        } else {
+          // x and -x may be negative: clamp at 0 (0 stays inside the range)
+          const uint32_t mx = __reduce_max_sync(0xffffffffu, __float_as_uint(fmaxf(fmaxf(hf.x, hf.y), 0.0f)));
+          if (lane == 0) s_red[warp * kMaxGroup + g] = __uint_as_float(mx);
+          const float2 nf = __half22float2(hn);
+          const uint32_t mn = __reduce_max_sync(0xffffffffu, __float_as_uint(fmaxf(fmaxf(nf.x, nf.y), 0.0f)));
+          if (lane == 0) s_nred[warp * kMaxGroup + g] = __uint_as_float(mn);
+        }
       }
       if (warp == 0 && !listed) build_list();
       listed = true;
@@ -364,9 +388,23 @@ __global__ void __launch_bounds__(kThreads, VPT == 1 ? 2 : 1)
         float m = 0.0f;
 #pragma unroll
         for (int i = 0; i < kWarps; ++i) m = fmaxf(m, s_red[i * kMaxGroup + tid]);
-        s_row[tid] = m;
-        s_rcp[tid] = quant_rcp(m);
-        a.x_scale[wb + gb + tid] = m;
+        if constexpr (!zp) {
+          s_row[tid] = m;
+          s_rcp[tid] = quant_rcp(m);
+          a.x_scale[wb + gb + tid] = m;
+        } else {
+          // hi = m, lo = -nlo; step = fl(fl(hi - lo) / 255); z = -128 - rint(lo / step)
+          float nlo = 0.0f;
+#pragma unroll
+          for (int i = 0; i < kWarps; ++i) nlo = fmaxf(nlo, s_nred[i * kMaxGroup + tid]);
+          const float step = __fdiv_rn(__fadd_rn(m, nlo), 255.0f);
+          int z = 0;
+          if (step > 0.0f) z = max(-128, min(127, -128 - __float2int_rn(__fdiv_rn(-nlo, step))));
+          s_row[tid] = step;
+          s_zero[tid] = z;
+          a.x_scale[wb + gb + tid] = step;
+          a.x_zero[wb + gb + tid] = z;
+        }
       }
       __syncthreads();
       if (count < 0) setup_panels();
@@ -378,6 +416,31 @@ __global__ void __launch_bounds__(kThreads, VPT == 1 ? 2 : 1)
         const float ra = s_rcp[g];
         const uint4* srow = reinterpret_cast<const uint4*>(s_rows + (gb + g) * row_bytes);
         uint2* dst = reinterpret_cast<uint2*>(Xq + static_cast<size_t>(row) * K);
+        if constexpr (zp) {
+          // q = clamp(rint(x / step) + z, -128, 127); z at the outlier columns
+          const int z = s_zero[g];
+#pragma unroll
+          for (int c = 0; c < VPT; ++c) {
+            const int v = tid + kThreads * c;
+            if (v < nv) {
+              float f[8];
+              unpack8(srow[v], f);
+              uint32_t b[2] = {0u, 0u};
+#pragma unroll
+              for (int i = 0; i < 8; ++i) {
+                int qv = 0;
+                if ((m8[c] >> i) & 1u) {
+                  qv = z;
+                } else if (am > 0.0f) {
+                  qv = max(-128, min(127, __float2int_rn(__fdiv_rn(f[i], am)) + z));
+                }
+                b[i >> 2] |= (static_cast<uint32_t>(qv) & 0xFFu) << (8 * (i & 3));
+              }
+              dst[v] = make_uint2(b[0], b[1]);
+            }
+          }
+          continue;
+        }
 #pragma unroll
         for (int c = 0; c < VPT; ++c) {
           const int v = tid + kThreads * c;
@@ -455,12 +518,18 @@ int fused_vpt(int K) {
 cudaError_t launch_detect_quantize_compact(const FusedArgs& a, cudaStream_t s) {
   const int vpt = fused_vpt(a.K);
   const void* fn = nullptr;
+  const bool zp = a.x_zero != nullptr;
   switch (vpt) {
-    case 1: fn = reinterpret_cast<const void*>(detect_quantize_compact_kernel<1>); break;
-    case 2: fn = reinterpret_cast<const void*>(detect_quantize_compact_kernel<2>); break;
-    case 4: fn = reinterpret_cast<const void*>(detect_quantize_compact_kernel<4>); break;
-    case 8: fn = reinterpret_cast<const void*>(detect_quantize_compact_kernel<8>); break;
-    default: fn = reinterpret_cast<const void*>(detect_quantize_compact_kernel<16>); break;
+    case 1: fn = zp ? reinterpret_cast<const void*>(detect_quantize_compact_kernel<1, true>)
+                    : reinterpret_cast<const void*>(detect_quantize_compact_kernel<1, false>); break;
+    case 2: fn = zp ? reinterpret_cast<const void*>(detect_quantize_compact_kernel<2, true>)
+                    : reinterpret_cast<const void*>(detect_quantize_compact_kernel<2, false>); break;
+    case 4: fn = zp ? reinterpret_cast<const void*>(detect_quantize_compact_kernel<4, true>)
+                    : reinterpret_cast<const void*>(detect_quantize_compact_kernel<4, false>); break;
+    case 8: fn = zp ? reinterpret_cast<const void*>(detect_quantize_compact_kernel<8, true>)
+                    : reinterpret_cast<const void*>(detect_quantize_compact_kernel<8, false>); break;
+    default: fn = zp ? reinterpret_cast<const void*>(detect_quantize_compact_kernel<16, true>)
+                     : reinterpret_cast<const void*>(detect_quantize_compact_kernel<16, false>); break;
   }
   // Row buffer: ~96 KB when two CTAs share an SM (vpt 1), ~180 KB otherwise.
   const size_t row_bytes = static_cast<size_t>(a.K) * 2;

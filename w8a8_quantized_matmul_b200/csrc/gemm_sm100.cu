@@ -79,7 +79,8 @@ struct Cfg {
   static constexpr int STG_BYTES = kEpiWarps * 2 * STG_BUF_BYTES;
   static constexpr int WO_BYTES = kCcMax * BN * 2;   // W outlier tile, fp16, [j][column]
   static constexpr int SW_BYTES = BN * 4;            // w_scale tile
-  static constexpr int BAR_OFF = RING_BYTES + STG_BYTES + WO_BYTES + SW_BYTES;
+  static constexpr int ZS_BYTES = BN * 4;            // weight row sums (zero-point mode)
+  static constexpr int BAR_OFF = RING_BYTES + STG_BYTES + WO_BYTES + SW_BYTES + ZS_BYTES;
   static constexpr int BAR_BYTES = (2 * STAGES + 4) * 8 + 16;
   static constexpr int SMEM_BYTES = 1024 /*alignment slack*/ + BAR_OFF + BAR_BYTES;
 };
@@ -94,7 +95,9 @@ __device__ __forceinline__ void epi_sync() {
 
 // 18 warps: two of the four SM sub-partitions hold five warps, so the register
 // budget is 96 per thread (16K registers per sub-partition).
-template <bool OUT_I32, bool PAIR>
+// ZP: the activation codes carry a per-token zero point z (scholia section 6);
+// the epilogue forms (C - z * sum_k Wq[n, k]) * step * w_scale / 127.
+template <bool OUT_I32, bool PAIR, bool ZP>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_i8_persistent_kernel(const __grid_constant__ CUtensorMap tmA,
                               const __grid_constant__ CUtensorMap tmB,
@@ -103,6 +106,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                               const __grid_constant__ CUtensorMap tmY, int y_tma,
                               const float* __restrict__ x_scale,
                               const float* __restrict__ w_scale,
+                              const int32_t* __restrict__ x_zero,
+                              const int32_t* __restrict__ w_rowsum,
                               const int32_t* __restrict__ n_outliers,
                               const __half* __restrict__ X_O, const __half* __restrict__ W_O,
                               int ld, void* __restrict__ out, int M, int N, int K,
@@ -117,6 +122,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* stg = smem + C::RING_BYTES;                                          // staging
   __half* wo_s = reinterpret_cast<__half*>(stg + C::STG_BYTES);                // [kCcMax][BN]
   float* sw_s = reinterpret_cast<float*>(stg + C::STG_BYTES + C::WO_BYTES);     // [BN]
+  int32_t* zs_s = reinterpret_cast<int32_t*>(stg + C::STG_BYTES + C::WO_BYTES + C::SW_BYTES);
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::BAR_OFF);
   uint64_t* empty = full + STAGES;
   uint64_t* acc_full = empty + STAGES;   // [2]
@@ -292,6 +298,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int col_lo = part * (BN / 4);
 
     float sw_next = 0.0f;
+    int32_t ws_next = 0, zr_next = 0;
     uint4 wo_next[2] = {make_uint4(0, 0, 0, 0), make_uint4(0, 0, 0, 0)};
     uint4 xo_next[2] = {make_uint4(0, 0, 0, 0), make_uint4(0, 0, 0, 0)};
     float rs_next = 0.0f;
@@ -300,10 +307,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int m0 = (tile % m_tiles) * C::TILE_M + static_cast<int>(rank) * BM;
       const int n0 = (tile / m_tiles) * BN;
       const int row = m0 + q * 32 + lane;
-      rs_next = (row < M) ? x_scale[row] * (1.0f / 16129.0f) : 0.0f;
+      // absmax codes: x_absmax * w_absmax / 127^2; zero-point codes: step * w_absmax / 127
+      rs_next = (row < M) ? x_scale[row] * (ZP ? (1.0f / 127.0f) : (1.0f / 16129.0f)) : 0.0f;
+      if constexpr (ZP) zr_next = (row < M) ? x_zero[row] : 0;
       if (et < BN) {
         const int n = n0 + et;
         sw_next = (n < N) ? w_scale[n] : 0.0f;
+        if constexpr (ZP) ws_next = (n < N) ? w_rowsum[n] : 0;
         if (cc_out && n < N) {
           const uint4* src = reinterpret_cast<const uint4*>(W_O + static_cast<size_t>(n) * ld);
           wo_next[0] = src[0];
@@ -334,9 +344,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       // Stage this tile's column data in shared memory; keep the row data in registers.
       __half2 xo2[kCcMax / 2];
       const float rs = rs_next;
+      const int32_t zr = zr_next;
       if (!OUT_I32) {
         if (et < BN) {
           sw_s[et] = sw_next;
+          if constexpr (ZP) zs_s[et] = ws_next;
           if (cc_out) {
             const __half* h = reinterpret_cast<const __half*>(wo_next);
 #pragma unroll
@@ -394,6 +406,18 @@ __global__ void __launch_bounds__(kThreads, 1)
             } else {
               float y[16];
               const float4* sw4 = reinterpret_cast<const float4*>(sw_s + c);
+              if constexpr (ZP) {
+                // C - z * sum_k Wq[n, k], exact in int32 (|.| <= 2 * 128 * 127 * K)
+                const int4* zs4 = reinterpret_cast<const int4*>(zs_s + c);
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                  const int4 zw = zs4[j];
+                  acc[4 * j + 0] = static_cast<uint32_t>(static_cast<int32_t>(acc[4 * j + 0]) - zr * zw.x);
+                  acc[4 * j + 1] = static_cast<uint32_t>(static_cast<int32_t>(acc[4 * j + 1]) - zr * zw.y);
+                  acc[4 * j + 2] = static_cast<uint32_t>(static_cast<int32_t>(acc[4 * j + 2]) - zr * zw.z);
+                  acc[4 * j + 3] = static_cast<uint32_t>(static_cast<int32_t>(acc[4 * j + 3]) - zr * zw.w);
+                }
+              }
 #pragma unroll
               for (int j = 0; j < 4; ++j) {
                 const float4 w = sw4[j];
@@ -545,7 +569,7 @@ int sm_count(int dev) {
   return n;
 }
 
-template <bool OUT_I32, bool PAIR>
+template <bool OUT_I32, bool PAIR, bool ZP>
 cudaError_t launch(const GemmArgs& a, cudaStream_t s) {
   using C = Cfg<PAIR>;
   CUtensorMap maps[5];
@@ -568,7 +592,7 @@ cudaError_t launch(const GemmArgs& a, cudaStream_t s) {
                 CU_TENSOR_MAP_SWIZZLE_32B))
     y_tma = 1;
   if (!y_tma) maps[4] = maps[0];
-  auto kern = gemm_i8_persistent_kernel<OUT_I32, PAIR>;
+  auto kern = gemm_i8_persistent_kernel<OUT_I32, PAIR, ZP>;
   static bool attr_set[64] = {};  // per instantiation and device
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -604,7 +628,7 @@ cudaError_t launch(const GemmArgs& a, cudaStream_t s) {
   cfg.attrs = attr;
   cfg.numAttrs = na;
   e = cudaLaunchKernelEx(&cfg, kern, maps[0], maps[1], maps[2], maps[3], maps[4], y_tma,
-                         a.x_scale, a.w_scale,
+                         a.x_scale, a.w_scale, a.x_zero, a.w_rowsum,
                          OUT_I32 ? nullptr : a.n_outliers, a.X_O, a.W_O, a.ld, a.out, a.M, a.N,
                          a.K, a.status);
   if (e != cudaSuccess) (void)cudaGetLastError();   // do not leave it for the next launch
@@ -621,11 +645,13 @@ bool make_tmap_2d(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int 
 
 // CTA pairs whenever there is more than one 128-row block of output rows.
 cudaError_t launch_gemm_mixed(const GemmArgs& a, cudaStream_t s) {
-  return a.M > BM ? launch<false, true>(a, s) : launch<false, false>(a, s);
+  if (a.x_zero && a.w_rowsum)
+    return a.M > BM ? launch<false, true, true>(a, s) : launch<false, false, true>(a, s);
+  return a.M > BM ? launch<false, true, false>(a, s) : launch<false, false, false>(a, s);
 }
 
 cudaError_t launch_gemm_i32(const GemmArgs& a, cudaStream_t s) {
-  return a.M > BM ? launch<true, true>(a, s) : launch<true, false>(a, s);
+  return a.M > BM ? launch<true, true, false>(a, s) : launch<true, false, false>(a, s);
 }
 
 }  // namespace i8mm

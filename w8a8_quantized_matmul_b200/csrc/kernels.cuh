@@ -58,6 +58,9 @@ struct FusedArgs {
   // the grid barrier are skipped and the OR is written to bitmap.
   const uint32_t* given;
   int given_n;
+  // Zero-point codes (scholia section 6) instead of absmax codes when not null:
+  // x_scale gets the step (hi - lo)/255 and x_zero [M] the zero point.
+  int32_t* x_zero;
 };
 
 cudaError_t launch_detect_quantize_compact(const FusedArgs& a, cudaStream_t s);
@@ -76,6 +79,8 @@ struct GemmArgs {
   const float* x_scale;       // [M]
   const float* w_scale;       // [N]
   const int32_t* n_outliers;  // device count, or nullptr for no outlier pass
+  const int32_t* x_zero;      // [M] zero points (zero-point codes), or nullptr (absmax codes)
+  const int32_t* w_rowsum;    // [N] sum_k Wq[n, k] (with x_zero)
   void* out;                  // fp16 Y [M][N] or int32 C [M][N]
   int M, N, K;
   int32_t* status;            // device status word (may be nullptr)
@@ -117,6 +122,8 @@ bool decode_supported(int M, int K);
 
 // Running column max |x| of an fp16 [rows][K] matrix into fp32 colmax [K]
 // (smoothquant.cu) and the top-k column selection into a bitmap (topk.cu).
+cudaError_t launch_weight_rowsum(const int8_t* Wq, int N, int K, int32_t* rowsum,
+                                 cudaStream_t s);
 cudaError_t launch_column_absmax(const __half* X, int rows, int K, float* colmax, cudaStream_t s);
 cudaError_t launch_topk_select(const float* colmax, int K, int k, uint32_t* bitmap,
                                cudaStream_t s);

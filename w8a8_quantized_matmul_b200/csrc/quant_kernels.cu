@@ -235,4 +235,29 @@ cudaError_t launch_quantize_rows(int vpl, int grid, size_t smem, cudaStream_t s,
   return cudaGetLastError();
 }
 
+// sum_k Wq[n, k] per row (the zero-point correction's weight factor), one warp
+// per row, exact in int32 (|sum| <= 127 * 65536).
+__global__ void weight_rowsum_kernel(const int8_t* __restrict__ Wq, int N, int K,
+                                     int32_t* __restrict__ rowsum) {
+  const int n = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (n >= N) return;
+  const int8_t* w = Wq + static_cast<size_t>(n) * K;
+  int acc = 0;
+  for (int k = lane * 16; k < K; k += 32 * 16) {
+    const int4 v = *reinterpret_cast<const int4*>(w + k);
+    const int vv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) acc = __dp4a(vv[i], 0x01010101, acc);
+  }
+  acc = __reduce_add_sync(0xffffffffu, acc);
+  if (lane == 0) rowsum[n] = acc;
+}
+
+cudaError_t launch_weight_rowsum(const int8_t* Wq, int N, int K, int32_t* rowsum,
+                                 cudaStream_t s) {
+  weight_rowsum_kernel<<<(N + 7) / 8, 256, 0, s>>>(Wq, N, K, rowsum);
+  return cudaGetLastError();
+}
+
 }  // namespace i8mm
