@@ -28,3 +28,21 @@ from .smoothquant import (  # noqa: F401,E402
     smoothquant_matmul,
     per_tensor_quant_dequant,
 )
+from .rotation import (  # noqa: F401,E402
+    QMAX_W8,
+    QMAX_W4,
+    hadamard,
+    rotation_scale,
+    hadamard_sums,
+    rotate_groups,
+    rotate_groups_f64,
+    quantize_rows_rotated,
+    rotated_w8a8_matmul,
+    quantize_act_groups,
+    quantize_weight_blocks,
+    pack_int4,
+    unpack_int4,
+    group_gemm,
+    dequantize_groups,
+    rotated_w4a4_matmul,
+)

@@ -123,3 +123,42 @@ def test_zeropoint_pins_catch_planted_mistake(name, tmp_path):
                         "tests/test_zeropoint_pins.py"], cwd=tmp_path, capture_output=True,
                        text=True, timeout=300)
     assert r.returncode != 0, f"mutant {name} survived the pins:\n{r.stdout[-2000:]}"
+
+
+ROT_MUTANTS = {
+    "rot_normalised_by_g": ("return np.float32(1.0 / np.sqrt(float(G)))",
+                            "return np.float32(1.0 / float(G))"),
+    "rot_f64_normalised_by_g": ("return hadamard_sums(X, G) / np.sqrt(float(G))",
+                                "return hadamard_sums(X, G) / float(G)"),
+    "rot_sylvester_sign_moved": ("H = np.block([[H, H], [H, -H]])",
+                                 "H = np.block([[H, -H], [H, H]])"),
+    "rot_matrix_rows_reversed": ("S[:, g * G:(g + 1) * G] = Xf[:, g * G:(g + 1) * G] @ H",
+                                 "S[:, g * G:(g + 1) * G] = Xf[:, g * G:(g + 1) * G] @ H[::-1]"),
+    "rot_scaled_before_rounding": ("return S.astype(np.float32) * rotation_scale(G)",
+                                   "return (S * float(rotation_scale(G))).astype(np.float32)"),
+    "w4_block_absmax_first_row_only": ("a = np.abs(r).reshape(N // G, G, K // G, G).max(axis=(1, 3))",
+                                       "a = np.abs(r).reshape(N // G, G, K // G, G)[:, :1].max(axis=(1, 3))"),
+    "w4_pack_nibbles_reversed": ("return np.bitwise_or.reduce(nib << shifts, axis=2).astype(np.uint32)",
+                                 "return np.bitwise_or.reduce(nib << shifts[:, :, ::-1], axis=2).astype(np.uint32)"),
+    "w4_dequant_block_index_tiled": ("awn = np.repeat(np.asarray(aw, np.float64), G, axis=0)",
+                                     "awn = np.tile(np.asarray(aw, np.float64), (G, 1))"),
+    "w8_rot_dequant_over_127": ("/ float(QMAX_W8 * QMAX_W8))", "/ float(QMAX_W8))"),
+    "w4_act_absmax_over_whole_row": (
+        "a = np.abs(r).reshape(rows, K // G, G).max(axis=2) if K",
+        "a = np.abs(r).reshape(rows, K // G, G).max(axis=(1, 2))[:, None] * np.ones((1, K // G), np.float32) if K"),
+}
+
+
+@pytest.mark.parametrize("name", sorted(ROT_MUTANTS))
+def test_rotation_pins_catch_planted_mistake(name, tmp_path):
+    src = open(os.path.join(ROOT, "oracle", "rotation.py")).read()
+    old, new = ROT_MUTANTS[name]
+    assert old in src, f"mutation site for {name} no longer exists"
+    for d in ("oracle", "synth", "tests"):
+        shutil.copytree(os.path.join(ROOT, d), tmp_path / d,
+                        ignore=shutil.ignore_patterns("__pycache__", "test_oracle_mutants.py"))
+    (tmp_path / "oracle" / "rotation.py").write_text(src.replace(old, new, 1))
+    r = subprocess.run([sys.executable, "-m", "pytest", "-q", "-x", "-p", "no:cacheprovider",
+                        "tests/test_rotation_pins.py"], cwd=tmp_path, capture_output=True,
+                       text=True, timeout=300)
+    assert r.returncode != 0, f"mutant {name} survived the pins:\n{r.stdout[-2000:]}"
