@@ -256,9 +256,9 @@ CC_MAX_OUTLIERS = 16   # up to this many outlier columns no fp16 panels are writ
 # DRAM traffic per launch (dram__bytes_read.sum + dram__bytes_write.sum) from one
 # ncu capture of each kernel as it is now; the summaries and commands are in profiles/.
 NCU_TRAFFIC = {
-    "gemm": {"bytes": 78.000128e6 + 35.856896e6,
+    "gemm": {"bytes": 78.027008e6 + 34.86208e6,
              "source": "profiles/gemm_i8_persistent_opt-6.7b-ffn-up-prefill.md"},
-    "quantize": {"bytes": 27.357952e6 + 6.656e3,
+    "quantize": {"bytes": 27.326976e6 + 1.792e3,
                  "source": "profiles/detect_quantize_compact_opt-6.7b-ffn-up-prefill.md"},
     "decode": {"bytes": 19.596544e6,
                "source": "profiles/decode_kernel_decode-16x4096x4096.md"},
@@ -429,6 +429,8 @@ def run_ours(args, ws, rank, local):
         i8p = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]) * INT8_OVER_BF16
         result["topk"] = [bench_topk(args, stream, l2, i8p, f) for f in (0.01, 0.02)]
         result["zeropoint"] = bench_zeropoint(args, stream, l2, i8p)
+        hbm_peak = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
+        result["rotation"] = bench_rotation(args, stream, l2, i8p, hbm_peak)
     if rank == 0 and not args.no_cpu_baseline:
         import oracle
         Wq_o, ws_o = oracle.quantize_weight_rows(W)
@@ -631,6 +633,65 @@ def bench_zeropoint(args, stream, l2, int8_peak):
             "steps": steps, "rotating_sets": n_sets,
             "kernels": "detect_quantize_compact_kernel<., zero-point> + "
                        "gemm_i8_persistent_kernel<., ., zero-point>"}
+
+
+def bench_rotation(args, stream, l2, int8_peak, hbm, G=128):
+    """W8A8 after grouped Hadamard rotation on the default prefill shape: the weight
+    rotated and quantised once (offline), then the runtime call (rotation +
+    per-token quantisation kernel, INT8 GEMM) timed back to back over rotating
+    buffers; the rotation kernel is also timed alone (its HBM roofline)."""
+    import torch
+    import w8a8_quantized_matmul_b200 as m
+    w = synth.WORKLOADS[DEFAULT_WORKLOAD]
+    X, W, _ = synth.make_workload(w)
+    Xd = torch.from_numpy(X).cuda()
+    Wd = torch.from_numpy(W).cuda()
+    Wq, ws = m.int8_rotate_quantize_rows(Wd, G)
+    n_sets = n_sets_for(w, l2)
+    need = m.int8_rotated_workspace_size(w.M, w.N, w.K)
+    sets = [dict(X=Xd if i == 0 else Xd.clone(), Wq=Wq if i == 0 else Wq.clone(), ws=ws,
+                 Y=torch.empty((w.M, w.N), dtype=torch.float16, device="cuda"),
+                 work=torch.empty((need,), dtype=torch.uint8, device="cuda"),
+                 q=torch.empty((w.M, w.K), dtype=torch.int8, device="cuda"),
+                 a=torch.empty((w.M,), dtype=torch.float32, device="cuda"))
+            for i in range(n_sets)]
+
+    def step(i):
+        st = sets[i % n_sets]
+        m.int8_rotated_matmul(st["X"], st["Wq"], st["ws"], G, Y=st["Y"], workspace=st["work"])
+
+    def rot(i):
+        st = sets[i % n_sets]
+        m.int8_rotate_quantize_rows(st["X"], G, Xq=st["q"], absmax=st["a"])
+
+    def timed(fn, steps):
+        for i in range(max(3, args.warmup)):
+            fn(i)
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        a.record(stream)
+        for i in range(steps):
+            fn(i)
+        b.record(stream)
+        torch.cuda.synchronize()
+        return a.elapsed_time(b) / steps
+
+    steps = max(20, min(args.steps, 500))
+    ms = timed(step, steps)
+    r_ms = timed(rot, steps)
+    tops = 2.0 * w.M * w.N * w.K / (ms / 1e3) / 1e12
+    rbytes = 2 * w.M * w.K + w.M * w.K + 4 * w.M
+    r_gbs = rbytes / (r_ms / 1e3) / 1e9
+    del sets
+    return {"workload": w.name, "group": G, "ms_per_call": ms, "value": round(tops, 2),
+            "unit": "TOPS", "frac_of_int8_peak": round(tops / int8_peak, 4), "steps": steps,
+            "rotating_sets": n_sets,
+            "kernels": "rotate_rows_kernel + gemm_i8_persistent_kernel (no outlier pass)",
+            "rotate_kernel": {"ms": r_ms, "achieved": round(r_gbs, 1), "unit": "GB/s",
+                              "peak": hbm, "frac": round(r_gbs / hbm, 4),
+                              "algorithmic_bytes": rbytes,
+                              "bytes_note": "X fp16 read + codes written + scales"}}
 
 
 # --------------------------------------------------------------------------- reference arm

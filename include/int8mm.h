@@ -239,6 +239,73 @@ int int8_smoothquant_matmul(const void* X, const int8_t* Wq, const float* w_scal
                             const float* s_rcp, int M, int N, int K, void* Y, void* workspace,
                             size_t workspace_bytes, i8mm_stream_t stream);
 
+// ---------------------------------------------------------------- grouped Hadamard rotation
+// developer.baidu.com "分组旋转方法从W8A8到W4A4" (grouped rotation from W8A8 to
+// W4A4), sections 2, 5.1, 5.2, 5.4: before quantising, both operands are
+// multiplied along K by the block-diagonal orthogonal matrix with blocks
+// H_G/sqrt(G) (H_G the Sylvester Hadamard matrix, H[i][j] = (-1)^popcount(i&j)),
+// which leaves X W^T unchanged and spreads an outlier channel over its group.
+// G is 16, 32, 64, 128 or 256 and divides K; K <= 32768. The rotated value of an
+// fp16 row is r = fl32(fl32(S) * fl32(1/sqrt(G))), S the exact +-1 sum over the
+// group. Codes clamp(rint(fl32(fl32(r*qmax)/a)), +-qmax), a the group's absmax
+// (0 gives 0), qmax 127 (W8A8) or 7 (W4A4, the symmetric INT4 grid).
+
+// W8A8 side: rotate each row of X fp16 [rows][K], one absmax per row over all K:
+// Xq int8 [rows][K], absmax fp32 [rows]; R (optional, may be null) fp32
+// [rows][K] receives the rotated values. Serves the weight offline (rows = N)
+// and the activations. X, Xq, R 16-byte aligned.
+int int8_rotate_quantize_rows(const void* X, int rows, int K, int G, int8_t* Xq, float* absmax,
+                              float* R, i8mm_stream_t stream);
+
+// Bytes of workspace int8_rotated_matmul needs (0 for invalid sizes).
+size_t int8_rotated_workspace_size(int M, int N, int K);
+
+// Runtime W8A8 path after rotation: rotate and quantise X per token (Xq and
+// x_scale left in the workspace: status 16 B, x_scale fp32 [M], Xq int8 [M][K],
+// each 256-byte aligned), INT8 x INT8 -> INT32 on the tensor cores, Y =
+// fp16(C * x_scale * w_scale / 127^2). Wq int8 [N][K] and w_scale fp32 [N] come
+// from int8_rotate_quantize_rows on the weight with the same G. No outlier
+// split. Alignment, workspace and error rules as int8_mixed_matmul.
+int int8_rotated_matmul(const void* X, const int8_t* Wq, const float* w_scale, int M, int N, int K,
+                        int G, void* Y, void* workspace, size_t workspace_bytes,
+                        i8mm_stream_t stream);
+
+// W4A4 activation side: rotate, one absmax per (row, group of G columns):
+// absmax fp32 [rows][K/G]; Xq (optional) int8 [rows][K] holds the codes one
+// per byte (the form the INT8 tensor cores read), Xp (optional) uint32
+// [rows][K/8] holds them packed: code j of each run of eight along K in bits
+// 4j..4j+3 (two's complement nibble). At least one of Xq, Xp; X, Xq 16-byte
+// and Xp 8-byte aligned.
+int int4_rotate_quantize_groups(const void* X, int rows, int K, int G, int8_t* Xq, uint32_t* Xp,
+                                float* absmax, i8mm_stream_t stream);
+
+// W4A4 weight side (offline): rotate the rows of W fp16 [N][K], one absmax per
+// G x G sub-block (G output rows by G columns): absmax fp32 [N/G][K/G]; codes
+// packed as in int4_rotate_quantize_groups into Wp uint32 [N][K/8]. N % G == 0.
+int int4_rotate_quantize_weight_blocks(const void* W, int N, int K, int G, uint32_t* Wp,
+                                       float* absmax, i8mm_stream_t stream);
+
+// Packed 4-bit codes (as written by the two functions above) to one signed
+// byte each: P uint32 [rows][K/8] -> Q int8 [rows][K]. K % 32 == 0; P and Q
+// 16-byte aligned. The 4-bit product runs on the INT8 tensor cores (sm_100a
+// has no 4-bit integer MMA), so the weight is expanded once, at load time.
+int int4_unpack(const uint32_t* P, int rows, int K, int8_t* Q, i8mm_stream_t stream);
+
+// Bytes of workspace int4_rotated_matmul needs (0 for invalid sizes).
+size_t int4_rotated_workspace_size(int M, int N, int K, int G);
+
+// Runtime W4A4 path after rotation: rotate X and quantise it per (token, group)
+// (workspace: status 16 B, x_absmax fp32 [M][K/G], Xq int8 [M][K], each 256-byte
+// aligned), then Y = fp16(sum_g C_g * x_absmax[m][g] * w_absmax[n/G][g] / 7^2),
+// C_g the INT32 product over group g on the tensor cores. Wq4 int8 [N][K] holds
+// the weight's 4-bit codes one per byte (int4_unpack of the packed words of
+// int4_rotate_quantize_weight_blocks), w_absmax fp32 [N/G][K/G] its block
+// maxima. G in {64, 128, 256}; K % 128 == 0; N % G == 0. Alignment, workspace
+// and error rules as int8_mixed_matmul.
+int int4_rotated_matmul(const void* X, const int8_t* Wq4, const float* w_absmax, int M, int N,
+                        int K, int G, void* Y, void* workspace, size_t workspace_bytes,
+                        i8mm_stream_t stream);
+
 // Token-sharded (data-parallel over tokens) form of int8_mixed_matmul, one call
 // per rank on that rank's rows of X. AIInfra "05Quantization01", LLM.int8()
 // section: the outlier feature dimensions are those where any token of the

@@ -27,7 +27,7 @@ def lib():
 def declared_functions():
     src = open(HEADER).read()
     src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
-    names = re.findall(r"^\s*(?:const\s+)?[A-Za-z_][A-Za-z0-9_]*\s*\*?\s*(int8_[a-z0-9_]+)\s*\(", src, re.M)
+    names = re.findall(r"^\s*(?:const\s+)?[A-Za-z_][A-Za-z0-9_]*\s*\*?\s*(int[48]_[a-z0-9_]+)\s*\(", src, re.M)
     return sorted(set(names))
 
 
@@ -151,3 +151,29 @@ def test_workspace_size_rejects_bad_sizes(lib):
     assert lib.int8_mixed_matmul_workspace_size(-1, 4, 32) == 0
     lay = _lib.WorkspaceLayout()
     assert lib.int8_mixed_matmul_workspace_layout(4, 4, 20, ctypes.byref(lay)) == _lib.I8MM_ERR_ALIGNMENT
+
+
+def test_rotation_entry_points_validation(lib):
+    # G must be a power of two in [16, 256] dividing K; K <= 32768
+    assert lib.int8_rotate_quantize_rows(A, 4, 256, 24, A, A, None, None) == _lib.I8MM_ERR_INVALID_ARG
+    assert lib.int8_rotate_quantize_rows(A, 4, 256, 512, A, A, None, None) == _lib.I8MM_ERR_INVALID_ARG
+    assert lib.int8_rotate_quantize_rows(A, 4, 96, 64, A, A, None, None) == _lib.I8MM_ERR_INVALID_ARG
+    assert lib.int8_rotate_quantize_rows(A, 4, 65536, 128, A, A, None, None) == _lib.I8MM_ERR_INVALID_ARG
+    assert lib.int8_rotate_quantize_rows(None, 4, 256, 128, A, A, None, None) == _lib.I8MM_ERR_INVALID_ARG
+    assert lib.int8_rotate_quantize_rows(A, 4, 256, 128, MIS, A, None, None) == _lib.I8MM_ERR_ALIGNMENT
+    assert lib.int8_rotate_quantize_rows(A, 4, 256, 128, A, A, MIS, None) == _lib.I8MM_ERR_ALIGNMENT
+    assert lib.int8_rotate_quantize_rows(A, 0, 256, 128, None, None, None, None) == _lib.I8MM_OK
+    need = lib.int8_rotated_workspace_size(64, 64, 256)
+    assert need > 64 * 256
+    assert lib.int8_rotated_workspace_size(64, 64, 65536) == 0
+    assert lib.int8_rotated_matmul(A, A, A, 64, 64, 256, 128, A, A, need - 1, None) == _lib.I8MM_ERR_WORKSPACE
+    assert lib.int8_rotated_matmul(A, A, A, 64, 64, 256, 48, A, A, need, None) == _lib.I8MM_ERR_INVALID_ARG
+    assert lib.int8_rotated_matmul(A, A, A, 64, 64, 256, 128, MIS, A, need, None) == _lib.I8MM_ERR_ALIGNMENT
+    assert lib.int8_rotated_matmul(A, A, A, 64, 64, 256, 128, A, A + 16, need, None) == _lib.I8MM_ERR_ALIGNMENT
+    assert lib.int8_rotated_matmul(A, A, A, 0, 64, 256, 128, A, None, 0, None) == _lib.I8MM_OK
+    assert lib.int4_rotate_quantize_groups(A, 4, 256, 128, None, None, A, None) == _lib.I8MM_ERR_INVALID_ARG
+    assert lib.int4_rotate_quantize_groups(A, 4, 256, 128, A, A + 4, A, None) == _lib.I8MM_ERR_ALIGNMENT
+    assert lib.int4_rotate_quantize_groups(A, 4, 256, 8, A, A, A, None) == _lib.I8MM_ERR_INVALID_ARG
+    assert lib.int4_rotate_quantize_weight_blocks(A, 96, 256, 64, A, A, None) == _lib.I8MM_ERR_INVALID_ARG
+    assert lib.int4_rotate_quantize_weight_blocks(A, 128, 256, 64, None, A, None) == _lib.I8MM_ERR_INVALID_ARG
+    assert lib.int4_rotate_quantize_weight_blocks(A, 0, 256, 64, None, None, None) == _lib.I8MM_OK

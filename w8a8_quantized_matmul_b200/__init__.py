@@ -386,3 +386,141 @@ def workspace_views(workspace: torch.Tensor, M: int, N: int, K: int) -> dict:
         X_O=view(lay.X_O, 2 * M * ld, torch.float16, (M, ld)),
         W_O=view(lay.W_O, 2 * N * ld, torch.float16, (N, ld)),
     )
+
+
+# --------------------------------------------------------------- grouped Hadamard rotation
+def int8_rotate_quantize_rows(X, G=128, Xq=None, absmax=None, R=None, stream=None):
+    """Rotate each row of X fp16 [rows, K] in groups of G, per-row absmax INT8 codes.
+    Returns (Xq int8 [rows, K], absmax fp32 [rows]); R (fp32 [rows, K]) if given
+    receives the rotated values."""
+    rows, K = X.shape
+    _need(X, "X", torch.float16, (rows, K))
+    Xq = torch.empty((rows, K), dtype=torch.int8, device=X.device) if Xq is None else Xq
+    absmax = torch.empty((rows,), dtype=torch.float32, device=X.device) if absmax is None else absmax
+    _need(Xq, "Xq", torch.int8, (rows, K))
+    _need(absmax, "absmax", torch.float32, (rows,))
+    if R is not None:
+        _need(R, "R", torch.float32, (rows, K))
+    check("int8_rotate_quantize_rows",
+          load().int8_rotate_quantize_rows(_ptr(X), rows, K, int(G), _ptr(Xq), _ptr(absmax),
+                                           _ptr(R) if R is not None else None, _stream(stream)))
+    return Xq, absmax
+
+
+def int8_rotated_workspace_size(M: int, N: int, K: int) -> int:
+    return int(load().int8_rotated_workspace_size(M, N, K))
+
+
+def int8_rotated_matmul(X, Wq, w_scale, G=128, Y=None, workspace=None, stream=None):
+    """W8A8 after grouped Hadamard rotation; returns (Y fp16 [M, N], workspace)."""
+    M, K = X.shape
+    N = Wq.shape[0]
+    _need(X, "X", torch.float16, (M, K))
+    _need(Wq, "Wq", torch.int8, (N, K))
+    _need(w_scale, "w_scale", torch.float32, (N,))
+    Y = torch.empty((M, N), dtype=torch.float16, device=X.device) if Y is None else Y
+    _need(Y, "Y", torch.float16, (M, N))
+    need = int8_rotated_workspace_size(M, N, K)
+    if workspace is None:
+        workspace = torch.empty((max(need, 1),), dtype=torch.uint8, device=X.device)
+    check("int8_rotated_matmul",
+          load().int8_rotated_matmul(_ptr(X), _ptr(Wq), _ptr(w_scale), M, N, K, int(G), _ptr(Y),
+                                     _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                     _stream(stream)))
+    return Y, workspace
+
+
+def rotated_workspace_views(workspace: torch.Tensor, M: int, K: int) -> dict:
+    """status / x_scale / Xq views of an int8_rotated_matmul workspace."""
+    def up(x):
+        return (x + 255) // 256 * 256
+    xs = up(16)
+    xq = up(xs + 4 * M)
+    return {"status": workspace[0:4].view(torch.int32),
+            "x_scale": workspace[xs:xs + 4 * M].view(torch.float32),
+            "Xq": workspace[xq:xq + M * K].view(torch.int8).view(M, K)}
+
+
+def int4_rotate_quantize_groups(X, G=128, Xq=True, Xp=True, absmax=None, stream=None):
+    """Rotate, per-(row, group) absmax, 4-bit codes. Xq / Xp: True to allocate,
+    None to skip, or a tensor (int8 [rows, K] / int32 [rows, K/8] holding the
+    packed uint32 words). Returns (Xq or None, Xp or None, absmax fp32 [rows, K/G])."""
+    rows, K = X.shape
+    _need(X, "X", torch.float16, (rows, K))
+    if Xq is True:
+        Xq = torch.empty((rows, K), dtype=torch.int8, device=X.device)
+    if Xp is True:
+        Xp = torch.empty((rows, K // 8), dtype=torch.int32, device=X.device)
+    if absmax is None:
+        absmax = torch.empty((rows, K // max(int(G), 1)), dtype=torch.float32, device=X.device)
+    if Xq is not None:
+        _need(Xq, "Xq", torch.int8, (rows, K))
+    if Xp is not None:
+        _need(Xp, "Xp", torch.int32, (rows, K // 8))
+    check("int4_rotate_quantize_groups",
+          load().int4_rotate_quantize_groups(_ptr(X), rows, K, int(G),
+                                             _ptr(Xq) if Xq is not None else None,
+                                             _ptr(Xp) if Xp is not None else None,
+                                             _ptr(absmax), _stream(stream)))
+    return Xq, Xp, absmax
+
+
+def int4_rotate_quantize_weight_blocks(W, G=128, Wp=None, absmax=None, stream=None):
+    """Offline W4 weight: rotate rows, per G x G block absmax, packed codes.
+    Returns (Wp int32 [N, K/8] holding uint32 words, absmax fp32 [N/G, K/G])."""
+    N, K = W.shape
+    _need(W, "W", torch.float16, (N, K))
+    Wp = torch.empty((N, K // 8), dtype=torch.int32, device=W.device) if Wp is None else Wp
+    if absmax is None:
+        absmax = torch.empty((max(N // int(G), 0), K // int(G)), dtype=torch.float32,
+                             device=W.device)
+    _need(Wp, "Wp", torch.int32, (N, K // 8))
+    check("int4_rotate_quantize_weight_blocks",
+          load().int4_rotate_quantize_weight_blocks(_ptr(W), N, K, int(G), _ptr(Wp), _ptr(absmax),
+                                                    _stream(stream)))
+    return Wp, absmax
+
+
+def int4_unpack(P, K, Q=None, stream=None):
+    """Packed 4-bit codes int32 [rows, K/8] (uint32 words) -> int8 [rows, K]."""
+    rows = P.shape[0]
+    _need(P, "P", torch.int32, (rows, K // 8))
+    Q = torch.empty((rows, K), dtype=torch.int8, device=P.device) if Q is None else Q
+    _need(Q, "Q", torch.int8, (rows, K))
+    check("int4_unpack", load().int4_unpack(_ptr(P), rows, K, _ptr(Q), _stream(stream)))
+    return Q
+
+
+def int4_rotated_workspace_size(M: int, N: int, K: int, G: int) -> int:
+    return int(load().int4_rotated_workspace_size(M, N, K, G))
+
+
+def int4_rotated_matmul(X, Wq4, w_absmax, G=128, Y=None, workspace=None, stream=None):
+    """W4A4 after grouped Hadamard rotation; Wq4 int8 [N, K] holds the weight's
+    4-bit codes one per byte, w_absmax fp32 [N/G, K/G]. Returns (Y, workspace)."""
+    M, K = X.shape
+    N = Wq4.shape[0]
+    _need(X, "X", torch.float16, (M, K))
+    _need(Wq4, "Wq4", torch.int8, (N, K))
+    _need(w_absmax, "w_absmax", torch.float32, (N // int(G), K // int(G)))
+    Y = torch.empty((M, N), dtype=torch.float16, device=X.device) if Y is None else Y
+    _need(Y, "Y", torch.float16, (M, N))
+    need = int4_rotated_workspace_size(M, N, K, G)
+    if workspace is None:
+        workspace = torch.empty((max(need, 1),), dtype=torch.uint8, device=X.device)
+    check("int4_rotated_matmul",
+          load().int4_rotated_matmul(_ptr(X), _ptr(Wq4), _ptr(w_absmax), M, N, K, int(G), _ptr(Y),
+                                     _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                     _stream(stream)))
+    return Y, workspace
+
+
+def int4_rotated_workspace_views(workspace: torch.Tensor, M: int, K: int, G: int) -> dict:
+    """status / x_absmax / Xq views of an int4_rotated_matmul workspace."""
+    def up(x):
+        return (x + 255) // 256 * 256
+    xa = up(16)
+    xq = up(xa + 4 * M * (K // G))
+    return {"status": workspace[0:4].view(torch.int32),
+            "x_absmax": workspace[xa:xa + 4 * M * (K // G)].view(torch.float32).view(M, K // G),
+            "Xq": workspace[xq:xq + M * K].view(torch.int8).view(M, K)}

@@ -49,6 +49,14 @@ PROTOTYPES = {
     "int8_smoothquant_weight_rows": (_i, [_vp, _vp, _i, _i, _vp, _vp, _vp]),
     "int8_smoothquant_workspace_size": (_sz, [_i, _i, _i]),
     "int8_smoothquant_matmul": (_i, [_vp, _vp, _vp, _vp, _i, _i, _i, _vp, _vp, _sz, _vp]),
+    "int8_rotate_quantize_rows": (_i, [_vp, _i, _i, _i, _vp, _vp, _vp, _vp]),
+    "int8_rotated_workspace_size": (_sz, [_i, _i, _i]),
+    "int8_rotated_matmul": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _vp, _vp, _sz, _vp]),
+    "int4_rotate_quantize_groups": (_i, [_vp, _i, _i, _i, _vp, _vp, _vp, _vp]),
+    "int4_rotate_quantize_weight_blocks": (_i, [_vp, _i, _i, _i, _vp, _vp, _vp]),
+    "int4_unpack": (_i, [_vp, _i, _i, _vp, _vp]),
+    "int4_rotated_workspace_size": (_sz, [_i, _i, _i, _i]),
+    "int4_rotated_matmul": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _vp, _vp, _sz, _vp]),
     "int8_device_status": (_i, [_vp, _vp]),
     "int8_status_string": (ctypes.c_char_p, [_i]),
     "int8_last_error_string": (ctypes.c_char_p, []),

@@ -89,6 +89,13 @@ struct GemmArgs {
 cudaError_t launch_gemm_mixed(const GemmArgs& a, cudaStream_t s);
 cudaError_t launch_gemm_i32(const GemmArgs& a, cudaStream_t s);
 
+// Group-scaled GEMM of the W4A4 path (gemm_groups.cu): Y = fp16(sum_g C_g *
+// x_absmax[m][g] * w_absmax[n/G][g] / 49) over groups of G columns of K.
+// G in {64, 128, 256}; K % 128 == 0, K % G == 0, N % G == 0.
+cudaError_t launch_gemm_groups(const int8_t* Xq, const int8_t* Wq, const float* x_absmax,
+                               const float* w_absmax, __half* Y, int M, int N, int K, int G,
+                               int32_t* status, cudaStream_t s);
+
 // Row-major [rows][cols] tensor map with a box of box_rows x box_bytes (one
 // swizzle span wide); defined in gemm_sm100.cu.
 bool make_tmap_2d(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int elem_bytes,
