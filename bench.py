@@ -431,6 +431,7 @@ def run_ours(args, ws, rank, local):
         result["zeropoint"] = bench_zeropoint(args, stream, l2, i8p)
         hbm_peak = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
         result["rotation"] = bench_rotation(args, stream, l2, i8p, hbm_peak)
+        result["rotation_w4a4"] = bench_w4a4(args, stream, l2, i8p)
     if rank == 0 and not args.no_cpu_baseline:
         import oracle
         Wq_o, ws_o = oracle.quantize_weight_rows(W)
@@ -692,6 +693,53 @@ def bench_rotation(args, stream, l2, int8_peak, hbm, G=128):
                               "peak": hbm, "frac": round(r_gbs / hbm, 4),
                               "algorithmic_bytes": rbytes,
                               "bytes_note": "X fp16 read + codes written + scales"}}
+
+
+def bench_w4a4(args, stream, l2, int8_peak, G=128):
+    """W4A4 after grouped Hadamard rotation on the default prefill shape: the weight
+    rotated, block-quantised, packed and expanded to one code per byte once
+    (offline), then the runtime call (rotation + per-(token, group) 4-bit codes,
+    group-scaled tensor-core GEMM) timed back to back over rotating buffers."""
+    import torch
+    import w8a8_quantized_matmul_b200 as m
+    w = synth.WORKLOADS[DEFAULT_WORKLOAD]
+    X, W, _ = synth.make_workload(w)
+    Xd = torch.from_numpy(X).cuda()
+    Wd = torch.from_numpy(W).cuda()
+    Wp, aw = m.int4_rotate_quantize_weight_blocks(Wd, G)
+    Wq4 = m.int4_unpack(Wp, w.K)
+    del Wd
+    n_sets = n_sets_for(w, l2)
+    need = m.int4_rotated_workspace_size(w.M, w.N, w.K, G)
+    sets = [dict(X=Xd if i == 0 else Xd.clone(), Wq=Wq4 if i == 0 else Wq4.clone(),
+                 Y=torch.empty((w.M, w.N), dtype=torch.float16, device="cuda"),
+                 work=torch.empty((need,), dtype=torch.uint8, device="cuda"))
+            for i in range(n_sets)]
+
+    def step(i):
+        st = sets[i % n_sets]
+        m.int4_rotated_matmul(st["X"], st["Wq"], aw, G, Y=st["Y"], workspace=st["work"])
+
+    for i in range(max(3, args.warmup)):
+        step(i)
+    steps = max(20, min(args.steps, 500))
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    a.record(stream)
+    for i in range(steps):
+        step(i)
+    b.record(stream)
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b) / steps
+    tops = 2.0 * w.M * w.N * w.K / (ms / 1e3) / 1e12
+    del sets
+    return {"workload": w.name, "group": G, "ms_per_call": ms, "value": round(tops, 2),
+            "unit": "TOPS", "frac_of_int8_peak": round(tops / int8_peak, 4), "steps": steps,
+            "rotating_sets": n_sets,
+            "kernels": "rotate_groups_kernel + gemm_groups_kernel (4-bit codes on the INT8 "
+                       "tensor cores, per-group promotion)",
+            "weight_bytes_packed": w.N * w.K // 2}
 
 
 # --------------------------------------------------------------------------- reference arm

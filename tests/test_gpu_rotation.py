@@ -174,3 +174,37 @@ def test_int4_rotated_matmul_parity(case):
     np.testing.assert_array_equal(v["x_absmax"].cpu().numpy(), ref["x_scale"])
     np.testing.assert_array_equal(v["Xq"].cpu().numpy(), ref["Xq"])
     _y_close(Y.cpu().numpy(), ref["Y"])
+
+
+def test_exact_half_integer_quotients_round_to_even():
+    """Groups of G = 64 with two spikes v1 = 255 + 2k, v2 = 253 - 2k rotate to
+    (v1 + v2)/8 = 63.5 (the row absmax) and (v1 - v2)/8, so the odd columns'
+    quotient r * 127 / a is exactly k + 1/2: the code path's near-tie fallback
+    must give the ties-to-even integer. Same for the 4-bit grid with
+    v1 = 15 + 2k, v2 = 13 - 2k (quotient k + 1/2 of r * 7 / a)."""
+    G = 64
+    ks = np.arange(0, 127)
+    X = np.zeros((1, G * len(ks)), np.float16)
+    for i, k in enumerate(ks):
+        X[0, G * i] = 255 + 2 * k
+        X[0, G * i + 1] = 253 - 2 * k
+    q_ref, a_ref, _ = oracle.quantize_rows_rotated(X, G)
+    assert a_ref[0] == 63.5
+    Xq, a = m.int8_rotate_quantize_rows(torch.from_numpy(X).cuda(), G)
+    q = Xq.cpu().numpy()
+    np.testing.assert_array_equal(q, q_ref)
+    even = np.where(ks % 2 == 0, ks, ks + 1)            # rint(k + 1/2), ties to even
+    np.testing.assert_array_equal(q[0, G * np.arange(len(ks)) + 1], even)
+
+    ks4 = np.arange(0, 7)
+    X4 = np.zeros((1, G * len(ks4)), np.float16)
+    for i, k in enumerate(ks4):
+        X4[0, G * i] = 15 + 2 * k
+        X4[0, G * i + 1] = 13 - 2 * k
+    q4_ref, a4_ref, _ = oracle.quantize_act_groups(X4, G)
+    Xq4, _, a4 = m.int4_rotate_quantize_groups(torch.from_numpy(X4).cuda(), G, Xp=None)
+    q4 = Xq4.cpu().numpy()
+    np.testing.assert_array_equal(q4, q4_ref)
+    np.testing.assert_array_equal(a4.cpu().numpy(), a4_ref)
+    even4 = np.where(ks4 % 2 == 0, ks4, ks4 + 1)
+    np.testing.assert_array_equal(q4[0, G * np.arange(len(ks4)) + 1], even4)

@@ -37,6 +37,7 @@
 #include "int8mm.h"
 #include "kernels.cuh"
 #include "ptx.cuh"
+#include "quant_common.cuh"
 
 namespace i8mm {
 
@@ -87,15 +88,55 @@ __device__ __forceinline__ void rotate16(const __half* __restrict__ src, bool li
   const int lane = threadIdx.x & 31;
 #pragma unroll
   for (int s = 1; s < G / 16; s <<= 1) {
-    const bool upper = (lane & s) != 0;
+    // lower lane: v + p; upper lane: p - v; one exact FMA by +-1 either way
+    const double sg = (lane & s) ? -1.0 : 1.0;
 #pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      const double p = __shfl_xor_sync(0xffffffffu, v[i], s);
-      v[i] = upper ? p - v[i] : v[i] + p;
-    }
+    for (int i = 0; i < 16; ++i) v[i] = __fma_rn(sg, v[i], __shfl_xor_sync(0xffffffffu, v[i], s));
   }
 #pragma unroll
   for (int i = 0; i < 16; ++i) r[i] = __fmul_rn(__double2float_rn(v[i]), c);
+}
+
+// Codes of 16 rotated values against the absmax a of their group, ra =
+// quant_rcp(a): q = rint(fl32(n / a)) with n = fl32(r * qmax). The quotient is
+// formed without a division: q0 = fl(n * ra), e = fma(q0, -a, n) (exact),
+// qc = fma(e, ra, q0), within about one ulp of n / a. Where qc lies within
+// 2^-15 (four ulps at |q| < 128) of a half-integer the correctly rounded
+// quotient could round the other way, so those codes are recomputed with a
+// correctly rounded division; everywhere else rint(qc) is the code. rint is
+// the low bits of fl(qc + 1.5 * 2^23) (ties to even).
+__device__ __forceinline__ void rot_codes16(const float (&r)[16], float a, float ra, float qmax,
+                                            int (&q)[16]) {
+  const uint64_t na2 = f2pack(-a, -a), ra2 = f2pack(ra, ra), qm2 = f2pack(qmax, qmax);
+  const uint64_t mg2 = f2pack(kMagic, kMagic);
+  bool tie = false;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    const uint64_t n = mul2(f2pack(r[2 * j], r[2 * j + 1]), qm2);
+    const uint64_t q0 = mul2(n, ra2);
+    const uint64_t qc = fma2(fma2(q0, na2, n), ra2, q0);
+    const uint64_t sm = add2(qc, mg2);
+    const uint64_t t = sub2(qc, sub2(sm, mg2));            // qc - rint(qc), exact
+    q[2 * j] = __float_as_int(lo(sm)) - 0x4B400000;
+    q[2 * j + 1] = __float_as_int(hi(sm)) - 0x4B400000;
+    tie |= fabsf(fabsf(lo(t)) - 0.5f) < 0x1p-15f;
+    tie |= fabsf(fabsf(hi(t)) - 0.5f) < 0x1p-15f;
+  }
+  if (tie) {
+#pragma unroll
+    for (int i = 0; i < 16; ++i) q[i] = rot_code(r[i], a, qmax);
+  }
+}
+
+__device__ __forceinline__ void store_codes16(const int (&q)[16], int8_t* dst) {
+  uint32_t b[4];
+#pragma unroll
+  for (int j = 0; j < 4; ++j)
+    b[j] = (static_cast<uint32_t>(q[4 * j]) & 0xFFu) |
+           ((static_cast<uint32_t>(q[4 * j + 1]) & 0xFFu) << 8) |
+           ((static_cast<uint32_t>(q[4 * j + 2]) & 0xFFu) << 16) |
+           ((static_cast<uint32_t>(q[4 * j + 3]) & 0xFFu) << 24);
+  *reinterpret_cast<uint4*>(dst) = make_uint4(b[0], b[1], b[2], b[3]);
 }
 
 __device__ __forceinline__ float max16(const float (&r)[16]) {
@@ -105,8 +146,10 @@ __device__ __forceinline__ float max16(const float (&r)[16]) {
   return m;
 }
 
-// One CTA per row; pieces p = it * blockDim.x + tid. Rotated values go to
-// shared memory, the row max to `red`, then the codes.
+// One CTA per row; pieces p = it * blockDim.x + tid. A row of at most
+// blockDim.x pieces keeps its rotated values in registers; a longer row stages
+// them in shared memory. Then the row max (warp redux, then across warps) and
+// the codes.
 template <int G>
 __global__ void __launch_bounds__(kRowThreads) rotate_rows_kernel(
     const __half* __restrict__ X, int K, float c, int8_t* __restrict__ Xq,
@@ -117,17 +160,20 @@ __global__ void __launch_bounds__(kRowThreads) rotate_rows_kernel(
   const size_t row = blockIdx.x;
   const int np = K >> 4;
   const int nt = blockDim.x;
+  const bool single = np <= nt;
+  float r[16];
   float m = 0.0f;
   for (int base = 0; base < np; base += nt) {
     const int p = base + threadIdx.x;
-    float r[16];
     rotate16<G>(X + row * K + 16 * p, p < np, c, r);
     if (p < np) {
       m = fmaxf(m, max16(r));
+      if (!single) {
 #pragma unroll
-      for (int i = 0; i < 4; ++i)
-        reinterpret_cast<float4*>(rs + 16 * p)[i] = make_float4(r[4 * i], r[4 * i + 1],
-                                                               r[4 * i + 2], r[4 * i + 3]);
+        for (int i = 0; i < 4; ++i)
+          reinterpret_cast<float4*>(rs + 16 * p)[i] = make_float4(r[4 * i], r[4 * i + 1],
+                                                                 r[4 * i + 2], r[4 * i + 3]);
+      }
     }
   }
   const uint32_t w = __reduce_max_sync(0xffffffffu, __float_as_uint(m));
@@ -135,21 +181,18 @@ __global__ void __launch_bounds__(kRowThreads) rotate_rows_kernel(
   __syncthreads();
   float a = 0.0f;
   for (int i = 0; i < (nt >> 5); ++i) a = fmaxf(a, red[i]);
+  const float ra = a == 0.0f ? 0.0f : __frcp_rn(a);
   for (int p = threadIdx.x; p < np; p += nt) {
-    float r[16];
+    if (!single) {
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const float4 f = reinterpret_cast<const float4*>(rs + 16 * p)[i];
-      r[4 * i] = f.x; r[4 * i + 1] = f.y; r[4 * i + 2] = f.z; r[4 * i + 3] = f.w;
+      for (int i = 0; i < 4; ++i) {
+        const float4 f = reinterpret_cast<const float4*>(rs + 16 * p)[i];
+        r[4 * i] = f.x; r[4 * i + 1] = f.y; r[4 * i + 2] = f.z; r[4 * i + 3] = f.w;
+      }
     }
-    uint32_t b[4];
-#pragma unroll
-    for (int j = 0; j < 4; ++j)
-      b[j] = (static_cast<uint32_t>(rot_code(r[4 * j], a, 127.0f)) & 0xFFu) |
-             ((static_cast<uint32_t>(rot_code(r[4 * j + 1], a, 127.0f)) & 0xFFu) << 8) |
-             ((static_cast<uint32_t>(rot_code(r[4 * j + 2], a, 127.0f)) & 0xFFu) << 16) |
-             ((static_cast<uint32_t>(rot_code(r[4 * j + 3], a, 127.0f)) & 0xFFu) << 24);
-    *reinterpret_cast<uint4*>(Xq + row * K + 16 * p) = make_uint4(b[0], b[1], b[2], b[3]);
+    int q[16];
+    rot_codes16(r, a, ra, 127.0f, q);
+    store_codes16(q, Xq + row * K + 16 * p);
     if (R) {
 #pragma unroll
       for (int i = 0; i < 4; ++i)
@@ -193,18 +236,8 @@ __global__ void __launch_bounds__(256) rotate_groups_kernel(
     a = __ldg(scale + (row / G) * ng + g);
   }
   int q[16];
-#pragma unroll
-  for (int i = 0; i < 16; ++i) q[i] = rot_code(r[i], a, 7.0f);
-  if (Xq) {
-    uint32_t b[4];
-#pragma unroll
-    for (int j = 0; j < 4; ++j)
-      b[j] = (static_cast<uint32_t>(q[4 * j]) & 0xFFu) |
-             ((static_cast<uint32_t>(q[4 * j + 1]) & 0xFFu) << 8) |
-             ((static_cast<uint32_t>(q[4 * j + 2]) & 0xFFu) << 16) |
-             ((static_cast<uint32_t>(q[4 * j + 3]) & 0xFFu) << 24);
-    *reinterpret_cast<uint4*>(Xq + row * K + 16 * p) = make_uint4(b[0], b[1], b[2], b[3]);
-  }
+  rot_codes16(r, a, a == 0.0f ? 0.0f : __frcp_rn(a), 7.0f, q);
+  if (Xq) store_codes16(q, Xq + row * K + 16 * p);
   if (Xp) {
     uint32_t w0 = 0u, w1 = 0u;
 #pragma unroll
