@@ -19,13 +19,19 @@
 // (both as paired f32x2 operations). The epilogue writes the constant back
 // with tcgen05.st before it releases the buffer to the MMA warp.
 //
-// Persistent, one CTA per SM, 128 x 256 output tiles walked with stride
-// gridDim.x (M-tile index fastest). Warp roles:
+// Persistent, one CTA per SM, 128 x 128 output tiles walked with stride
+// gridDim.x (M-tile index fastest). The fold of every group is on the
+// epilogue's critical path and its fixed cost (wait, fence, release) is paid
+// per warp, so few warps with many columns each do it best: eight epilogue
+// warps of 64 columns (64 fp32 accumulators and one group's 64 INT32 values
+// per thread), in a CTA of ten warps that can give each thread ~200 registers.
+// Warp roles:
 //   warp 0      TMA producer: 128-byte-swizzled K-blocks (128 int8 columns of
-//               Xq and Wq) into a 4-deep shared-memory ring
-//   warp 1      owns the 512-column TMEM allocation (two 256-column buffers)
-//               and issues the MMAs (G/32 per group, K = 32 each)
-//   warps 2-17  epilogue: warp w reads TMEM lane quarter (w % 4) and the 64
+//               Xq and Wq) into a 6-deep shared-memory ring
+//   warp 1      owns the 512-column TMEM allocation (four 128-column buffers,
+//               so the MMAs run up to three groups ahead of the fold) and
+//               issues the MMAs (G/32 per group, K = 32 each)
+//   warps 2-9   epilogue: warp w reads TMEM lane quarter (w % 4) and the 64
 //               columns [64 p, 64 p + 64) of the tile, p = (w - 2) / 4
 // Every mbarrier wait is bounded; a wait that gives up records
 // I8MM_ERR_TIMEOUT in the status word and the CTA stops issuing work.
@@ -45,16 +51,17 @@ namespace i8mm {
 namespace {
 
 constexpr int BM = 128;
-constexpr int BN = 256;
+constexpr int BN = 128;
+constexpr int NBUF = 4;                // TMEM accumulator buffers of BN columns
 constexpr int KB = 128;                // int8 columns per K-block
-constexpr int STAGES = 4;
+constexpr int STAGES = 6;
 constexpr int A_BYTES = BM * KB;
 constexpr int B_BYTES = BN * KB;
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
 constexpr int RING_BYTES = STAGES * STAGE_BYTES;
-constexpr int BAR_BYTES = (2 * STAGES + 4) * 8 + 16;
+constexpr int BAR_BYTES = (2 * STAGES + 2 * NBUF) * 8 + 16;
 constexpr int SMEM_BYTES = 1024 + RING_BYTES + BAR_BYTES;
-constexpr int kEpiWarps = 16;
+constexpr int kEpiWarps = 8;
 constexpr int kThreads = 64 + 32 * kEpiWarps;
 constexpr int kStatusTimeout = -5;     // == I8MM_ERR_TIMEOUT
 constexpr uint32_t TMEM_COLS = 512;
@@ -76,9 +83,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* smem = smem_raw + ((1024u - (smem_addr(smem_raw) & 1023u)) & 1023u);
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + RING_BYTES);
   uint64_t* empty = full + STAGES;
-  uint64_t* acc_full = empty + STAGES;   // [2]
-  uint64_t* acc_free = acc_full + 2;     // [2]
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_free + 2);
+  uint64_t* acc_full = empty + STAGES;   // [NBUF]
+  uint64_t* acc_free = acc_full + NBUF;  // [NBUF]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_free + NBUF);
   volatile int32_t* abort_flag = reinterpret_cast<volatile int32_t*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5;
@@ -94,7 +101,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
-    for (int b = 0; b < 2; ++b) {
+    for (int b = 0; b < NBUF; ++b) {
       mbar_init(&acc_full[b], 1);
       mbar_init(&acc_free[b], kEpiWarps);
     }
@@ -135,50 +142,56 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
   } else if (warp == 1) {
-    if (lane == 0) {
-      // ------------------------------------------------------------ MMA issuer
-      constexpr uint32_t idesc = make_idesc(2 /*s32*/, 1 /*signed*/, BM, BN);
-      uint32_t g = 0;    // K-blocks consumed (ring position)
-      uint32_t u = 0;    // groups issued (buffer u & 1, its use u >> 1)
-      int mm = 0;        // MMAs issued into the current group
-      uint32_t d = tmem;
-      bool ok = true;
-      for (int tile = blockIdx.x; tile < num_tiles && ok && !*abort_flag; tile += gridDim.x) {
-        for (int it = 0; it < nk && ok; ++it, ++g) {
-          const int s = g % STAGES;
-          if (!mbar_wait(&full[s], (g / STAGES) & 1)) {
-            ok = false;
-            break;
-          }
-          const uint32_t a = smem_addr(smem + s * STAGE_BYTES);
-          const uint32_t b = a + A_BYTES;
+    // -------------------------------------------------------------- MMA issuer
+    // The whole warp runs the loop (waits are warp-uniform through __all_sync)
+    // and one elected lane issues each MMA and commit: a converged warp issues
+    // MMAs faster than a lone lane of a diverged branch.
+    constexpr uint32_t idesc = make_idesc(2 /*s32*/, 1 /*signed*/, BM, BN);
+    uint32_t g = 0;    // K-blocks consumed (ring position)
+    uint32_t u = 0;    // groups issued (buffer u % NBUF, its use u / NBUF)
+    int mm = 0;        // MMAs issued into the current group
+    uint32_t d = tmem;
+    bool ok = true;
+    for (int tile = blockIdx.x; tile < num_tiles && ok && !*abort_flag; tile += gridDim.x) {
+      for (int it = 0; it < nk && ok; ++it, ++g) {
+        const int s = g % STAGES;
+        ok = __all_sync(0xffffffffu, mbar_wait(&full[s], (g / STAGES) & 1));
+        if (!ok) break;
+        const uint32_t a = smem_addr(smem + s * STAGE_BYTES);
+        const uint32_t b = a + A_BYTES;
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk) {
-            if (mm == 0) {
-              // The buffer holds the 1.5 * 2^23 pattern again (written by the
-              // epilogue after its previous group).
-              if (!mbar_wait(&acc_free[u & 1], (u >> 1) & 1)) {
-                ok = false;
-                break;
-              }
+        for (int kk = 0; kk < 4; ++kk) {
+          if (mm == 0) {
+            // The buffer holds the 1.5 * 2^23 pattern again (written by the
+            // epilogue after its previous group). The fence that orders those
+            // stores before the MMAs stalls the issue for several hundred
+            // cycles, so the buffers are claimed two groups at a time, with one
+            // fence. (A claim past the last group waits for a release that
+            // still comes: the epilogue frees every buffer it reads.)
+            if ((u & 1) == 0) {
+              ok = __all_sync(0xffffffffu,
+                              mbar_wait(&acc_free[u % NBUF], (u / NBUF) & 1) &&
+                                  mbar_wait(&acc_free[(u + 1) % NBUF], ((u + 1) / NBUF) & 1));
+              if (!ok) break;
               tc_fence_after();
-              d = tmem + (u & 1) * BN;
             }
-            mma_i8(d, sw128_kmajor_desc(a + 32 * kk), sw128_kmajor_desc(b + 32 * kk), idesc, 1u);
-            if (++mm == kPerGroup) {
-              mma_commit(&acc_full[u & 1]);
-              mm = 0;
-              ++u;
-            }
+            d = tmem + (u % NBUF) * BN;
           }
-          if (!ok) break;
-          mma_commit(&empty[s]);
+          mma_i8_elect(d, sw128_kmajor_desc(a + 32 * kk), sw128_kmajor_desc(b + 32 * kk), idesc,
+                       1u);
+          if (++mm == kPerGroup) {
+            mma_commit_elect(&acc_full[u % NBUF]);
+            mm = 0;
+            ++u;
+          }
         }
+        if (!ok) break;
+        mma_commit_elect(&empty[s]);
       }
-      if (!ok) {
-        record_error(status, kStatusTimeout);
-        *abort_flag = 1;
-      }
+    }
+    if (!ok && lane == 0) {
+      record_error(status, kStatusTimeout);
+      *abort_flag = 1;
     }
   } else {
     // -------------------------------------------------------------- epilogue
@@ -186,9 +199,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int part = (warp - 2) >> 2;
     const int col_lo = part * 64;
     const uint32_t lane_base = tmem + (static_cast<uint32_t>(q * 32) << 16);
-    // Both buffers start as the 1.5 * 2^23 pattern.
+    // Every buffer starts as the 1.5 * 2^23 pattern.
 #pragma unroll
-    for (int b = 0; b < 2; ++b)
+    for (int b = 0; b < NBUF; ++b)
 #pragma unroll
       for (int c = 0; c < 64; c += 16)
         tmem_st_32x32b_x16_fill(lane_base + b * BN + col_lo + c, kMagicBits);
@@ -196,8 +209,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_before();
     __syncwarp();
     if (lane == 0) {
-      mbar_arrive(&acc_free[0]);
-      mbar_arrive(&acc_free[1]);
+#pragma unroll
+      for (int b = 0; b < NBUF; ++b) mbar_arrive(&acc_free[b]);
     }
     const uint64_t magic2 = f2pack(12582912.0f, 12582912.0f);
     uint32_t u = 0;
@@ -214,13 +227,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint64_t acc[32];
 #pragma unroll
       for (int j = 0; j < 32; ++j) acc[j] = 0ull;
+      float sx = live_r ? __ldg(x_absmax + xoff) : 0.0f;
+      float sw = live_c ? __ldg(w_absmax + woff) : 0.0f;
       for (int gi = 0; gi < ng; ++gi, ++u) {
-        const float sx = live_r ? __ldg(x_absmax + xoff + gi) : 0.0f;
-        const float sw = live_c ? __ldg(w_absmax + woff + gi) : 0.0f;
         const float sc = __fmul_rn(sx, sw);
+        if (gi + 1 < ng) {                    // next group's scales, loaded under the wait
+          sx = live_r ? __ldg(x_absmax + xoff + gi + 1) : 0.0f;
+          sw = live_c ? __ldg(w_absmax + woff + gi + 1) : 0.0f;
+        }
         const uint64_t sc2 = f2pack(sc, sc);
-        const uint32_t buf = u & 1;
-        ok = __all_sync(0xffffffffu, mbar_wait(&acc_full[buf], (u >> 1) & 1));
+        const uint32_t buf = u % NBUF;
+        ok = __all_sync(0xffffffffu, mbar_wait(&acc_full[buf], (u / NBUF) & 1));
         if (!ok) {
           record_error(status, kStatusTimeout);
           *abort_flag = 1;
@@ -228,20 +245,19 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tc_fence_after();
         const uint32_t base = lane_base + buf * BN + col_lo;
+        uint32_t v[64];
+        tmem_ld_32x32b_x32(base, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
+        tmem_ld_32x32b_x32(base + 32, *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
+        tmem_ld_wait();
 #pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          uint32_t v[8];
-          tmem_ld_32x32b_x8(base + 8 * c, v);
-          tmem_ld_wait();
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            const uint64_t cg = sub2(static_cast<uint64_t>(v[2 * j]) |
-                                         (static_cast<uint64_t>(v[2 * j + 1]) << 32),
-                                     magic2);
-            acc[4 * c + j] = fma2(cg, sc2, acc[4 * c + j]);
-          }
-          if (c & 1) tmem_st_32x32b_x16_fill(base + 8 * (c - 1), kMagicBits);
+        for (int j = 0; j < 32; ++j) {
+          const uint64_t cg = sub2(static_cast<uint64_t>(v[2 * j]) |
+                                       (static_cast<uint64_t>(v[2 * j + 1]) << 32),
+                                   magic2);
+          acc[j] = fma2(cg, sc2, acc[j]);
         }
+#pragma unroll
+        for (int c = 0; c < 64; c += 16) tmem_st_32x32b_x16_fill(base + c, kMagicBits);
         tmem_st_wait();
         tc_fence_before();
         __syncwarp();

@@ -50,33 +50,51 @@ __device__ __forceinline__ float block_max(float v, float* red) {
   return m;
 }
 
-// One thread per column group of 8, a slice of rows per CTA (blockIdx.y);
-// partial maxima merged with atomicMax on the bit patterns.
+// A CTA covers 256 columns (32 threads of 8-column vectors) of a slice of rows
+// (blockIdx.y); its 8 row lanes take every 8th row of the slice, reduce in
+// shared memory, and merge with atomicMax on the bit patterns (one atomic per
+// column per CTA).
 __global__ void __launch_bounds__(kThreads) column_absmax_kernel(const __half* __restrict__ X,
                                                                  int rows, int K, int row_slice,
                                                                  float* __restrict__ colmax) {
-  const int v = blockIdx.x * kThreads + threadIdx.x;   // 8-column vector index
-  if (v * 8 >= K) return;
+  __shared__ uint4 part[8][32];
+  const int cv = threadIdx.x & 31;           // vector within the CTA's 32
+  const int rl = threadIdx.x >> 5;           // row lane 0..7
+  const int v = blockIdx.x * 32 + cv;        // 8-column vector index
+  const bool live = v * 8 < K;
   const int r0 = blockIdx.y * row_slice;
   const int r1 = min(rows, r0 + row_slice);
   __half2 m[4];
 #pragma unroll
   for (int i = 0; i < 4; ++i) m[i] = __float2half2_rn(0.0f);
-  for (int r = r0; r < r1; ++r) {
-    const uint4 u = __ldg(reinterpret_cast<const uint4*>(X + static_cast<size_t>(r) * K) + v);
-    const uint32_t* w = reinterpret_cast<const uint32_t*>(&u);
+  if (live) {
+    for (int r = r0 + rl; r < r1; r += 8) {
+      const uint4 u = __ldg(reinterpret_cast<const uint4*>(X + static_cast<size_t>(r) * K) + v);
+      const uint32_t* w = reinterpret_cast<const uint32_t*>(&u);
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const uint32_t ab = w[i] & 0x7FFF7FFFu;
-      m[i] = __hmax2(m[i], *reinterpret_cast<const __half2*>(&ab));
+      for (int i = 0; i < 4; ++i) {
+        const uint32_t ab = w[i] & 0x7FFF7FFFu;
+        m[i] = __hmax2(m[i], *reinterpret_cast<const __half2*>(&ab));
+      }
     }
   }
-  unsigned int* out = reinterpret_cast<unsigned int*>(colmax) + v * 8;
+  part[rl][cv] = *reinterpret_cast<const uint4*>(m);
+  __syncthreads();
+  if (rl == 0 && live) {
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const float2 f = __half22float2(m[i]);
-    if (f.x > 0.0f) atomicMax(out + 2 * i, __float_as_uint(f.x));
-    if (f.y > 0.0f) atomicMax(out + 2 * i + 1, __float_as_uint(f.y));
+    for (int l = 1; l < 8; ++l) {
+      const uint4 o = part[l][cv];
+      const __half2* h = reinterpret_cast<const __half2*>(&o);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) m[i] = __hmax2(m[i], h[i]);
+    }
+    unsigned int* out = reinterpret_cast<unsigned int*>(colmax) + v * 8;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float2 f = __half22float2(m[i]);
+      if (f.x > 0.0f) atomicMax(out + 2 * i, __float_as_uint(f.x));
+      if (f.y > 0.0f) atomicMax(out + 2 * i + 1, __float_as_uint(f.y));
+    }
   }
 }
 
@@ -179,8 +197,12 @@ int sq_sizes(int M, int N, int K) {
 cudaError_t launch_column_absmax(const __half* X, int rows, int K, float* colmax,
                                  cudaStream_t s) {
   const int nv = K / 8;
-  const int row_slice = 64;
-  dim3 grid((nv + kThreads - 1) / kThreads, (rows + row_slice - 1) / row_slice);
+  const int col_blocks = (nv + 31) / 32;
+  // about four CTAs per SM over the whole matrix, at least 8 rows per slice
+  int slices = (4 * 148 + col_blocks - 1) / col_blocks;
+  int row_slice = (rows + slices - 1) / slices;
+  row_slice = row_slice < 8 ? 8 : row_slice;
+  dim3 grid(col_blocks, (rows + row_slice - 1) / row_slice);
   column_absmax_kernel<<<grid, kThreads, 0, s>>>(X, rows, K, row_slice, colmax);
   return cudaGetLastError();
 }

@@ -4,10 +4,12 @@
 // tokens, ties to the lower column index.
 //
 // One CTA: radix select of the k-th largest key over the column maxima (fp32
-// >= 0, whose bit patterns order like the values), four passes of 8-bit digits
-// with a shared-memory histogram; then every key above it is selected, and of
-// the keys equal to it the ones with the lowest column indices, by an
-// index-ordered block scan. The result is an outlier bitmap.
+// >= 0, whose bit patterns order like the values), held in registers; four
+// passes of 8-bit digits, each a shared-memory histogram (one atomic per
+// distinct digit per warp) and a warp scan of its 256 bins; then every key
+// above the k-th is selected, and of the keys equal to it the ones with the
+// lowest column indices, by an index-ordered block scan. The result is an
+// outlier bitmap.
 #include <cuda_runtime.h>
 
 #include <cstdint>
@@ -19,17 +21,75 @@ namespace i8mm {
 namespace {
 
 constexpr int kThreads = 1024;
+constexpr int kWarps = kThreads / 32;
 constexpr int kMaxWords = 65536 / 32;
 
+// The digit d of the current pass such that the keys with that digit (and the
+// prefix so far) hold the `remaining`-th largest: suffix sums of the histogram
+// from digit 255 down, by warp 0 (eight bins per lane, then a warp scan).
+__device__ __forceinline__ void pick_digit(const unsigned int* hist, unsigned int remaining,
+                                           unsigned int* s_digit, unsigned int* s_above) {
+  const int lane = threadIdx.x & 31;
+  // lane l owns bins 255 - 8l - i, i = 0..7 (highest digits first)
+  unsigned int c[8], tot = 0u;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    c[i] = hist[255 - 8 * lane - i];
+    tot += c[i];
+  }
+  unsigned int incl = tot;   // inclusive prefix over lanes 0..lane
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const unsigned int t = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += t;
+  }
+  unsigned int before = incl - tot;   // keys in higher digits than this lane's bins
+  // the lane whose range contains the remaining-th key
+  const bool mine = before < remaining && incl >= remaining;
+  if (mine) {
+    unsigned int cum = before;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      if (cum + c[i] >= remaining) {
+        *s_digit = static_cast<unsigned int>(255 - 8 * lane - i);
+        *s_above = cum;
+        break;
+      }
+      cum += c[i];
+    }
+  }
+}
+
+// KPT keys per thread (keys t + i * kThreads) held in registers, K <= KPT *
+// kThreads; KPT = 64 reads them from global memory (L2) in every pass instead.
+template <int KPT>
 __global__ void __launch_bounds__(kThreads) topk_select_kernel(const float* __restrict__ colmax,
                                                                int K, int k,
                                                                uint32_t* __restrict__ bitmap) {
+  constexpr bool kRegs = KPT <= 16;
+  constexpr int kMaxKeys = KPT;
   __shared__ unsigned int hist[256];
   __shared__ uint32_t words[kMaxWords];
-  __shared__ unsigned int s_prefix, s_remaining, s_taken;
-  __shared__ unsigned int warp_cnt[kThreads / 32];
+  __shared__ unsigned int s_digit, s_above;
+  __shared__ unsigned int warp_cnt[kWarps];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int nw = (K + 31) / 32;
+  const int per = (K + kThreads - 1) / kThreads;
+  // Thread t holds keys j = t + i * kThreads (coalesced loads, once).
+  unsigned int kr[kRegs ? KPT : 1];
+#pragma unroll
+  for (int i = 0; i < (kRegs ? KPT : 1); ++i) {
+    const int j = tid + i * kThreads;
+    kr[i] = (kRegs && i < per && j < K) ? __float_as_uint(__ldg(colmax + j)) : 0u;
+  }
+  auto key_of = [&](int i) -> unsigned int {
+    if constexpr (kRegs) {
+      return kr[i];
+    } else {
+      const int j = tid + i * kThreads;
+      return j < K ? __float_as_uint(__ldg(colmax + j)) : 0u;
+    }
+  };
   for (int w = tid; w < nw; w += kThreads) words[w] = 0u;
   __syncthreads();
   if (k >= K) {
@@ -40,50 +100,50 @@ __global__ void __launch_bounds__(kThreads) topk_select_kernel(const float* __re
       const int shift = 24 - 8 * pass;
       for (int i = tid; i < 256; i += kThreads) hist[i] = 0u;
       __syncthreads();
-      for (int j = tid; j < K; j += kThreads) {
-        const unsigned int key = __float_as_uint(colmax[j]);
-        if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & 255u], 1u);
-      }
-      __syncthreads();
-      if (tid == 0) {
-        unsigned int cum = 0u;
-        for (int d = 255; d >= 0; --d) {
-          if (cum + hist[d] >= remaining) {
-            s_prefix = prefix | (static_cast<unsigned int>(d) << shift);
-            s_remaining = remaining - cum;
-            break;
+#pragma unroll
+      for (int i = 0; i < kMaxKeys; ++i) {
+        const int j = tid + i * kThreads;
+        if (i < per) {
+          const unsigned int ki = key_of(i);
+          const bool in = j < K && (ki & mask) == prefix;
+          const unsigned int d = (ki >> shift) & 255u;
+          // one atomic per distinct digit among the warp's matching lanes
+          const unsigned int act = __ballot_sync(0xffffffffu, in);
+          if (in) {
+            const unsigned int peers = __match_any_sync(act, d);
+            if (lane == __ffs(peers) - 1) atomicAdd(&hist[d], __popc(peers));
           }
-          cum += hist[d];
         }
       }
       __syncthreads();
-      prefix = s_prefix;
-      remaining = s_remaining;
+      if (warp == 0) pick_digit(hist, remaining, &s_digit, &s_above);
+      __syncthreads();
+      prefix |= s_digit << shift;
+      remaining -= s_above;
       mask |= 0xFFu << shift;
-      __syncthreads();
     }
-    // prefix is the k-th largest key; `remaining` keys equal to it are taken.
-    if (tid == 0) s_taken = 0u;
-    __syncthreads();
-    for (int base = 0; base < K; base += kThreads) {
-      const int j = base + tid;
-      const unsigned int key = (j < K) ? __float_as_uint(colmax[j]) : 0u;
-      const bool eq = (j < K) && key == prefix;
-      const unsigned int ball = __ballot_sync(0xffffffffu, eq);
-      if (lane == 0) warp_cnt[warp] = __popc(ball);
-      __syncthreads();
-      unsigned int before = s_taken;
-      for (int w = 0; w < warp; ++w) before += warp_cnt[w];
-      before += __popc(ball & ((1u << lane) - 1u));
-      const bool take = (j < K) && (key > prefix || (eq && before < remaining));
-      if (take) atomicOr(&words[j >> 5], 1u << (j & 31));
-      __syncthreads();
-      if (tid == 0) {
+    // prefix is the k-th largest key; `remaining` keys equal to it are taken,
+    // the ones with the lowest column indices.
+    unsigned int taken = 0u;
+#pragma unroll
+    for (int i = 0; i < kMaxKeys; ++i) {
+      if (i < per) {
+        const int j = tid + i * kThreads;
+        const unsigned int ki = key_of(i);
+        const bool eq = j < K && ki == prefix;
+        const unsigned int ball = __ballot_sync(0xffffffffu, eq);
+        if (lane == 0) warp_cnt[warp] = __popc(ball);
+        __syncthreads();
+        unsigned int before = taken;
+        for (int w = 0; w < warp; ++w) before += warp_cnt[w];
+        before += __popc(ball & ((1u << lane) - 1u));
+        const bool take = j < K && (ki > prefix || (eq && before < remaining));
+        if (take) atomicOr(&words[j >> 5], 1u << (j & 31));
         unsigned int tot = 0u;
-        for (int w = 0; w < kThreads / 32; ++w) tot += warp_cnt[w];
-        s_taken += tot;
+        for (int w = 0; w < kWarps; ++w) tot += warp_cnt[w];
+        taken += tot;
+        __syncthreads();
       }
-      __syncthreads();
     }
   }
   __syncthreads();
@@ -95,7 +155,12 @@ __global__ void __launch_bounds__(kThreads) topk_select_kernel(const float* __re
 cudaError_t launch_topk_select(const float* colmax, int K, int k, uint32_t* bitmap,
                                cudaStream_t s) {
   if (K <= 0 || K > 65536) return cudaErrorInvalidValue;
-  topk_select_kernel<<<1, kThreads, 0, s>>>(colmax, K, k, bitmap);
+  if (K <= 4 * kThreads)
+    topk_select_kernel<4><<<1, kThreads, 0, s>>>(colmax, K, k, bitmap);
+  else if (K <= 16 * kThreads)
+    topk_select_kernel<16><<<1, kThreads, 0, s>>>(colmax, K, k, bitmap);
+  else
+    topk_select_kernel<64><<<1, kThreads, 0, s>>>(colmax, K, k, bitmap);
   return cudaGetLastError();
 }
 
