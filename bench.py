@@ -274,7 +274,7 @@ NCU_TRAFFIC = {
              "source": "profiles/gemm_i8_persistent_opt-6.7b-ffn-up-prefill.md"},
     "quantize": {"bytes": 27.326976e6 + 1.792e3,
                  "source": "profiles/detect_quantize_compact_opt-6.7b-ffn-up-prefill.md"},
-    "rotate": {"bytes": 16.80512e6,
+    "rotate": {"bytes": 16.804608e6,
                "source": "profiles/rotate_rows_opt-6.7b-ffn-up-prefill.md"},
     "decode": {"bytes": 19.596544e6,
                "source": "profiles/decode_kernel_decode-16x4096x4096.md"},

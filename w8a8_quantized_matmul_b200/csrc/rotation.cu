@@ -53,6 +53,13 @@ __device__ __forceinline__ int rot_code(float r, float a, float qmax) {
   return max(-m, min(m, q));
 }
 
+// fp16 -> fp64 in one conversion (exact).
+__device__ __forceinline__ double h2d(__half h) {
+  double d;
+  asm("cvt.f64.f16 %0, %1;" : "=d"(d) : "h"(__half_as_ushort(h)));
+  return d;
+}
+
 // The 16 rotated values of columns [16p, 16p + 16) of a row, p = piece index;
 // lanes of one group of G columns hold consecutive pieces. `live` false gives
 // zeros (a piece past the end of the row; whole groups only).
@@ -67,8 +74,8 @@ __device__ __forceinline__ void rotate16(const __half* __restrict__ src, bool li
     const __half* h1 = reinterpret_cast<const __half*>(&u1);
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
-      v[i] = static_cast<double>(__half2float(h0[i]));
-      v[8 + i] = static_cast<double>(__half2float(h1[i]));
+      v[i] = h2d(h0[i]);
+      v[8 + i] = h2d(h1[i]);
     }
   } else {
 #pragma unroll
@@ -101,15 +108,18 @@ __device__ __forceinline__ void rotate16(const __half* __restrict__ src, bool li
 // quant_rcp(a): q = rint(fl32(n / a)) with n = fl32(r * qmax). The quotient is
 // formed without a division: q0 = fl(n * ra), e = fma(q0, -a, n) (exact),
 // qc = fma(e, ra, q0), within about one ulp of n / a. Where qc lies within
-// 2^-15 (four ulps at |q| < 128) of a half-integer the correctly rounded
+// about 2^-15 (four ulps at |q| < 128) of a half-integer the correctly rounded
 // quotient could round the other way, so those codes are recomputed with a
 // correctly rounded division; everywhere else rint(qc) is the code. rint is
-// the low bits of fl(qc + 1.5 * 2^23) (ties to even).
+// the low bits of fl(qc + 1.5 * 2^23) (ties to even); the near-tie test is
+// |t^2 - 1/4| < 2^-15 with t = qc - rint(qc) (exact), i.e. ||t| - 1/2| < ~2^-15.
+// The codes come back packed, four bytes per word.
 __device__ __forceinline__ void rot_codes16(const float (&r)[16], float a, float ra, float qmax,
-                                            int (&q)[16]) {
+                                            uint32_t (&b)[4]) {
   const uint64_t na2 = f2pack(-a, -a), ra2 = f2pack(ra, ra), qm2 = f2pack(qmax, qmax);
-  const uint64_t mg2 = f2pack(kMagic, kMagic);
+  const uint64_t mg2 = f2pack(kMagic, kMagic), nq2 = f2pack(-0.25f, -0.25f);
   bool tie = false;
+  uint32_t lo16[8];
 #pragma unroll
   for (int j = 0; j < 8; ++j) {
     const uint64_t n = mul2(f2pack(r[2 * j], r[2 * j + 1]), qm2);
@@ -117,25 +127,25 @@ __device__ __forceinline__ void rot_codes16(const float (&r)[16], float a, float
     const uint64_t qc = fma2(fma2(q0, na2, n), ra2, q0);
     const uint64_t sm = add2(qc, mg2);
     const uint64_t t = sub2(qc, sub2(sm, mg2));            // qc - rint(qc), exact
-    q[2 * j] = __float_as_int(lo(sm)) - 0x4B400000;
-    q[2 * j + 1] = __float_as_int(hi(sm)) - 0x4B400000;
-    tie |= fabsf(fabsf(lo(t)) - 0.5f) < 0x1p-15f;
-    tie |= fabsf(fabsf(hi(t)) - 0.5f) < 0x1p-15f;
+    const uint64_t d = fma2(t, t, nq2);                    // t^2 - 1/4
+    tie |= fabsf(lo(d)) < 0x1p-15f;
+    tie |= fabsf(hi(d)) < 0x1p-15f;
+    lo16[j] = __byte_perm(static_cast<uint32_t>(sm), static_cast<uint32_t>(sm >> 32), 0x0040);
   }
+#pragma unroll
+  for (int w = 0; w < 4; ++w) b[w] = __byte_perm(lo16[2 * w], lo16[2 * w + 1], 0x5410);
   if (tie) {
 #pragma unroll
-    for (int i = 0; i < 16; ++i) q[i] = rot_code(r[i], a, qmax);
+    for (int w = 0; w < 4; ++w) {
+      b[w] = 0u;
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+        b[w] |= (static_cast<uint32_t>(rot_code(r[4 * w + i], a, qmax)) & 0xFFu) << (8 * i);
+    }
   }
 }
 
-__device__ __forceinline__ void store_codes16(const int (&q)[16], int8_t* dst) {
-  uint32_t b[4];
-#pragma unroll
-  for (int j = 0; j < 4; ++j)
-    b[j] = (static_cast<uint32_t>(q[4 * j]) & 0xFFu) |
-           ((static_cast<uint32_t>(q[4 * j + 1]) & 0xFFu) << 8) |
-           ((static_cast<uint32_t>(q[4 * j + 2]) & 0xFFu) << 16) |
-           ((static_cast<uint32_t>(q[4 * j + 3]) & 0xFFu) << 24);
+__device__ __forceinline__ void store_codes16(const uint32_t (&b)[4], int8_t* dst) {
   *reinterpret_cast<uint4*>(dst) = make_uint4(b[0], b[1], b[2], b[3]);
 }
 
@@ -190,7 +200,7 @@ __global__ void __launch_bounds__(kRowThreads) rotate_rows_kernel(
         r[4 * i] = f.x; r[4 * i + 1] = f.y; r[4 * i + 2] = f.z; r[4 * i + 3] = f.w;
       }
     }
-    int q[16];
+    uint32_t q[4];
     rot_codes16(r, a, ra, 127.0f, q);
     store_codes16(q, Xq + row * K + 16 * p);
     if (R) {
@@ -235,15 +245,16 @@ __global__ void __launch_bounds__(256) rotate_groups_kernel(
   } else {
     a = __ldg(scale + (row / G) * ng + g);
   }
-  int q[16];
+  uint32_t q[4];
   rot_codes16(r, a, a == 0.0f ? 0.0f : __frcp_rn(a), 7.0f, q);
   if (Xq) store_codes16(q, Xq + row * K + 16 * p);
   if (Xp) {
+    // bytes (two's complement, |q| <= 7) to nibbles: code i of byte word w
     uint32_t w0 = 0u, w1 = 0u;
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
-      w0 |= (static_cast<uint32_t>(q[i]) & 0xFu) << (4 * i);
-      w1 |= (static_cast<uint32_t>(q[8 + i]) & 0xFu) << (4 * i);
+      w0 |= ((q[i >> 2] >> (8 * (i & 3))) & 0xFu) << (4 * i);
+      w1 |= ((q[2 + (i >> 2)] >> (8 * (i & 3))) & 0xFu) << (4 * i);
     }
     *reinterpret_cast<uint2*>(Xp + row * (K / 8) + 2 * p) = make_uint2(w0, w1);
   }
@@ -284,7 +295,8 @@ cudaError_t launch_rows_g(const __half* X, int rows, int K, int8_t* Xq, float* s
   const int np = K / 16;
   int nt = ((np + 31) / 32) * 32;
   if (nt > kRowThreads) nt = kRowThreads;
-  const size_t smem = static_cast<size_t>(K) * sizeof(float);
+  // A row of at most nt pieces keeps its rotated values in registers.
+  const size_t smem = np <= nt ? 0 : static_cast<size_t>(K) * sizeof(float);
   if (smem > 48 * 1024) {
     cudaError_t e = cudaFuncSetAttribute(rotate_rows_kernel<G>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
