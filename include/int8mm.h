@@ -350,6 +350,15 @@ int int8_debug_gemm_i32(const int8_t* Xq, const int8_t* Wq, int M, int N, int K,
                         i8mm_stream_t stream);
 
 /*
+ * Self-test of the bounded device-side waits: launches one CTA that waits on an
+ * mbarrier phase nothing completes; after the library's wait limit (2 s) the
+ * wait gives up and the CTA writes I8MM_ERR_TIMEOUT into *status (device int32,
+ * cleared first) and exits normally. Returns I8MM_OK once launched; the caller
+ * synchronises `stream` and reads *status. Nothing faults or hangs.
+ */
+int int8_selftest_wait_timeout(int32_t* status, i8mm_stream_t stream);
+
+/*
  * Reads the device status word a previous int8_mixed_matmul left in its
  * workspace (synchronises `stream`). Returns I8MM_OK, I8MM_ERR_TIMEOUT if
  * a bounded device-side wait gave up, or I8MM_ERR_CUDA.

@@ -524,3 +524,13 @@ def int4_rotated_workspace_views(workspace: torch.Tensor, M: int, K: int, G: int
     return {"status": workspace[0:4].view(torch.int32),
             "x_absmax": workspace[xa:xa + 4 * M * (K // G)].view(torch.float32).view(M, K // G),
             "Xq": workspace[xq:xq + M * K].view(torch.int8).view(M, K)}
+
+
+def selftest_wait_timeout(stream=None) -> int:
+    """Runs the bounded-wait self-test; returns the status the device recorded
+    (I8MM_ERR_TIMEOUT when the wait gave up as designed). Takes about 2 s."""
+    status = torch.zeros((1,), dtype=torch.int32, device="cuda")
+    check("int8_selftest_wait_timeout",
+          load().int8_selftest_wait_timeout(_ptr(status), _stream(stream)))
+    torch.cuda.synchronize()
+    return int(status.item())
