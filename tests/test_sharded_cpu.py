@@ -84,3 +84,62 @@ def test_token_sharded_matches_whole_batch(world, split):
     np.testing.assert_array_equal(Y, ref["Y"])
     for r in range(world):
         np.testing.assert_array_equal(results[r][1].view(np.uint32), ref["bitmap"])
+
+
+def _report_and_exit(q, msg):
+    # flush the queue's feeder thread before leaving without the process
+    # group's teardown (its peer is gone)
+    q.put(msg)
+    q.close()
+    q.join_thread()
+    os._exit(0)
+
+
+def _failing_worker(rank, world, port, mode, q):
+    """Rank 1 leaves (mode "exit") or stalls (mode "stall") before the exchange;
+    rank 0 must get an error from its collective instead of waiting forever."""
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    import datetime
+    import time
+    try:
+        dist.init_process_group("gloo", rank=rank, world_size=world,
+                                timeout=datetime.timedelta(seconds=3))
+        dist.barrier()          # both ranks are up before one of them goes away
+    except Exception as e:
+        _report_and_exit(q, ("setup failed: " + type(e).__name__, 0.0))
+    if rank == 1:
+        if mode == "stall":
+            time.sleep(12)
+        os._exit(0)
+    from w8a8_quantized_matmul_b200.sharded import token_sharded_mixed_matmul
+    X, W, _ = synth.random_case(16, 64, 8, 1, seed=3)
+    Wq, w_scale = oracle.quantize_weight_rows(W)
+    t0 = time.perf_counter()
+    try:
+        token_sharded_mixed_matmul(torch.from_numpy(X), torch.from_numpy(Wq),
+                                   torch.from_numpy(w_scale), torch.from_numpy(W), 6.0,
+                                   find=_find, apply=_apply)
+        msg = ("no error", time.perf_counter() - t0)
+    except Exception as e:  # the collective's failure reaches the host as an exception
+        msg = (type(e).__name__, time.perf_counter() - t0)
+    _report_and_exit(q, msg)
+
+
+@pytest.mark.parametrize("mode", ["exit", "stall"])
+def test_lost_rank_ends_the_exchange_with_an_error(mode):
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_failing_worker, args=(r, 2, port, mode, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    try:
+        what, secs = q.get(timeout=90)
+        assert what != "no error" and not what.startswith("setup failed"), what
+        assert secs < 30            # the process-group timeout (3 s), not a hang
+    finally:
+        for p in procs:
+            p.join(timeout=30)
+            if p.is_alive():
+                p.kill()
