@@ -177,3 +177,25 @@ def test_rotation_entry_points_validation(lib):
     assert lib.int4_rotate_quantize_weight_blocks(A, 96, 256, 64, A, A, None) == _lib.I8MM_ERR_INVALID_ARG
     assert lib.int4_rotate_quantize_weight_blocks(A, 128, 256, 64, None, A, None) == _lib.I8MM_ERR_INVALID_ARG
     assert lib.int4_rotate_quantize_weight_blocks(A, 0, 256, 64, None, None, None) == _lib.I8MM_OK
+
+
+def test_int4_entry_points_validation(lib):
+    # unpack: K % 32, 16-byte alignment, empty
+    assert lib.int4_unpack(A, 4, 48, A, None) == _lib.I8MM_ERR_INVALID_ARG
+    assert lib.int4_unpack(A, 4, 64, MIS, None) == _lib.I8MM_ERR_ALIGNMENT
+    assert lib.int4_unpack(None, 4, 64, A, None) == _lib.I8MM_ERR_INVALID_ARG
+    assert lib.int4_unpack(None, 0, 64, None, None) == _lib.I8MM_OK
+    # W4A4 matmul: G in {64, 128, 256}, K % 128, N % G, workspace
+    need = lib.int4_rotated_workspace_size(64, 256, 512, 128)
+    assert need >= 64 * 512 + 4 * 64 * 4
+    assert lib.int4_rotated_workspace_size(64, 256, 520, 128) == 0
+    assert lib.int4_rotated_matmul(A, A, A, 64, 256, 512, 32, A, A, need, None) == _lib.I8MM_ERR_INVALID_ARG
+    assert lib.int4_rotated_matmul(A, A, A, 64, 256, 320, 64, A, A, need, None) == _lib.I8MM_ERR_INVALID_ARG
+    assert lib.int4_rotated_matmul(A, A, A, 64, 200, 512, 128, A, A, need, None) == _lib.I8MM_ERR_INVALID_ARG
+    assert lib.int4_rotated_matmul(A, A, A, 64, 256, 512, 128, A, A, need - 1, None) == _lib.I8MM_ERR_WORKSPACE
+    assert lib.int4_rotated_matmul(A, A, A, 64, 256, 512, 128, A, A + 16, need, None) == _lib.I8MM_ERR_ALIGNMENT
+    assert lib.int4_rotated_matmul(MIS, A, A, 64, 256, 512, 128, A, A, need, None) == _lib.I8MM_ERR_ALIGNMENT
+    assert lib.int4_rotated_matmul(A, None, A, 64, 256, 512, 128, A, A, need, None) == _lib.I8MM_ERR_INVALID_ARG
+    assert lib.int4_rotated_matmul(A, A, A, 0, 256, 512, 128, A, None, 0, None) == _lib.I8MM_OK
+    # self-test hook: a status pointer is required
+    assert lib.int8_selftest_wait_timeout(None, None) == _lib.I8MM_ERR_INVALID_ARG
