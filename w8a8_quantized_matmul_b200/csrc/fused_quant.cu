@@ -25,11 +25,11 @@
 //            the outlier product, or a multiple of 64 wide when the GEMM
 //            multiplies them on the tensor cores.
 //
-// The code of x is rint(fl32(fl32(x*127)/a)) clamped to +-127. It is computed as
-// y = fl32(x * fl32(127/a)) rounded with the 1.5*2^23 trick (round to nearest
-// even in one add; the code lands in the low byte). y is within 2.3e-5 of the
-// correctly rounded quotient, so the two round alike unless y lies within
-// 6.2e-5 of a half-integer; such vectors are recomputed with the division.
+// The code of x is rint(fl32(fl32(x*127)/a)) clamped to +-127. The correctly
+// rounded quotient is formed without a division (codes8 in quant_common.cuh:
+// the FMA-corrected product with fl(1/a), exact for every pair of fp16 values
+// with |x| <= a) and rounded with the 1.5*2^23 trick (ties to even in one add;
+// the code lands in the low byte).
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 

@@ -5,6 +5,8 @@
 //                                     ascending column list (stand-alone entry point)
 //   * quantize_rows_kernel          - per-token absmax over the non-outlier columns and
 //                                     INT8 codes, 0 at outliers (stand-alone entry point)
+//   * weight_rowsum_kernel          - sum_k Wq[n][k] per output row, the weight factor of
+//                                     the zero-point correction (offline)
 // (The full path uses the fused, cooperative form of both in fused_quant.cu.)
 //
 // Method: AIInfra "05Infer/06CompDistill/05Quantization01", LLM.int8() section
