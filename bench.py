@@ -85,24 +85,35 @@ class ClockSampler:
         except Exception:
             self.proc.kill()
         self.out.close()
-        rows = []
         with open(self.path) as f:
-            for line in f:
-                parts = [p.strip() for p in line.split(",")]
-                if len(parts) >= 9:
-                    rows.append(parts)
+            lines = f.readlines()
         os.unlink(self.path)
-        if not rows:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
-        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
-        smax = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
-        return {"sm_mhz": statistics.median(sm) if sm else None,
-                "sm_max_mhz": max(smax) if smax else None,
-                "reasons": reasons, "samples": len(rows),
-                "power_w_max": max(float(r[3]) for r in rows if r[3].replace(".", "").isdigit())
-                if any(r[3].replace(".", "").isdigit() for r in rows) else None}
+        return summarize_clock_samples(lines)
+
+
+def summarize_clock_samples(lines):
+    """Median SM clock, max clock, throttle reasons seen and peak power from
+    `nvidia-smi --format=csv,noheader,nounits` lines of ClockSampler.FIELDS."""
+    rows = []
+    for line in lines:
+        parts = [p.strip() for p in line.split(",")]
+        if len(parts) >= 9:
+            rows.append(parts)
+    if not rows:
+        return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+
+    def num(x):
+        return x.replace(".", "", 1).isdigit()
+
+    sm = [float(r[1]) for r in rows if num(r[1])]
+    smax = [float(r[2]) for r in rows if num(r[2])]
+    pw = [float(r[3]) for r in rows if num(r[3])]
+    names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+    reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
+    return {"sm_mhz": statistics.median(sm) if sm else None,
+            "sm_max_mhz": max(smax) if smax else None,
+            "reasons": reasons, "samples": len(rows),
+            "power_w_max": max(pw) if pw else None}
 
 
 # --------------------------------------------------------------------------- oracle timing

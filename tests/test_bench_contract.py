@@ -40,3 +40,34 @@ def test_too_few_warmup_steps_refused():
                         "--warmup", "2"], cwd=ROOT, capture_output=True, text=True, timeout=120)
     assert r.returncode == 2
     assert "warmup" in r.stderr
+
+
+def test_clock_samples_summary():
+    import bench
+    lines = [
+        "0, 1965, 1965, 412.50, 0x0000000000000000, Not Active, Not Active, Not Active, Not Active\n",
+        "0, 1950, 1965, 870.25, 0x0000000000000004, Not Active, Not Active, Not Active, Active\n",
+        "0, 1440, 1965, 990.00, 0x0000000000000004, Not Active, Not Active, Not Active, Active\n",
+        "garbage line\n",
+        "0, [N/A], 1965, [N/A], 0x0, Not Active, Not Active, Not Active, Not Active\n",
+    ]
+    s = bench.summarize_clock_samples(lines)
+    assert s["samples"] == 4
+    assert s["sm_mhz"] == 1950.0 and s["sm_max_mhz"] == 1965.0
+    assert s["reasons"] == ["sw_power_cap"]
+    assert s["power_w_max"] == 990.0
+    bad = bench.summarize_clock_samples(
+        ["0, 900, 1965, 300.0, 0x8, Not Active, Active, Not Active, Not Active\n"])
+    assert bad["reasons"] == ["hw_thermal_slowdown"]
+    assert bench.summarize_clock_samples([])["samples"] == 0
+
+
+def test_rotating_sets_exceed_l2():
+    import bench
+    import synth
+    l2 = 126 * 2 ** 20
+    for name in ("opt-6.7b-ffn-up-prefill", "decode", "llama-70b-ffn-prefill"):
+        w = synth.WORKLOADS[name]
+        n = bench.n_sets_for(w, l2)
+        per = 2 * w.M * w.K + w.M * w.K + w.N * w.K + 2 * w.M * w.N
+        assert n >= 2 and (n * per > 2 * l2 or n == 32)
