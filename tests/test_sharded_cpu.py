@@ -143,3 +143,64 @@ def test_lost_rank_ends_the_exchange_with_an_error(mode):
             p.join(timeout=30)
             if p.is_alive():
                 p.kill()
+
+
+def _apply_cols(X, Wq_local, w_scale_local, W_local, threshold, Y=None, workspace=None):
+    out = oracle.llm_int8_matmul(X.numpy(), W_local.numpy(), threshold, Wq=Wq_local.numpy(),
+                                 w_scale=w_scale_local.numpy())
+    return torch.from_numpy(out["Y"])
+
+
+def _cols_worker(rank, world, port, case, q):
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    import datetime
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=60))
+    try:
+        from w8a8_quantized_matmul_b200.sharded import column_block, column_sharded_mixed_matmul
+        M, K, N, n_out, seed = case
+        X, W, _ = synth.random_case(M, K, N, n_out, seed=seed)
+        n0, n1 = column_block(N, rank, world)
+        Wq, w_scale = oracle.quantize_weight_rows(W[n0:n1])
+        Y_local = column_sharded_mixed_matmul(torch.from_numpy(X), torch.from_numpy(Wq),
+                                              torch.from_numpy(w_scale),
+                                              torch.from_numpy(np.ascontiguousarray(W[n0:n1])),
+                                              6.0, apply=_apply_cols)
+        Y_full = column_sharded_mixed_matmul(torch.from_numpy(X), torch.from_numpy(Wq),
+                                             torch.from_numpy(w_scale),
+                                             torch.from_numpy(np.ascontiguousarray(W[n0:n1])),
+                                             6.0, N=N, gather=True, apply=_apply_cols)
+        q.put((rank, n0, n1, Y_local.numpy(), Y_full.numpy()))
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world,case", [(2, (40, 256, 96, 3, 5)), (3, (17, 320, 200, 4, 6))])
+def test_column_sharded_matches_whole_layer(world, case):
+    """Each rank holds all of X and a block of weight rows: no exchange, the same
+    outlier set everywhere, and the column blocks make up the whole Y exactly."""
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_cols_worker, args=(r, world, port, case, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    got = {}
+    for _ in range(world):
+        rank, n0, n1, Yl, Yf = q.get(timeout=120)
+        got[rank] = (n0, n1, Yl, Yf)
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    M, K, N, n_out, seed = case
+    X, W, _ = synth.random_case(M, K, N, n_out, seed=seed)
+    ref = oracle.llm_int8_matmul(X, W)["Y"]
+    covered = np.zeros(N, bool)
+    for r in range(world):
+        n0, n1, Yl, Yf = got[r]
+        assert Yl.shape == (M, n1 - n0)
+        np.testing.assert_array_equal(Yl, ref[:, n0:n1])
+        np.testing.assert_array_equal(Yf, ref)
+        covered[n0:n1] = True
+    assert covered.all()

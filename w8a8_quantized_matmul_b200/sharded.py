@@ -53,3 +53,53 @@ def token_sharded_mixed_matmul(X_local, Wq, w_scale, W_fp16, threshold=6.0, grou
     bitmap = find(X_local, threshold)
     bitmaps = gather(bitmap, group)
     return apply(X_local, Wq, w_scale, W_fp16, bitmaps, Y, workspace)
+
+
+# ---------------------------------------------------------------------------
+# Column-sharded (out-feature) form. The outlier set is a function of X alone
+# (AIInfra "05Quantization01", LLM.int8() section: a feature dimension is an
+# outlier when some activation in it exceeds the threshold), so ranks that each
+# hold all of X and a contiguous block of the weight's output rows derive the
+# same set with no exchange; every output column depends only on its own weight
+# row. Each rank's Y is a column block of the whole Y; gathering the blocks is
+# needed only if a caller wants the full Y on every rank.
+# ---------------------------------------------------------------------------
+def column_block(N: int, rank: int, world: int):
+    """[n0, n1) of rank's output rows: contiguous blocks, multiples of 8 rows
+    where possible (keeps the weight slices' addresses 16-byte aligned)."""
+    per = (N + world - 1) // world
+    per = (per + 7) // 8 * 8
+    n0 = min(N, rank * per)
+    return n0, min(N, n0 + per)
+
+
+def _apply_cols_cuda(X, Wq_local, w_scale_local, W_local, threshold, Y=None, workspace=None):
+    return _ops.int8_mixed_matmul(X, Wq_local, w_scale_local, W_local, threshold, Y=Y,
+                                  workspace=workspace)[0]
+
+
+def _gather_cols(Y_local, N, group=None):
+    """The column blocks of all ranks as one [M, N] tensor (blocks in rank order)."""
+    world = dist.get_world_size(group)
+    per = (N + world - 1) // world
+    per = (per + 7) // 8 * 8
+    parts = [torch.empty((Y_local.shape[0], per), dtype=Y_local.dtype, device=Y_local.device)
+             for _ in range(world)]
+    pad = torch.zeros((Y_local.shape[0], per), dtype=Y_local.dtype, device=Y_local.device)
+    pad[:, :Y_local.shape[1]] = Y_local
+    dist.all_gather(parts, pad, group=group)
+    return torch.cat(parts, dim=1)[:, :N]
+
+
+def column_sharded_mixed_matmul(X, Wq_local, w_scale_local, W_local, threshold=6.0, group=None,
+                                N=None, gather=False, Y=None, workspace=None, *,
+                                apply=_apply_cols_cuda):
+    """This rank's column block of Y = X . W^T from its block of weight rows
+    (`column_block`); no collective unless gather=True, which returns the full
+    [M, N] Y on every rank (N is then required)."""
+    Y_local = apply(X, Wq_local, w_scale_local, W_local, threshold, Y, workspace)
+    if not gather:
+        return Y_local
+    if N is None:
+        raise ValueError("gather=True needs the full N")
+    return _gather_cols(Y_local, N, group)
