@@ -199,3 +199,20 @@ def test_int4_entry_points_validation(lib):
     assert lib.int4_rotated_matmul(A, A, A, 0, 256, 512, 128, A, None, 0, None) == _lib.I8MM_OK
     # self-test hook: a status pointer is required
     assert lib.int8_selftest_wait_timeout(None, None) == _lib.I8MM_ERR_INVALID_ARG
+
+
+def test_header_is_plain_c(tmp_path):
+    """include/int8mm.h compiles as C99 (pedantic) and as C++17 on its own."""
+    import shutil
+    import subprocess
+    if shutil.which("gcc") is None:
+        pytest.skip("no gcc")
+    src = tmp_path / "use_header.c"
+    src.write_text('#include "int8mm.h"\nint main(void) { return I8MM_OK; }\n')
+    inc = os.path.join(ROOT, "include")
+    for cmd in (["gcc", "-std=c99", "-Wall", "-Wextra", "-pedantic", "-Werror", "-I", inc, "-c",
+                 str(src), "-o", str(tmp_path / "a.o")],
+                ["g++", "-std=c++17", "-Wall", "-Wextra", "-Werror", "-I", inc, "-x", "c++", "-c",
+                 str(src), "-o", str(tmp_path / "b.o")]):
+        r = subprocess.run(cmd, capture_output=True, text=True)
+        assert r.returncode == 0, r.stderr
