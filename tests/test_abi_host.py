@@ -216,3 +216,21 @@ def test_header_is_plain_c(tmp_path):
                  str(src), "-o", str(tmp_path / "b.o")]):
         r = subprocess.run(cmd, capture_output=True, text=True)
         assert r.returncode == 0, r.stderr
+
+
+def test_plain_c_program_links_and_calls_the_library(lib, tmp_path):
+    """A C program (tests/c_consumer.c) links libint8mm.so through the header
+    and exercises the entry points that need no GPU."""
+    import shutil
+    import subprocess
+    if shutil.which("gcc") is None:
+        pytest.skip("no gcc")
+    libdir = os.path.dirname(_lib.LIB_PATH)
+    exe = tmp_path / "c_consumer"
+    r = subprocess.run(["gcc", "-std=c99", "-Wall", "-Werror", "-I", os.path.join(ROOT, "include"),
+                        os.path.join(ROOT, "tests", "c_consumer.c"), "-L", libdir, "-lint8mm",
+                        "-Wl,-rpath," + libdir, "-o", str(exe)], capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
+    r = subprocess.run([str(exe)], capture_output=True, text=True, timeout=60)
+    assert r.returncode == 0, r.stderr + r.stdout
+    assert "c consumer ok" in r.stdout
