@@ -9,7 +9,6 @@ from .llm_int8 import (  # noqa: F401
     find_outlier_cols,
     quantize_act_rows,
     int32_gemm,
-    int32_dot,
     dequantize,
     outlier_gemm,
     llm_int8_matmul,
@@ -17,6 +16,7 @@ from .llm_int8 import (  # noqa: F401
 )
 from .llm_int8 import (  # noqa: F401,E402
     mask_to_bitmap, find_topk_cols, quantize_act_rows_zp, weight_rowsum, dequantize_zp,
+    half_to_float, double_to_half, threads, set_threads, lib,
     ZP_QMIN, ZP_QMAX,
 )
 from .smoothquant import (  # noqa: F401,E402

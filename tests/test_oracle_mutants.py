@@ -1,9 +1,12 @@
 """Planted mistakes in a copy of the oracle must each fail a pin.
 
-Each mutant rewrites one line of a temporary copy of oracle/llm_int8.py
-(a dropped term, a wrong comparison, a wrong rounding mode, a transposed
-or reversed operand, a wrong sign) and runs tests/test_oracle_pins.py
-against it in a subprocess. Nothing here touches a GPU.
+Each mutant rewrites one line of a temporary copy of an oracle source (a
+dropped term, a wrong comparison, a wrong rounding mode, a transposed or
+reversed operand, a wrong sign, a missing check): the C++ oracle
+(oracle/llm_int8.cpp, rebuilt into a temporary library that the shim loads
+through LLM_INT8_ORACLE_LIB) or one of the numpy oracles of the other rows.
+The pins of the changed part then run in a subprocess and must fail. Nothing
+here touches a GPU.
 """
 import os
 import shutil
@@ -14,35 +17,71 @@ import pytest
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
-MUTANTS = {
-    "dequant_over_127_not_127sq": ("/ float(QMAX_INT8 * QMAX_INT8))\n\n\n#", "/ float(QMAX_INT8))\n\n\n#"),
-    "detect_ge_not_gt": ("np.abs(X32) > thr", "np.abs(X32) >= thr"),
-    "round_half_up": ("q = np.rint(quot)", "q = np.floor(quot + 0.5)"),
-    "gemm_reversed_k": ("C = A @ B.T", "C = A @ B[:, ::-1].T"),
-    "act_absmax_over_all_cols": ("normal = np.where(keep[None, :], np.abs(X32), np.float32(0))",
-                                 "normal = np.abs(X32)"),
-    "outlier_sign_flipped": ("return np.asarray(X, np.float64)[:, idx] @",
-                             "return -np.asarray(X, np.float64)[:, idx] @"),
-    "outlier_term_dropped": ("Y = (Cn + Co).astype(np.float16)", "Y = (Cn).astype(np.float16)"),
-    "w_scale_index_reversed": ("* np.asarray(w_scale, np.float64)[None, :] /",
-                               "* np.asarray(w_scale, np.float64)[::-1][None, :] /"),
-    "weight_absmax_per_tensor": ("aw = np.max(np.abs(W32), axis=1)",
-                                 "aw = np.max(np.abs(W32), axis=1) * 0 + np.max(np.abs(W32))"),
+# Each entry: (text in oracle/llm_int8.cpp, its planted replacement, pins file).
+CPP_MUTANTS = {
+    "dequant_over_127_not_127sq": ("static_cast<double>(ws[n]) / 16129.0;",
+                                   "static_cast<double>(ws[n]) / 127.0;", "test_oracle_pins.py"),
+    "detect_ge_not_gt": ("* K + j])) > threshold) out = true;",
+                         "* K + j])) >= threshold) out = true;", "test_oracle_pins.py"),
+    "round_half_up": ("const float q = std::rint(quot);", "const float q = std::floor(quot + 0.5f);",
+                      "test_oracle_pins.py"),
+    "gemm_reversed_k": ("s += static_cast<int32_t>(a[k]) * static_cast<int32_t>(b[k]);",
+                        "s += static_cast<int32_t>(a[k]) * static_cast<int32_t>(b[K - 1 - k]);",
+                        "test_oracle_pins.py"),
+    "act_absmax_over_all_cols": ("if (!mask[j]) a = std::max(a, std::fabs(half_to_float(x[j])));",
+                                 "a = std::max(a, std::fabs(half_to_float(x[j])));",
+                                 "test_oracle_pins.py"),
+    "outlier_sign_flipped": ("        s += half_to_double(X[i * K + idx[p]])",
+                             "        s -= half_to_double(X[i * K + idx[p]])", "test_oracle_pins.py"),
+    "outlier_term_dropped": ("Y[e] = double_to_half(Cn[e] + Co[e]);", "Y[e] = double_to_half(Cn[e]);",
+                             "test_oracle_pins.py"),
+    "w_scale_index_reversed": ("static_cast<double>(ws[n]) / 16129.0;",
+                               "static_cast<double>(ws[N - 1 - n]) / 16129.0;", "test_oracle_pins.py"),
+    "weight_absmax_over_half_the_row": (
+        "for (int k = 0; k < K; ++k) a = std::max(a, std::fabs(half_to_float(w[k])));",
+        "for (int k = 0; k < K / 2; ++k) a = std::max(a, std::fabs(half_to_float(w[k])));",
+        "test_oracle_pins.py"),
+    "half_decode_exponent_bias": ("static_cast<float>(1024 + f), e - 25);",
+                                  "static_cast<float>(1024 + f), e - 24);", "test_oracle_pins.py"),
+    "half_encode_ties_away": ("double q = std::nearbyint(std::ldexp(a, 10 - E));",
+                              "double q = std::round(std::ldexp(a, 10 - E));", "test_oracle_pins.py"),
+    "half_decode_subnormal_scale": ("v = std::ldexp(static_cast<float>(f), -24);",
+                                    "v = std::ldexp(static_cast<float>(f), -25);", "test_oracle_pins.py"),
+    "gemm_overflow_unchecked": ("if (s > INT32_MAX || s < INT32_MIN) bad[i] = 1;", "",
+                                "test_oracle_pins.py"),
+    "topk_ties_to_higher_index": ("[&](int p, int q) { return colmax[p] > colmax[q]; });",
+                                  "[&](int p, int q) { return colmax[p] > colmax[q] || "
+                                  "(colmax[p] == colmax[q] && p > q); });", "test_topk_pins.py"),
+    "topk_one_extra_column": ("for (int t = 0; t < k; ++t) mask[order[t]] = 1;",
+                              "for (int t = 0; t < k + 1 && t < K; ++t) mask[order[t]] = 1;",
+                              "test_topk_pins.py"),
+    "topk_by_mean_magnitude": ("colmax[j] = std::max(colmax[j], std::fabs(",
+                               "colmax[j] = colmax[j] + (std::fabs(", "test_topk_pins.py"),
+    "zp_zero_sign_flipped": ("-128.0f - std::rint(lq)", "-128.0f + std::rint(lq)",
+                             "test_zeropoint_pins.py"),
+    "zp_range_without_zero": ("float lo = 0.0f, hi = 0.0f;", "float lo = INFINITY, hi = 0.0f;",
+                              "test_zeropoint_pins.py"),
+    "zp_correction_dropped": ("static_cast<int64_t>(zero[i]) * static_cast<int64_t>(wsum[n]);",
+                              "0 * static_cast<int64_t>(wsum[n]);", "test_zeropoint_pins.py"),
+    "zp_step_over_127": ("const float step = range / 255.0f;", "const float step = range / 127.0f;",
+                         "test_zeropoint_pins.py"),
 }
 
 
-@pytest.mark.parametrize("name", sorted(MUTANTS))
-def test_pins_catch_planted_mistake(name, tmp_path):
-    src = open(os.path.join(ROOT, "oracle", "llm_int8.py")).read()
-    old, new = MUTANTS[name]
-    assert old in src, f"mutation site for {name} no longer exists"
-    for d in ("oracle", "synth", "tests"):
-        shutil.copytree(os.path.join(ROOT, d), tmp_path / d,
-                        ignore=shutil.ignore_patterns("__pycache__", "test_oracle_mutants.py"))
-    (tmp_path / "oracle" / "llm_int8.py").write_text(src.replace(old, new, 1))
+@pytest.mark.parametrize("name", sorted(CPP_MUTANTS))
+def test_pins_catch_planted_mistake_in_cpp_oracle(name, tmp_path):
+    sys.path.insert(0, ROOT)
+    from oracle import build as obuild
+    src = open(os.path.join(ROOT, "oracle", "llm_int8.cpp")).read()
+    old, new, pins = CPP_MUTANTS[name]
+    assert src.count(old) >= 1, f"mutation site for {name} no longer exists"
+    mutant = tmp_path / "llm_int8.cpp"
+    mutant.write_text(src.replace(old, new, 1))
+    so = obuild.build(str(mutant), str(tmp_path / "liborc_mutant.so"), force=True)
+    env = dict(os.environ, LLM_INT8_ORACLE_LIB=so)
     r = subprocess.run([sys.executable, "-m", "pytest", "-q", "-x", "-p", "no:cacheprovider",
-                        "tests/test_oracle_pins.py"], cwd=tmp_path, capture_output=True, text=True,
-                       timeout=300)
+                        os.path.join("tests", pins)], cwd=ROOT, env=env, capture_output=True,
+                       text=True, timeout=300)
     assert r.returncode != 0, f"mutant {name} survived the pins:\n{r.stdout[-2000:]}"
 
 
@@ -71,56 +110,6 @@ def test_smoothquant_pins_catch_planted_mistake(name, tmp_path):
     (tmp_path / "oracle" / "smoothquant.py").write_text(src.replace(old, new, 1))
     r = subprocess.run([sys.executable, "-m", "pytest", "-q", "-x", "-p", "no:cacheprovider",
                         "tests/test_smoothquant_pins.py"], cwd=tmp_path, capture_output=True,
-                       text=True, timeout=300)
-    assert r.returncode != 0, f"mutant {name} survived the pins:\n{r.stdout[-2000:]}"
-
-
-TOPK_MUTANTS = {
-    "topk_ties_to_higher_index": ("key=lambda j: (-float(colmax[j]), j))", "key=lambda j: (-float(colmax[j]), -j))"),
-    "topk_one_extra_column": ("mask[order[:k]] = True", "mask[order[:k + 1]] = True"),
-    "topk_by_mean_magnitude": ("colmax = np.max(np.abs(X32), axis=0) if X32.shape[0] else np.zeros(K, np.float32)\n    order",
-                               "colmax = np.mean(np.abs(X32), axis=0) if X32.shape[0] else np.zeros(K, np.float32)\n    order"),
-}
-
-
-@pytest.mark.parametrize("name", sorted(TOPK_MUTANTS))
-def test_topk_pins_catch_planted_mistake(name, tmp_path):
-    src = open(os.path.join(ROOT, "oracle", "llm_int8.py")).read()
-    old, new = TOPK_MUTANTS[name]
-    assert old in src, f"mutation site for {name} no longer exists"
-    for d in ("oracle", "synth", "tests"):
-        shutil.copytree(os.path.join(ROOT, d), tmp_path / d,
-                        ignore=shutil.ignore_patterns("__pycache__", "test_oracle_mutants.py"))
-    (tmp_path / "oracle" / "llm_int8.py").write_text(src.replace(old, new, 1))
-    r = subprocess.run([sys.executable, "-m", "pytest", "-q", "-x", "-p", "no:cacheprovider",
-                        "tests/test_topk_pins.py"], cwd=tmp_path, capture_output=True, text=True,
-                       timeout=300)
-    assert r.returncode != 0, f"mutant {name} survived the pins:\n{r.stdout[-2000:]}"
-
-
-ZP_MUTANTS = {
-    "zp_zero_sign_flipped": ("zero = np.where(live, np.clip(ZP_QMIN - np.rint((lo / safe).astype(np.float32)), ZP_QMIN, ZP_QMAX), 0)",
-                             "zero = np.where(live, np.clip(ZP_QMIN + np.rint((lo / safe).astype(np.float32)), ZP_QMIN, ZP_QMAX), 0)"),
-    "zp_range_without_zero": ("lo = np.minimum(np.min(kept, axis=1), np.float32(0))",
-                              "lo = np.min(np.where(keep[None, :], X32, np.float32(np.inf)), axis=1) + 0 * np.float32(0)"),
-    "zp_correction_dropped": ("Ccor = (np.asarray(C, np.int64) - np.asarray(zero, np.int64)[:, None]",
-                              "Ccor = (np.asarray(C, np.int64) - 0 * np.asarray(zero, np.int64)[:, None]"),
-    "zp_step_over_127": ("step = ((hi - lo).astype(np.float32) / np.float32(255)).astype(np.float32)",
-                         "step = ((hi - lo).astype(np.float32) / np.float32(127)).astype(np.float32)"),
-}
-
-
-@pytest.mark.parametrize("name", sorted(ZP_MUTANTS))
-def test_zeropoint_pins_catch_planted_mistake(name, tmp_path):
-    src = open(os.path.join(ROOT, "oracle", "llm_int8.py")).read()
-    old, new = ZP_MUTANTS[name]
-    assert old in src, f"mutation site for {name} no longer exists"
-    for d in ("oracle", "synth", "tests"):
-        shutil.copytree(os.path.join(ROOT, d), tmp_path / d,
-                        ignore=shutil.ignore_patterns("__pycache__", "test_oracle_mutants.py"))
-    (tmp_path / "oracle" / "llm_int8.py").write_text(src.replace(old, new, 1))
-    r = subprocess.run([sys.executable, "-m", "pytest", "-q", "-x", "-p", "no:cacheprovider",
-                        "tests/test_zeropoint_pins.py"], cwd=tmp_path, capture_output=True,
                        text=True, timeout=300)
     assert r.returncode != 0, f"mutant {name} survived the pins:\n{r.stdout[-2000:]}"
 

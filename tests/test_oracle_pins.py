@@ -338,3 +338,55 @@ def test_synthetic_outliers_detected_exactly():
         X, W, cols = synth.make_workload(w)
         _, _, count, idx = oracle.find_outlier_cols(X, w.threshold)
         assert idx.tolist() == cols.tolist() and count == w.n_outliers
+
+
+# --------------------------------------------------------------------------
+# The C++ oracle's plumbing: binary16 conversions against numpy's on every bit
+# pattern and every rounding tie, the int32 overflow check, thread counts
+# --------------------------------------------------------------------------
+def test_half_decode_every_bit_pattern():
+    h = np.arange(65536, dtype=np.uint32).astype(np.uint16).view(np.float16)
+    got = oracle.half_to_float(h)
+    ref = h.astype(np.float32)
+    nan = np.isnan(ref)
+    assert np.array_equal(np.isnan(got), nan)
+    # bit patterns, so that -0 and +0 are told apart
+    assert np.array_equal(got[~nan].view(np.uint32), ref[~nan].view(np.uint32))
+
+
+def test_half_encode_values_ties_and_overflow():
+    pos = np.arange(0, 0x7C00, dtype=np.uint32).astype(np.uint16).view(np.float16).astype(np.float64)
+    mids = (pos[:-1] + pos[1:]) / 2                  # exact ties between neighbours
+    nxt = np.nextafter(mids, np.inf)
+    prv = np.nextafter(mids, -np.inf)
+    rs = np.random.default_rng(0)
+    rnd = np.ldexp(rs.random(200000) + 0.5, rs.integers(-30, 18, 200000))
+    edge = np.array([65504.0, 65519.99, 65520.0, 65536.0, 1e300, 2.0 ** -24, 2.0 ** -25,
+                     np.nextafter(2.0 ** -25, 1), 2.0 ** -26, 0.0, np.inf])
+    d = np.concatenate([pos, mids, nxt, prv, rnd, edge])
+    d = np.concatenate([d, -d])
+    got = oracle.double_to_half(d).view(np.uint16)
+    ref = d.astype(np.float16).view(np.uint16)
+    assert np.array_equal(got, ref)
+    # ties go to the even significand
+    t = oracle.double_to_half(mids).view(np.uint16)
+    assert np.all(t % 2 == 0)
+
+
+def test_int32_gemm_refuses_overflow():
+    K = 133160                                       # 127^2 * K > 2^31 - 1
+    with pytest.raises(AssertionError):
+        oracle.int32_gemm(np.full((1, K), 127, np.int8), np.full((1, K), 127, np.int8))
+
+
+def test_results_do_not_depend_on_thread_count():
+    X, W, _ = synth.random_case(37, 256, 29, 5, seed=19)
+    try:
+        oracle.set_threads(1)
+        r1 = oracle.llm_int8_matmul(X, W, 6.0)
+        oracle.set_threads(7)
+        r7 = oracle.llm_int8_matmul(X, W, 6.0)
+    finally:
+        oracle.set_threads(0)
+    for key in ("Y", "mask", "idx", "Xq", "x_scale", "Wq", "w_scale", "C", "C_normal", "C_outlier"):
+        assert np.array_equal(r1[key], r7[key]), key

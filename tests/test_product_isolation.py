@@ -29,10 +29,23 @@ def test_package_does_not_use_the_oracle():
 def test_oracle_does_not_use_the_package():
     pat = re.compile(r"^\s*(import\s+w8a8_quantized_matmul_b200|from\s+w8a8_quantized_matmul_b200)",
                      re.M)
-    for path in _sources(os.path.join(ROOT, "oracle"), (".py",)):
+    for path in _sources(os.path.join(ROOT, "oracle"), (".py", ".cpp", ".h")):
         src = open(path, encoding="utf-8").read()
         assert not pat.search(src), f"{path} imports the CUDA package"
-        assert "ctypes" not in src and "libint8mm" not in src
+        assert "libint8mm" not in src and "int8mm.h" not in src and "csrc" not in src, path
+        assert "w8a8_quantized_matmul_b200" not in src, path
+
+
+def test_cpp_oracle_includes_only_the_standard_library():
+    """The C++ oracle is self-contained: standard headers only, no CUDA, no
+    header or source of the package."""
+    src = open(os.path.join(ROOT, "oracle", "llm_int8.cpp"), encoding="utf-8").read()
+    incs = re.findall(r"^\s*#\s*include\s*([<\"][^>\"]+[>\"])", src, re.M)
+    assert incs and all(i.startswith("<") for i in incs), incs
+    assert not any("cuda" in i for i in incs), incs
+    # the ctypes shim loads one library: the oracle's own build (oracle/build.py)
+    shim = open(os.path.join(ROOT, "oracle", "llm_int8.py"), encoding="utf-8").read()
+    assert shim.count("ctypes.CDLL(") == 1 and "_build.build()" in shim
 
 
 def test_synth_holds_no_method_arithmetic():
