@@ -385,11 +385,25 @@ int int8_device_status(const void* workspace, i8mm_stream_t stream);
  *            call's contents (each call clears the words it needs first).
  *            Calls that can overlap on the GPU (several streams or host
  *            threads) race on the array; the caller must serialise them.
+ *   Status:  a bounded device-side wait that gives up writes I8MM_ERR_TIMEOUT
+ *            into the array's status word (cleared by every call);
+ *            int8_noalloc_device_status reads it.
+ *   Errors:  those of int8_mixed_matmul; a device other than sm_100 returns
+ *            I8MM_ERR_UNSUPPORTED_DEVICE before the array is looked up.
  */
 #define I8MM_NOALLOC_SCRATCH_BYTES ((size_t)64 << 20)
 int int8_mixed_matmul_noalloc(const void* X, const int8_t* Wq, const float* w_scale,
                               const void* W_fp16, int M, int N, int K, float threshold,
                               void* Y, i8mm_stream_t stream);
+
+/*
+ * The device status word of the last int8_mixed_matmul_noalloc call on the
+ * current device (synchronises `stream`; reads 4 bytes into host memory, no
+ * allocation). Returns I8MM_OK, I8MM_ERR_TIMEOUT if a bounded device-side wait
+ * of that call gave up, I8MM_ERR_UNSUPPORTED_DEVICE on a device other than
+ * sm_100, or I8MM_ERR_CUDA.
+ */
+int int8_noalloc_device_status(i8mm_stream_t stream);
 
 /* Static string for a status code. */
 const char* int8_status_string(int status);

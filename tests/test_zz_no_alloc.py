@@ -1,19 +1,26 @@
 """int8_mixed_matmul_noalloc: the matmul for callers that cannot give the library
 device memory (for example code whose host framework owns every device
-allocation, or code that must not grow its memory use while running).
+allocation and hands it no allocator, or code that must not grow its memory use
+while running).
 
 The entry point keeps its scratch in a fixed device array inside the library.
-This test calls it through the C ABI twice in a row, on different inputs, and
-checks each result against the regular entry point (caller workspace) within
-the Y tolerance used by the other GPU tests. It also checks that a problem too
-large for the built-in array is refused. The file is named so that pytest
-collects it last.
+These tests call it through the C ABI twice in a row, on different inputs, at a
+prefill shape (few outliers: the product in the GEMM epilogue; many: the
+tensor-core outlier pass) and at a decode shape (16 tokens: the clustered decode
+kernel; with 6 outlier columns and with none). The same kernels run as for the
+regular entry point with a caller workspace, on the same inputs, so each result
+must equal that entry point's bit for bit (which is within the Y tolerance of
+the other GPU tests); the first result of each pair is also checked against the
+CPU oracle within that tolerance. After the calls the status word of the
+built-in array must read I8MM_OK. A problem too large for the array is refused.
+The file is named so that pytest collects it last.
 """
 import ctypes
 
 import numpy as np
 import pytest
 
+import oracle
 import synth
 
 torch = pytest.importorskip("torch")
@@ -41,17 +48,22 @@ def _close(y, ref):
     assert d.mean() <= MEAN_TOL * np.abs(ref).mean() + 1e-7
 
 
-def test_noalloc_twice_in_a_row_matches_workspace_path(lib):
+def _pair(lib, M, K, N, cases):
+    """Two back-to-back no-alloc calls compared with the workspace entry point."""
     from w8a8_quantized_matmul_b200 import _lib
-    M, K, N = 300, 1024, 520
-    X1, W, _ = synth.random_case(M, K, N, 6, seed=41)        # few outliers: epilogue path
-    X2, _, _ = synth.random_case(M, K, N, 40, seed=42)       # many: tensor-core outlier pass
+    Xs_h = []
+    W = None
+    for n_out, seed in cases:
+        X, Wc, _ = synth.random_case(M, K, N, n_out, seed=seed)
+        Xs_h.append(X)
+        W = Wc if W is None else W
     Wd = torch.from_numpy(W).cuda()
     Wq = torch.empty((N, K), dtype=torch.int8, device="cuda")
     ws = torch.empty((N,), dtype=torch.float32, device="cuda")
     stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
-    assert lib.int8_quantize_weight_rows(Wd.data_ptr(), N, K, Wq.data_ptr(), ws.data_ptr(), stream) == 0
-    Xs = [torch.from_numpy(X1).cuda(), torch.from_numpy(X2).cuda()]
+    assert lib.int8_quantize_weight_rows(Wd.data_ptr(), N, K, Wq.data_ptr(), ws.data_ptr(),
+                                         stream) == 0
+    Xs = [torch.from_numpy(X).cuda() for X in Xs_h]
 
     # Regular entry point, caller-provided workspace.
     need = lib.int8_mixed_matmul_workspace_size(M, N, K)
@@ -70,9 +82,24 @@ def test_noalloc_twice_in_a_row_matches_workspace_path(lib):
         st = lib.int8_mixed_matmul_noalloc(Xd.data_ptr(), Wq.data_ptr(), ws.data_ptr(),
                                            Wd.data_ptr(), M, N, K, 6.0, Y.data_ptr(), stream)
         assert st == _lib.I8MM_OK
+    assert lib.int8_noalloc_device_status(stream) == _lib.I8MM_OK
     torch.cuda.synchronize()
     for Y, R in zip(outs, refs):
+        assert torch.equal(Y, R)
         _close(Y.cpu().numpy(), R.cpu().numpy())
+    r = oracle.llm_int8_matmul(Xs_h[0], W, 6.0, Wq=Wq.cpu().numpy(), w_scale=ws.cpu().numpy(),
+                               intermediates=False)
+    _close(outs[0].cpu().numpy(), r["Y"])
+
+
+def test_noalloc_prefill_twice_in_a_row_matches_workspace_path(lib):
+    # 6 outlier columns: the product in the GEMM epilogue; 40: the tensor-core pass.
+    _pair(lib, 300, 1024, 520, [(6, 41), (40, 42)])
+
+
+def test_noalloc_decode_shape_twice_in_a_row_matches_workspace_path(lib):
+    # 16 tokens: the clustered decode kernel; 6 outlier columns, then none.
+    _pair(lib, 16, 4096, 520, [(6, 43), (0, 44)])
 
 
 def test_noalloc_refuses_problems_larger_than_its_array(lib):

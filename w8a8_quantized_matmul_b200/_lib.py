@@ -59,6 +59,7 @@ PROTOTYPES = {
     "int4_rotated_matmul": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _vp, _vp, _sz, _vp]),
     "int8_selftest_wait_timeout": (_i, [_vp, _vp]),
     "int8_device_status": (_i, [_vp, _vp]),
+    "int8_noalloc_device_status": (_i, [_vp]),
     "int8_status_string": (ctypes.c_char_p, [_i]),
     "int8_last_error_string": (ctypes.c_char_p, []),
 }

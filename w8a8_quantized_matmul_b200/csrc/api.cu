@@ -117,6 +117,11 @@ bool make_layout(int M, int N, int K, Layout* out) {
 
 }  // namespace
 
+namespace i8mm {
+int abi_check_device() { return check_device(); }
+int abi_cuda_fail(const char* what, cudaError_t e) { return cuda_fail(what, e); }
+}  // namespace i8mm
+
 extern "C" {
 
 const char* int8_last_error_string(void) { return g_last_error; }

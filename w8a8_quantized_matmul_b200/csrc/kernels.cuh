@@ -136,4 +136,10 @@ cudaError_t launch_topk_select(const float* colmax, int K, int k, uint32_t* bitm
                                cudaStream_t s);
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t s);
 
+// The C-ABI layer's device check (I8MM_OK or I8MM_ERR_UNSUPPORTED_DEVICE /
+// I8MM_ERR_CUDA) and its error recorder (the text int8_last_error_string
+// returns; I8MM_ERR_CUDA unless e is cudaSuccess), for the other ABI files.
+int abi_check_device();
+int abi_cuda_fail(const char* what, cudaError_t e);
+
 }  // namespace i8mm

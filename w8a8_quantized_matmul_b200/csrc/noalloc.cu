@@ -20,10 +20,14 @@
 #include <mutex>
 
 #include "int8mm.h"
+#include "kernels.cuh"
 
 namespace {
 
 constexpr size_t kNoAllocScratchBytes = size_t(64) << 20;
+// Offset of the status word in the scratch: the array is carved exactly like a
+// caller workspace, whose second int32 is the status word.
+constexpr size_t kStatusOffset = 4;
 
 // The scratch itself. In host code this name is only a stand-in for the device
 // object: its device address must be obtained with cudaGetSymbolAddress.
@@ -34,17 +38,27 @@ std::mutex g_setup_mutex;
 void* g_scratch_addr[kMaxDevices] = {};
 
 // Device address of the scratch on the current device, looked up once per
-// device (with that device current) and cached.
+// device (with that device current) and cached. The device is checked first:
+// on anything but sm_100 the module holding the array does not load, and the
+// lookup would fail with an unrelated CUDA error.
 int scratch_address(void** out) {
+  const int st = i8mm::abi_check_device();
+  if (st != I8MM_OK) return st;
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return I8MM_ERR_CUDA;
+  if (e != cudaSuccess) return i8mm::abi_cuda_fail("cudaGetDevice", e);
   if (dev < 0 || dev >= kMaxDevices) return I8MM_ERR_UNSUPPORTED_DEVICE;
   std::lock_guard<std::mutex> lock(g_setup_mutex);
   if (!g_scratch_addr[dev]) {
     void* p = nullptr;
     e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
-    if (e != cudaSuccess || !p) return I8MM_ERR_CUDA;
+    if (e != cudaSuccess || !p) {
+      // Record why, and clear the error so that the caller's next
+      // cudaGetLastError does not blame an unrelated launch for it.
+      (void)cudaGetLastError();
+      return i8mm::abi_cuda_fail("cudaGetSymbolAddress of the built-in scratch",
+                                 e != cudaSuccess ? e : cudaErrorInvalidSymbol);
+    }
     g_scratch_addr[dev] = p;
   }
   *out = g_scratch_addr[dev];
@@ -58,8 +72,8 @@ static_assert(kNoAllocScratchBytes == I8MM_NOALLOC_SCRATCH_BYTES, "header and ar
 extern "C" {
 
 int int8_mixed_matmul_noalloc(const void* X, const int8_t* Wq, const float* w_scale,
-                              const void* W_fp16, int M, int N, int K, float threshold, void* Y,
-                              i8mm_stream_t stream) {
+                              const void* W_fp16, int M, int N, int K, float threshold,
+                              void* Y, i8mm_stream_t stream) {
   if (M == 0 || N == 0) {
     // Same empty-problem rule as int8_mixed_matmul, without touching the device.
     return int8_mixed_matmul(X, Wq, w_scale, W_fp16, M, N, K, threshold, Y, nullptr, 0, stream);
@@ -73,10 +87,23 @@ int int8_mixed_matmul_noalloc(const void* X, const int8_t* Wq, const float* w_sc
   void* scratch = nullptr;
   const int st = scratch_address(&scratch);
   if (st != I8MM_OK) return st;
-  // The regular path clears the control words it needs at the start of every
-  // call, so the previous call's contents of the array do not matter.
+  // The regular path clears the control words it needs (count, status, barrier
+  // counter, bitmap) at the start of every call, so the previous call's
+  // contents of the array do not matter.
   return int8_mixed_matmul(X, Wq, w_scale, W_fp16, M, N, K, threshold, Y, scratch,
                            kNoAllocScratchBytes, stream);
+}
+
+int int8_noalloc_device_status(i8mm_stream_t stream) {
+  void* scratch = nullptr;
+  const int st = scratch_address(&scratch);
+  if (st != I8MM_OK) return st;
+  int32_t h = 0;
+  cudaError_t e = cudaMemcpyAsync(&h, static_cast<const uint8_t*>(scratch) + kStatusOffset, 4,
+                                  cudaMemcpyDeviceToHost, stream);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(stream);
+  if (e != cudaSuccess) return i8mm::abi_cuda_fail("status read", e);
+  return h == 0 ? I8MM_OK : (h == I8MM_ERR_TIMEOUT ? I8MM_ERR_TIMEOUT : I8MM_ERR_CUDA);
 }
 
 }  // extern "C"
