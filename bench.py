@@ -1,17 +1,22 @@
 """Benchmark of the LLM.int8() mixed-precision matmul on B200.
 
 One step = one int8_mixed_matmul call (outlier detection, per-token INT8
-quantisation with outlier compaction, tcgen05 INT8 GEMM + fp16 outlier GEMM
+quantisation with outlier compaction, tcgen05 INT8 GEMM + fp16 outlier product
 + dequantising epilogue) over one batch of synthetic activations, with the
 weight already quantised (int8_quantize_weight_rows runs once, untimed, as
-a deployed layer would).
+a deployed layer would). The default workload is the largest single-GPU
+configuration, the Llama-70B-like FFN prefill (4096 x 8192 . 28672 x 8192);
+the same line carries the OPT-6.7B prefill, the outlier-density stress shapes,
+the decode shape and the next rows as extra objects.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
 
-Multi-GPU (torchrun, one rank per GPU): the op does not shard across ranks
-here, so every rank runs an independent replica of the same workload; the
-timed region is bracketed by barriers, the time is the max over ranks and
-`value` counts the work of all ranks ("scaling": "weak").
+Multi-GPU (torchrun, one rank per GPU): by default (--dp sharded) each rank
+holds its own tokens of one batch of N*M tokens; the ranks all-gather their
+outlier bitmaps once per step so that every rank quantises against the same
+outlier set. --dp replicas runs independent full replicas instead. The timed
+region is bracketed by barriers, the time is the max over ranks and `value`
+counts the work of all ranks ("scaling": "weak").
 
 Prints one JSON line (rank 0).
 """
@@ -34,8 +39,11 @@ sys.path.insert(0, ROOT)
 import synth  # noqa: E402
 
 METRIC = "int8_mixed_matmul TOPS & % of B200 INT8 peak; decode-shape HBM GB/s"
-DEFAULT_WORKLOAD = "opt-6.7b-ffn-up-prefill"
+DEFAULT_WORKLOAD = "llama-70b-ffn-prefill"
+OPT_WORKLOAD = "opt-6.7b-ffn-up-prefill"
 DECODE_WORKLOAD = "decode"
+STRESS_WORKLOADS = ["stress-o0", "stress-o7", "stress-o64", "stress-o256", "stress-thr-inf",
+                    "stress-thr-0"]
 # Fallback denominators when MEASURED_PEAKS.json is absent (earlier pool measurement).
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 # Dense INT8 : dense BF16 tensor throughput on B200 (4.5 : 2.25 PFLOP/s nominal).
@@ -121,16 +129,7 @@ def oracle_sample_step(X, W, Wq, w_scale, threshold, rows):
     """The CPU oracle on a `rows`-token batch of the workload (detection over that batch)."""
     import oracle
     Xs = X[:rows]
-    return oracle.llm_int8_matmul(Xs, W, threshold, Wq=Wq, w_scale=w_scale)
-
-
-def oracle_threads():
-    try:
-        from threadpoolctl import threadpool_info
-        info = threadpool_info()
-        return max((i.get("num_threads", 1) for i in info), default=1)
-    except Exception:
-        return os.cpu_count() or 1
+    return oracle.llm_int8_matmul(Xs, W, threshold, Wq=Wq, w_scale=w_scale, intermediates=False)
 
 
 def time_oracle(w, X, W, Wq, w_scale, budget_s: float, max_rows: int | None = None):
@@ -279,17 +278,26 @@ def n_sets_for(w, l2_bytes):
 CC_MAX_OUTLIERS = 16   # up to this many outlier columns no fp16 panels are written
 
 # DRAM traffic per launch (dram__bytes_read.sum + dram__bytes_write.sum) from one
-# ncu capture of each kernel as it is now; the summaries and commands are in profiles/.
+# ncu capture of each kernel as it is now, keyed by kernel and workload; the
+# summaries and their commands are in profiles/. A kernel changed since its
+# capture has no entry (its traffic is reported as null).
 NCU_TRAFFIC = {
-    "gemm": {"bytes": 78.027008e6 + 34.86208e6,
-             "source": "profiles/gemm_i8_persistent_opt-6.7b-ffn-up-prefill.md"},
-    "quantize": {"bytes": 27.326976e6 + 1.792e3,
-                 "source": "profiles/detect_quantize_compact_opt-6.7b-ffn-up-prefill.md"},
-    "rotate": {"bytes": 16.804608e6,
-               "source": "profiles/rotate_rows_opt-6.7b-ffn-up-prefill.md"},
-    "decode": {"bytes": 19.596544e6,
-               "source": "profiles/decode_kernel_decode-16x4096x4096.md"},
+    ("gemm", "opt-6.7b-ffn-up-prefill"): {
+        "bytes": 78.027008e6 + 34.86208e6,
+        "source": "profiles/gemm_i8_persistent_opt-6.7b-ffn-up-prefill.md"},
+    ("quantize", "opt-6.7b-ffn-up-prefill"): {
+        "bytes": 27.326976e6 + 1.792e3,
+        "source": "profiles/detect_quantize_compact_opt-6.7b-ffn-up-prefill.md"},
+    ("rotate", "opt-6.7b-ffn-up-prefill"): {
+        "bytes": 16.804608e6, "source": "profiles/rotate_rows_opt-6.7b-ffn-up-prefill.md"},
+    ("decode", "decode"): {
+        "bytes": 19.596544e6, "source": "profiles/decode_kernel_decode-16x4096x4096.md"},
 }
+
+
+def traffic(kernel, workload):
+    e = NCU_TRAFFIC.get((kernel, workload))
+    return (e["bytes"], e["source"]) if e else (None, None)
 
 
 def quantize_stage_bytes(w, count):
@@ -301,6 +309,64 @@ def quantize_stage_bytes(w, count):
     return b
 
 
+def timed_loop(fn, n, stream):
+    """Average device time (ms) of n back-to-back calls fn(i), CUDA events on `stream`."""
+    import torch
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    a.record(stream)
+    for i in range(n):
+        fn(i)
+    b.record(stream)
+    torch.cuda.synchronize()
+    return a.elapsed_time(b) / n
+
+
+class Peaks:
+    def __init__(self):
+        self.d, self.kind = load_peaks()
+        self.bf16 = self.d.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+        self.bf16_sus = self.d.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
+        self.int8 = self.bf16 * INT8_OVER_BF16
+        self.int8_sus = self.bf16_sus * INT8_OVER_BF16
+        self.hbm = self.d.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
+
+
+def measure_prefill(w, args, stream, l2, pk, X=None, W=None, steps=None):
+    """One prefill workload: whole steps back to back, then each stage alone.
+
+    Returns the object the JSON line carries for it: ms per step and TOPS of the
+    whole call, and per stage (quantisation kernel against HBM, GEMM against the
+    dense INT8 peak, or the FP16 peak when every column is an outlier)."""
+    import w8a8_quantized_matmul_b200 as m
+    if X is None:
+        X, W, _ = synth.make_workload(w)
+    prob = Problem(w, X, W, n_sets_for(w, l2))
+    for i in range(max(3, args.warmup)):
+        prob.step(i)
+    n = steps or max(20, min(args.steps, 200))
+    ms = timed_loop(prob.step, n, stream)
+    count = int(m.workspace_views(prob.sets[0]["work"], w.M, w.N, w.K)["n_outliers"].item())
+    q_ms = prob.time_stage(1, n, stream)
+    g_ms = prob.time_stage(2, n, stream)
+    ops = 2.0 * w.M * w.N * w.K
+    fp16 = count == w.K
+    peak = pk.bf16 if fp16 else pk.int8
+    qb = quantize_stage_bytes(w, count)
+    gt = ops / (g_ms / 1e3) / 1e12
+    del prob
+    return {"workload": w.name, "M": w.M, "K": w.K, "N": w.N, "threshold": w.threshold,
+            "detected_outliers": count, "ms_per_step": ms,
+            "value": round(ops / (ms / 1e3) / 1e12, 2), "unit": "TOPS",
+            "frac_of_peak": round(ops / (ms / 1e3) / 1e12 / peak, 4),
+            "peak": ("fp16 dense = measured bf16 burst" if fp16 else "int8 dense = 2 x measured bf16 burst"),
+            "gemm": {"ms": g_ms, "achieved": round(gt, 2), "frac": round(gt / peak, 4)},
+            "quantize": {"ms": q_ms, "achieved_gbs": round(qb / (q_ms / 1e3) / 1e9, 1),
+                         "algorithmic_bytes": qb, "frac_of_hbm": round(qb / (q_ms / 1e3) / 1e9 / pk.hbm, 4)},
+            "calls_timed": n}
+
+
 def run_ours(args, ws, rank, local):
     import torch
     import w8a8_quantized_matmul_b200 as m
@@ -309,7 +375,7 @@ def run_ours(args, ws, rank, local):
         _b.build()
     barrier(ws)
     m.load()
-    peaks, peaks_kind = load_peaks()
+    pk = Peaks()
     props = torch.cuda.get_device_properties(torch.cuda.current_device())
     l2 = getattr(props, "L2_cache_size", 126 * 2 ** 20) or 126 * 2 ** 20
 
@@ -352,19 +418,26 @@ def run_ours(args, ws, rank, local):
     ms_max = max_over_ranks(ms, ws)
 
     # ---- per-kernel times: each stage launched back to back on the same stream
-    # (stage 1 = control-word memset + detection/quantisation kernel, stage 2 = GEMM),
-    # over the same rotating buffer sets, bracketed by CUDA events.
+    # (stage 1 = detection/quantisation kernel, stage 2 = GEMM), over the same
+    # rotating buffer sets, bracketed by CUDA events.
     n_stage = max(20, min(args.steps, 500))
     q_ms = prob.time_stage(1, n_stage, stream)
     g_ms = prob.time_stage(2, n_stage, stream)
     ops_per_step = 2.0 * w.M * w.N * w.K
     value = ops_per_step * args.steps * ws / (ms_max / 1e3) / 1e12
-    bf16 = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
-    int8_peak = bf16 * INT8_OVER_BF16
-    hbm = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
     gemm_tops = ops_per_step / (g_ms / 1e3) / 1e12
     qbytes = quantize_stage_bytes(w, count)
     q_gbs = qbytes / (q_ms / 1e3) / 1e9
+
+    # ---- the GEMM stage sustained: back to back for a few seconds under the
+    # power cap, against the sustained peak, with its own clock record
+    sus_n = max(20, int(args.sustain_s * 1e3 / max(g_ms, 1e-3)))
+    sclk = ClockSampler(local)
+    sclk.start()
+    time.sleep(0.2)
+    g_sus_ms = prob.time_stage(2, sus_n, stream)
+    sus_clk = sclk.stop()
+    sus_tops = ops_per_step / (g_sus_ms / 1e3) / 1e12
 
     # ---- end to end through the public API with host buffers
     e2e_steps = min(args.steps, 200)
@@ -388,17 +461,11 @@ def run_ours(args, ws, rank, local):
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), ws)
     e2e_value = ops_per_step * e2e_steps * ws / (e2e_ms / 1e3) / 1e12
+    del prob, Xh, Yh
+    torch.cuda.empty_cache()
 
-    # ---- decode-shape line (weight-read bound), same process, rank-local
-    decode = None
-    if args.workload != DECODE_WORKLOAD and not args.no_decode:
-        decode = bench_decode(args, stream, l2, hbm)
-    smooth = None
-    if args.workload == DEFAULT_WORKLOAD and not args.no_decode:
-        smooth = bench_smoothquant(args, stream, l2,
-                                   peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
-                                   * INT8_OVER_BF16, hbm)
-
+    g_traffic, g_src = traffic("gemm", w.name)
+    q_traffic, q_src = traffic("quantize", w.name)
     result = {
         "metric": METRIC,
         "value": round(value, 3),
@@ -417,27 +484,30 @@ def run_ours(args, ws, rank, local):
                    "parallelism": (f"token-sharded dp{ws}: {ws}x{w.M} tokens per step, one "
                                    "all-gather of the ceil(K/32)-word outlier bitmaps" if sharded
                                    else f"replicas x{ws}"),
-                   "l2": f"rotating {n_sets} buffer sets of {prob.bytes_touched() / 1e6:.0f} MB "
+                   "l2": f"rotating {n_sets} buffer sets of {prob_bytes(w) / 1e6:.0f} MB "
                          f"touched per step (> 2x L2 of {l2 / 1e6:.0f} MB)"},
         "roofline": {"kernel": "gemm_i8_persistent_kernel (tcgen05 kind::i8, fp16 outlier epilogue)",
                      "bound": "tensor", "achieved": round(gemm_tops, 2),
-                     "peak": round(int8_peak, 1), "unit": "TOPS",
-                     "frac": round(gemm_tops / int8_peak, 4),
-                     "traffic": (NCU_TRAFFIC["gemm"]["bytes"]
-                                 if w.name == DEFAULT_WORKLOAD else None),
-                     "traffic_source": NCU_TRAFFIC["gemm"]["source"],
-                     "peak_note": f"{peaks_kind} bf16 burst {bf16} TFLOP/s x {INT8_OVER_BF16} "
+                     "peak": round(pk.int8, 1), "unit": "TOPS",
+                     "frac": round(gemm_tops / pk.int8, 4),
+                     "traffic": g_traffic, "traffic_source": g_src,
+                     "peak_note": f"{pk.kind} bf16 burst {pk.bf16} TFLOP/s x {INT8_OVER_BF16} "
                                   "(dense int8 : bf16 nominal ratio)",
                      "gemm_ms": g_ms,
-                     "timing": f"{n_stage} back-to-back launches of the GEMM stage, CUDA events"},
-        "roofline_quantize": {"kernel": "detect_quantize_compact_kernel (cooperative) + memset",
-                              "bound": "hbm", "achieved": round(q_gbs, 1), "peak": hbm,
-                              "unit": "GB/s", "frac": round(q_gbs / hbm, 4),
+                     "timing": f"{n_stage} back-to-back launches of the GEMM stage, CUDA events",
+                     "sustained": {"achieved": round(sus_tops, 2), "peak": round(pk.int8_sus, 1),
+                                   "frac_sustained": round(sus_tops / pk.int8_sus, 4),
+                                   "gemm_ms": g_sus_ms, "launches": sus_n,
+                                   "seconds": round(g_sus_ms * sus_n / 1e3, 2),
+                                   "peak_note": f"{pk.kind} bf16 sustained {pk.bf16_sus} TFLOP/s x "
+                                                f"{INT8_OVER_BF16}",
+                                   "clocks": sus_clk}},
+        "roofline_quantize": {"kernel": "detect_quantize_compact_kernel (cooperative)",
+                              "bound": "hbm", "achieved": round(q_gbs, 1), "peak": pk.hbm,
+                              "unit": "GB/s", "frac": round(q_gbs / pk.hbm, 4),
                               "algorithmic_bytes": qbytes, "stage_ms": q_ms,
-                              "traffic": (NCU_TRAFFIC["quantize"]["bytes"]
-                                          if w.name == DEFAULT_WORKLOAD else None),
-                              "traffic_source": NCU_TRAFFIC["quantize"]["source"],
-                              "peak_note": f"{peaks_kind} hbm_gbs"},
+                              "traffic": q_traffic, "traffic_source": q_src,
+                              "peak_note": f"{pk.kind} hbm_gbs"},
         "e2e": {"value": round(e2e_value, 3), "unit": "TOPS", "steps": e2e_steps,
                 "h2d_bytes_per_step": 2 * w.M * w.K, "d2h_bytes_per_step": 2 * w.M * w.N},
         "gpu_launches": (3 if sharded else 2) * args.steps,
@@ -448,27 +518,46 @@ def run_ours(args, ws, rank, local):
                               "(plus one cudaMemsetAsync of the control words)"),
         "clocks": clk,
     }
-    if decode is not None:
-        result["decode"] = decode
-    if smooth is not None:
-        result["smoothquant"] = smooth
-    if args.workload == DEFAULT_WORKLOAD and not args.no_decode:
-        i8p = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]) * INT8_OVER_BF16
-        result["topk"] = [bench_topk(args, stream, l2, i8p, f) for f in (0.01, 0.02)]
-        result["zeropoint"] = bench_zeropoint(args, stream, l2, i8p)
-        hbm_peak = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
-        result["rotation"] = bench_rotation(args, stream, l2, i8p, hbm_peak)
-        result["rotation_w4a4"] = bench_w4a4(args, stream, l2, i8p)
+    extras = w.name == DEFAULT_WORKLOAD and not args.no_extras and not sharded
+    if extras:
+        result["opt"] = measure_prefill(synth.WORKLOADS[OPT_WORKLOAD], args, stream, l2, pk)
+        result["stress"] = [measure_prefill(synth.WORKLOADS[n], args, stream, l2, pk)
+                            for n in STRESS_WORKLOADS]
+    if w.name != DECODE_WORKLOAD and not args.no_extras:
+        result["decode"] = bench_decode(args, stream, l2, pk.hbm)
+    if extras:
+        result["smoothquant"] = bench_smoothquant(args, stream, l2, pk.int8, pk.hbm)
+        result["topk"] = [bench_topk(args, stream, l2, pk.int8, f) for f in (0.01, 0.02)]
+        result["zeropoint"] = bench_zeropoint(args, stream, l2, pk.int8)
+        result["rotation"] = bench_rotation(args, stream, l2, pk.int8, pk.hbm)
+        result["rotation_w4a4"] = bench_w4a4(args, stream, l2, pk.int8)
     if rank == 0 and not args.no_cpu_baseline:
         import oracle
         Wq_o, ws_o = oracle.quantize_weight_rows(W)
         tops, rows, t, n = time_oracle(w, X, W, Wq_o, ws_o, budget_s=args.cpu_budget)
         result["cpu_baseline"] = {"value": round(tops, 6), "unit": "TOPS",
-                                  "cores": oracle_threads(), "kind": "oracle",
+                                  "cores": oracle.threads(), "kind": "oracle",
+                                  "oracle": "C++17 (oracle/llm_int8.cpp), std::thread over rows",
+                                  "cpu": cpu_model(),
                                   "sample": f"{rows} of {w.M} tokens of the same workload "
                                             f"(detection over those tokens), {t:.2f} s per "
                                             f"sample, mean of {n}"}
     return result
+
+
+def prob_bytes(w):
+    return 2 * w.M * w.K + w.M * w.K + w.N * w.K + 2 * w.M * w.N
+
+
+def cpu_model():
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return None
 
 
 def bench_decode(args, stream, l2, hbm):
@@ -522,8 +611,8 @@ def bench_decode(args, stream, l2, hbm):
     gbs = nbytes / (ms / 1e3) / 1e9
     return {"workload": w.name, "M": w.M, "K": w.K, "N": w.N, "us_per_call": round(ms * 1e3, 2),
             "value": round(gbs, 1), "unit": "GB/s", "frac_of_hbm": round(gbs / hbm, 4),
-            "algorithmic_bytes": nbytes, "traffic": NCU_TRAFFIC["decode"]["bytes"],
-            "traffic_source": NCU_TRAFFIC["decode"]["source"], "rotating_sets": n_sets,
+            "algorithmic_bytes": nbytes, "traffic": traffic("decode", w.name)[0],
+            "traffic_source": traffic("decode", w.name)[1], "rotating_sets": n_sets,
             "calls_timed": replays * per_graph, "timing": "cuda-graph replay",
             "eager_us_per_call": round(eager_ms * 1e3, 2)}
 
@@ -534,7 +623,7 @@ def bench_smoothquant(args, stream, l2, int8_peak, hbm):
     INT8 GEMM) timed back to back over rotating buffers."""
     import torch
     import w8a8_quantized_matmul_b200 as m
-    w = synth.WORKLOADS[DEFAULT_WORKLOAD]
+    w = synth.WORKLOADS[OPT_WORKLOAD]
     X, W, _ = synth.make_workload(w)
     Xd = torch.from_numpy(X).cuda()
     Wd = torch.from_numpy(W).cuda()
@@ -579,7 +668,7 @@ def bench_topk(args, stream, l2, int8_peak, fraction):
     columns of largest max |x| in FP16, timed back to back over rotating buffers."""
     import torch
     import w8a8_quantized_matmul_b200 as m
-    w = synth.WORKLOADS[DEFAULT_WORKLOAD]
+    w = synth.WORKLOADS[OPT_WORKLOAD]
     X, W, _ = synth.make_workload(w)
     Xd = torch.from_numpy(X).cuda()
     Wd = torch.from_numpy(W).cuda()
@@ -624,7 +713,7 @@ def bench_zeropoint(args, stream, l2, int8_peak):
     back to back over rotating buffers (weight row sums computed once, offline)."""
     import torch
     import w8a8_quantized_matmul_b200 as m
-    w = synth.WORKLOADS[DEFAULT_WORKLOAD]
+    w = synth.WORKLOADS[OPT_WORKLOAD]
     X, W, _ = synth.make_workload(w)
     Xd = torch.from_numpy(X).cuda()
     Wd = torch.from_numpy(W).cuda()
@@ -671,7 +760,7 @@ def bench_rotation(args, stream, l2, int8_peak, hbm, G=128):
     buffers; the rotation kernel is also timed alone (its HBM roofline)."""
     import torch
     import w8a8_quantized_matmul_b200 as m
-    w = synth.WORKLOADS[DEFAULT_WORKLOAD]
+    w = synth.WORKLOADS[OPT_WORKLOAD]
     X, W, _ = synth.make_workload(w)
     Xd = torch.from_numpy(X).cuda()
     Wd = torch.from_numpy(W).cuda()
@@ -721,8 +810,8 @@ def bench_rotation(args, stream, l2, int8_peak, hbm, G=128):
                               "peak": hbm, "frac": round(r_gbs / hbm, 4),
                               "algorithmic_bytes": rbytes,
                               "bytes_note": "X fp16 read + codes written + scales",
-                              "traffic": (NCU_TRAFFIC["rotate"]["bytes"] if G == 128 else None),
-                              "traffic_source": NCU_TRAFFIC["rotate"]["source"]}}
+                              "traffic": (traffic("rotate", w.name)[0] if G == 128 else None),
+                              "traffic_source": traffic("rotate", w.name)[1]}}
 
 
 def bench_w4a4(args, stream, l2, int8_peak, G=128):
@@ -732,7 +821,7 @@ def bench_w4a4(args, stream, l2, int8_peak, G=128):
     group-scaled tensor-core GEMM) timed back to back over rotating buffers."""
     import torch
     import w8a8_quantized_matmul_b200 as m
-    w = synth.WORKLOADS[DEFAULT_WORKLOAD]
+    w = synth.WORKLOADS[OPT_WORKLOAD]
     X, W, _ = synth.make_workload(w)
     Xd = torch.from_numpy(X).cuda()
     Wd = torch.from_numpy(W).cuda()
@@ -780,7 +869,7 @@ def run_reference(args, ws, rank):
     X, W, _ = synth.make_workload(w)
     Wq, w_scale = oracle.quantize_weight_rows(W)
     total = args.steps + args.warmup
-    per_step_budget = max(0.02, 120.0 / max(total, 1))
+    per_step_budget = max(0.02, args.ref_budget / max(total, 1))
     rows = min(w.M, 16)
     t0 = time.perf_counter()
     oracle_sample_step(X, W, Wq, w_scale, w.threshold, rows)
@@ -793,7 +882,7 @@ def run_reference(args, ws, rank):
         oracle_sample_step(X, W, Wq, w_scale, w.threshold, rows)
     t = time.perf_counter() - t0
     tops = 2.0 * rows * w.N * w.K * args.steps / t / 1e12
-    cores = oracle_threads()
+    cores = oracle.threads()
     sample = f"{rows} of {w.M} tokens per step (detection over those tokens)"
     return {
         "impl": "reference", "metric": METRIC, "value": round(tops, 6), "unit": "TOPS",
@@ -802,7 +891,8 @@ def run_reference(args, ws, rank):
         "vs_baseline": None, "dtype": "int8", "data": "synthetic",
         "config": {"workload": w.name, "M": w.M, "K": w.K, "N": w.N, "threshold": w.threshold},
         "cpu_baseline": {"value": round(tops, 6), "unit": "TOPS", "cores": cores,
-                         "kind": "oracle", "sample": sample},
+                         "kind": "oracle", "oracle": "C++17 (oracle/llm_int8.cpp), std::thread over rows",
+                         "cpu": cpu_model(), "sample": sample},
         "e2e": {"value": round(tops, 6), "unit": "TOPS", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
@@ -818,7 +908,12 @@ def main():
     ap.add_argument("--cpu-budget", type=float, default=15.0,
                     help="seconds of oracle work for the cpu_baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--ref-budget", type=float, default=120.0,
+                    help="seconds of oracle work in all steps of --impl reference together")
+    ap.add_argument("--no-extras", action="store_true",
+                    help="only the chosen workload (no OPT, stress, decode and next-row objects)")
+    ap.add_argument("--sustain-s", type=float, default=2.5,
+                    help="seconds of back-to-back GEMM launches for the sustained figure")
     ap.add_argument("--dp", default="sharded", choices=["sharded", "replicas"],
                     help="with several ranks: split the tokens of one batch over the ranks "
                          "(one all-gather of the outlier bitmaps per step) or run full replicas")

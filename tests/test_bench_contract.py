@@ -18,7 +18,8 @@ KEYS = {"impl", "metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_
 
 def test_reference_arm_prints_one_json_line():
     r = subprocess.run([sys.executable, "bench.py", "--impl", "reference", "--steps", "1",
-                        "--warmup", "3"], cwd=ROOT, capture_output=True, text=True, timeout=600)
+                        "--warmup", "3", "--ref-budget", "4"], cwd=ROOT, capture_output=True,
+                       text=True, timeout=600)
     assert r.returncode == 0, r.stderr[-2000:]
     lines = [x for x in r.stdout.splitlines() if x.startswith("{")]
     assert len(lines) == 1
@@ -26,9 +27,10 @@ def test_reference_arm_prints_one_json_line():
     assert KEYS <= set(d)
     assert d["impl"] == "reference" and d["value"] > 0 and d["steps"] == 1 and d["warmup"] == 3
     assert d["higher_is_better"] is True and d["scaling"] == "weak"
-    assert d["config"]["workload"] == "opt-6.7b-ffn-up-prefill"
+    assert d["config"]["workload"] == "llama-70b-ffn-prefill"
     cb = d["cpu_baseline"]
     assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["value"] == d["value"]
+    assert "C++" in cb["oracle"]
     assert cb["unit"] == d["unit"] and "tokens" in cb["sample"]
     e = d["e2e"]
     assert e["value"] == d["value"] and e["unit"] == d["unit"]

@@ -212,12 +212,15 @@ DECODE_CASES = [
     (12, 4096, 1000, 0, 6.0),
     (16, 4096, 256, 64, 6.0),      # more outliers per CTA than are gathered ahead
     (5, 1040, 136, 3, 6.0),        # two ranks, the last K-block 16 columns wide
+    (8, 12288, 256, 5, 6.0),       # K > 8192: too long for one cluster, the prefill kernels run
+    (16, 16384, 136, 7, 6.0),      # the same, 16 tokens, ragged N
 ]
 
 
 @pytest.mark.parametrize("case", DECODE_CASES, ids=[f"M{c[0]}-K{c[1]}-N{c[2]}-o{c[3]}-t{c[4]}" for c in DECODE_CASES])
 def test_decode_path_parity(case):
-    """Shapes of at most 16 tokens go through the clustered decode kernel."""
+    """Shapes of at most 16 tokens go through the clustered decode kernel (K <= 8192)
+    or, for longer rows, through the prefill kernels."""
     M, K, N, n_out, thr = case
     X, W, _ = synth.random_case(M, K, N, n_out, seed=M * 1000 + K + N)
     if M > 2:

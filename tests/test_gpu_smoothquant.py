@@ -81,6 +81,37 @@ def test_matmul_parity(case):
     _y_close(Y.cpu().numpy(), ref["Y"])
 
 
+@pytest.mark.parametrize("alpha", [0.5, 0.85])
+def test_all_gpu_pipeline_parity(alpha):
+    """The pipeline the benchmark times, all on the GPU (calibration maxima, fp32
+    factors, smoothed weight, runtime call), element by element against the
+    oracle fed the GPU's factors: the factors themselves are fp32 powers that
+    match the oracle's within 4e-7 relative, so the oracle takes them as input
+    and everything after them is compared bit for bit (codes, scales) or within
+    the Y tolerance."""
+    M, K, N = 384, 2048, 520
+    X, W, _ = synth.random_case(M, K, N, 6, seed=91)
+    Xd, Wd = torch.from_numpy(X).cuda(), torch.from_numpy(W).cuda()
+    act = m.int8_column_absmax(Xd)
+    wmax = m.int8_column_absmax(Wd)
+    s, r = m.int8_smoothquant_factors(act, wmax, alpha)
+    Wq, ws = m.int8_smoothquant_weight_rows(Wd, s)
+    Y, work = m.int8_smoothquant_matmul(Xd, Wq, ws, r)
+    torch.cuda.synchronize()
+    s_gpu, r_gpu = s.cpu().numpy(), r.cpu().numpy()
+    np.testing.assert_array_equal(act.cpu().numpy(), oracle.column_absmax(X))
+    np.testing.assert_array_equal(r_gpu, oracle.smooth_rcp(s_gpu))
+    Wq_ref, ws_ref, _ = oracle.smooth_weight_rows(W, s_gpu)
+    np.testing.assert_array_equal(Wq.cpu().numpy(), Wq_ref)
+    np.testing.assert_array_equal(ws.cpu().numpy(), ws_ref)
+    ref = oracle.smoothquant_matmul(X, Wq_ref, ws_ref, r_gpu)
+    v = m.smoothquant_workspace_views(work, M, K)
+    assert int(v["status"].item()) == 0
+    np.testing.assert_array_equal(v["x_scale"].cpu().numpy(), ref["x_scale"])
+    np.testing.assert_array_equal(v["Xq"].cpu().numpy(), ref["Xq"])
+    _y_close(Y.cpu().numpy(), ref["Y"])
+
+
 def test_all_gpu_pipeline_beats_plain_int8():
     """Calibrate, smooth and run entirely on the GPU; the smoothed W8A8 output is
     closer to the exact product than the unsmoothed one (section 4.5's claim)."""

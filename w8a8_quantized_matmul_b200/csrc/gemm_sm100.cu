@@ -8,9 +8,12 @@
 // INT8 matmul accumulated in INT32, dequantisation by the outer product of the
 // row and column scales, FP16 matmul over the outlier dimensions, final sum.
 //
-// Persistent kernel, one CTA per SM, 128 x 256 output tiles walked with stride
-// gridDim.x (M-tile index fastest, so the CTAs in flight share Wq column blocks
-// and all of Xq through L2). Warp roles:
+// Persistent kernel, one CTA per SM, output tiles walked with stride over the
+// grid (M-tile index fastest, so the CTAs in flight share Wq column blocks and
+// all of Xq through L2). With more than 128 rows the CTAs run as pairs (2-CTA
+// clusters, tcgen05 cta_group::2) on 256 x 256 tiles, each CTA staging its 128
+// rows of Xq and 128 of the 256 rows of Wq; otherwise one CTA takes a 128 x 256
+// tile. Warp roles:
 //   warp 0      TMA producer: 128-byte-swizzled K-blocks (128 int8 columns of
 //               Xq and Wq) into a STAGES-deep shared-memory ring that runs
 //               continuously across tiles
@@ -30,7 +33,8 @@
 //                    multiplied with kind::f16 into an FP32 accumulator in the
 //                    other half of TMEM (single-buffered).
 // The outlier count is read from device memory, so the host never syncs.
-// No clusters and no TMA multicast are used. Every mbarrier wait is bounded;
+// No TMA load uses cluster multicast: both CTAs of a pair load their own halves,
+// completing on the even CTA's barrier. Every mbarrier wait is bounded;
 // a wait that gives up records I8MM_ERR_TIMEOUT in the status word and the
 // CTA stops issuing work.
 #include <cuda.h>

@@ -9,9 +9,14 @@
 // The kernels form the correctly rounded quotient without a division: with
 // n = x*127 (exact), ra = fl(1/a) (one correctly rounded reciprocal per group),
 // q = fl(n*ra), r = fma(q, -a, n) and q' = fma(r, ra, q), q' equals fl(n/a)
-// for every pair of fp16 values x, a with |x| <= a (the one-step FMA
-// correction of a reciprocal-based quotient). This was checked for all such
-// pairs exhaustively; the check ships with the tests. The integer code of q'
+// for every pair of fp16 values x, a with |x| <= a. This is Markstein's
+// correction step for division with a fused multiply-add (P. Markstein,
+// "Computation of elementary functions on the IBM RISC System/6000 processor",
+// IBM J. Res. Dev. 34(1), 1990; also "IA-64 and Elementary Functions", 2000):
+// the exact remainder r = n - q*a comes from one FMA, and one more FMA adds
+// its scaled value to the first quotient. Markstein's theorem needs a
+// correctly rounded reciprocal; here the result was also checked for all such
+// fp16 pairs exhaustively, and the check ships with the tests. The integer code of q'
 // (|q'| <= 127) is then the low byte of fl(q' + 1.5*2^23), which rounds half
 // to even. Entries of outlier columns may exceed a; their codes are discarded.
 #pragma once
