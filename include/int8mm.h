@@ -106,11 +106,11 @@ size_t int8_mixed_matmul_workspace_size(int M, int N, int K);
  * (byte offsets from the workspace base; each at least 16-byte aligned). Lets a
  * caller or a test read the outlier set, codes and scales of the last call.
  * The outlier panels have row stride panel_ld elements (fp16) and hold the
- * compacted outlier columns in ascending column order, zero-padded to 16
- * columns when there are 1..16 outliers (the GEMM epilogue then adds the
- * outlier product on CUDA cores) or to a multiple of 64 when there are more
- * (the GEMM multiplies them on the tensor cores). Nothing is written when
- * there are no outliers.
+ * compacted outlier columns in ascending column order, zero-padded to a
+ * multiple of 64 columns; they are written only when there are more than 16
+ * outlier columns (the GEMM multiplies them on the tensor cores). With 1..16
+ * the GEMM epilogue reads the outlier values of X and W through col_idx and
+ * adds the product on CUDA cores, and the panels are not written.
  */
 typedef struct {
   size_t n_outliers;   /* int32 [1] */

@@ -1,7 +1,8 @@
 """GPU parity: the CUDA path (through the C ABI) against the CPU oracle.
 
 Integer and byte outputs (outlier bitmap, count, ascending column list,
-INT8 codes, absmax scales, INT32 accumulators, compacted panels) must match
+INT8 codes, absmax scales, INT32 accumulators, compacted panels when there are
+more than 16 outlier columns) must match
 bit for bit. The fp16 Y must satisfy, against the oracle's Y,
     max|dY| <= 1e-2 * max|Y_ref|   and   mean|dY| <= 1e-3 * mean|Y_ref|.
 Both sides take every integer decision (|x| > threshold, rint of the fp32
@@ -76,15 +77,16 @@ def check_intermediates(ref, got, K):
     assert np.array_equal(got["x_scale"].view(np.uint32), ref["x_scale"].view(np.uint32))
 
 
-CC_MAX_OUTLIERS = 16   # up to this many outlier columns the panels are 16 wide
+CC_MAX_OUTLIERS = 16   # up to this many outlier columns the GEMM reads X and W itself
 
 
 def check_panels(X, W, ref, got):
-    """Compacted fp16 outlier panels: 16 columns wide for 1..16 outliers, else 64-padded."""
+    """Compacted fp16 outlier panels, 64-padded: written only when there are more
+    than 16 outlier columns (the tensor-core outlier product)."""
     count = ref["count"]
-    if count == 0 or X.shape[0] <= 16:   # the decode path (<= 16 tokens) writes no panels
+    if count <= CC_MAX_OUTLIERS or X.shape[0] <= 16:   # no panels (or the decode path)
         return
-    pad = CC_MAX_OUTLIERS if count <= CC_MAX_OUTLIERS else (count + 63) // 64 * 64
+    pad = (count + 63) // 64 * 64
     idx = ref["idx"]
     assert np.array_equal(got["X_O"][:, :count], X[:, idx])
     assert np.all(got["X_O"][:, count:pad] == 0)
@@ -229,6 +231,37 @@ def test_decode_path_parity(case):
     ref = oracle.llm_int8_matmul(X, W, thr)
     check_intermediates(ref, got, K)
     assert_y_close(Y, ref["Y"], f"decode {case}")
+
+
+RECHECK_CASES = [
+    # M, K, N: the first has more rows per CTA than the kernel's row slots
+    (4096, 8192, 256),
+    (2048, 4096, 520),
+    (300, 1040, 136),
+    (37, 4096, 64),
+]
+
+
+@pytest.mark.parametrize("case", RECHECK_CASES, ids=[f"M{c[0]}-K{c[1]}-N{c[2]}" for c in RECHECK_CASES])
+def test_outliers_on_few_tokens_force_the_recheck(case):
+    """The fused kernel quantises each CTA's rows against the CTA's own outlier
+    columns and checks them against the whole batch's afterwards. Outlier columns
+    whose outliers sit on one or two tokens are missing from almost every CTA's
+    own set, so those CTAs must redo their rows (re-reading them through the
+    row slots when they do not all fit); the result must not change."""
+    M, K, N = case
+    X, W, cols = synth.random_case(M, K, N, 3, seed=M + K + N)
+    free = [j for j in range(K) if j not in set(cols.tolist())]
+    j1, j2 = free[K // 3], free[2 * K // 3 + 5]
+    X[M // 2 + 3, j1] = np.float16(50.0)             # one token only
+    X[1, j2] = np.float16(-7.5)                      # two tokens far apart
+    X[M - 1, j2] = np.float16(9.0)
+    Y, got, Wq, ws = run_mixed(X, W, 6.0)
+    ref = oracle.llm_int8_matmul(X, W, 6.0)
+    assert ref["count"] == 5
+    check_intermediates(ref, got, K)
+    check_panels(X, W, ref, got)
+    assert_y_close(Y, ref["Y"], f"recheck {case}")
 
 
 def test_mixed_matmul_guard_bands():

@@ -23,11 +23,11 @@
 //               lane quarter splitting the 256 columns), dequantise, add the
 //               outlier product, round to fp16, store
 // Two ways of forming C_out, chosen on the device from the outlier count:
-//   count <= kCcMax  on CUDA cores in the epilogue from the 16-column compacted
-//                    panels (fp16 products are exact in fp32; <= 16 FMAs per
-//                    output). The two 256-column INT32
-//                    accumulators are double-buffered, so the epilogue of one
-//                    tile overlaps the MMAs of the next.
+//   count <= kCcMax  on CUDA cores in the epilogue (fp16 products are exact in
+//                    fp32; <= 16 FMAs per output), from the outlier values of X
+//                    and W gathered through the column list one tile ahead. The
+//                    two 256-column INT32 accumulators are double-buffered, so
+//                    the epilogue of one tile overlaps the MMAs of the next.
 //   count >  kCcMax  on the tensor cores: the compacted fp16 panels X_O, W_O are
 //                    streamed through the same ring after the int8 K-blocks and
 //                    multiplied with kind::f16 into an FP32 accumulator in the
@@ -82,9 +82,12 @@ struct Cfg {
   static constexpr int RING_BYTES = STAGES * STAGE_BYTES;
   static constexpr int STG_BYTES = kEpiWarps * 2 * STG_BUF_BYTES;
   static constexpr int WO_BYTES = kCcMax * BN * 2;   // W outlier tile, fp16, [j][column]
+  static constexpr int XO_BYTES = BM * kCcMax * 2;   // X outlier rows, fp16, [row][j]
   static constexpr int SW_BYTES = BN * 4;            // w_scale tile
   static constexpr int ZS_BYTES = BN * 4;            // weight row sums (zero-point mode)
-  static constexpr int BAR_OFF = RING_BYTES + STG_BYTES + WO_BYTES + SW_BYTES + ZS_BYTES;
+  static constexpr int CI_BYTES = kCcMax * 4;        // outlier column list (<= kCcMax)
+  static constexpr int BAR_OFF = RING_BYTES + STG_BYTES + WO_BYTES + XO_BYTES + SW_BYTES +
+                                 ZS_BYTES + CI_BYTES;
   static constexpr int BAR_BYTES = (2 * STAGES + 4) * 8 + 16;
   static constexpr int SMEM_BYTES = 1024 /*alignment slack*/ + BAR_OFF + BAR_BYTES;
 };
@@ -113,9 +116,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                               const int32_t* __restrict__ x_zero,
                               const int32_t* __restrict__ w_rowsum,
                               const int32_t* __restrict__ n_outliers,
-                              const __half* __restrict__ X_O, const __half* __restrict__ W_O,
-                              int ld, void* __restrict__ out, int M, int N, int K,
-                              int32_t* status) {
+                              const __half* __restrict__ X, const __half* __restrict__ W,
+                              const int32_t* __restrict__ col_idx, void* __restrict__ out,
+                              int M, int N, int K, int32_t* status) {
   using C = Cfg<PAIR>;
   constexpr int STAGES = C::STAGES;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -125,8 +128,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* smem = smem_raw + ((1024u - (smem_addr(smem_raw) & 1023u)) & 1023u);
   uint8_t* stg = smem + C::RING_BYTES;                                          // staging
   __half* wo_s = reinterpret_cast<__half*>(stg + C::STG_BYTES);                // [kCcMax][BN]
-  float* sw_s = reinterpret_cast<float*>(stg + C::STG_BYTES + C::WO_BYTES);     // [BN]
-  int32_t* zs_s = reinterpret_cast<int32_t*>(stg + C::STG_BYTES + C::WO_BYTES + C::SW_BYTES);
+  __half* xo_s = reinterpret_cast<__half*>(stg + C::STG_BYTES + C::WO_BYTES);   // [BM][kCcMax]
+  float* sw_s = reinterpret_cast<float*>(stg + C::STG_BYTES + C::WO_BYTES + C::XO_BYTES);  // [BN]
+  int32_t* zs_s = reinterpret_cast<int32_t*>(stg + C::STG_BYTES + C::WO_BYTES + C::XO_BYTES +
+                                             C::SW_BYTES);
+  int32_t* ci_s = zs_s + BN;                                                    // [kCcMax]
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::BAR_OFF);
   uint64_t* empty = full + STAGES;
   uint64_t* acc_full = empty + STAGES;   // [2]
@@ -292,8 +298,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else {
     // -------------------------------------------------------------- epilogue
     // Warp w reads TMEM lane quarter (w % 4) and the 64 columns [part*64, part*64+64)
-    // of the tile. The per-tile operands of the epilogue (w_scale of the tile's
-    // columns, the outlier panel rows) are fetched one tile ahead into registers.
+    // of the tile. The per-tile operands of the epilogue (scales, and with few
+    // outliers the outlier values of X and W) are fetched one tile ahead into
+    // registers and staged in shared memory at the start of the tile.
     const int q = warp & 3;
     const int part = (warp - 2) >> 2;
     const int et = threadIdx.x - 64;        // 0 .. 32*kEpiWarps-1
@@ -303,9 +310,20 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     float sw_next = 0.0f;
     int32_t ws_next = 0, zr_next = 0;
-    uint4 wo_next[2] = {make_uint4(0, 0, 0, 0), make_uint4(0, 0, 0, 0)};
-    uint4 xo_next[2] = {make_uint4(0, 0, 0, 0), make_uint4(0, 0, 0, 0)};
     float rs_next = 0.0f;
+    // Few outliers: the epilogue gathers the outlier values itself through the
+    // column list, one tile ahead. Thread et takes, for column n0 + (et % 256),
+    // the weights of list entries [jw, jw + 8); for its row, the activations of
+    // entries [jx, jx + 4) (the four threads of a row share them through xo_s).
+    __half wv[kCcMax / 2];
+    __half xv[kCcMax / 4];
+    const int n_l = et & (BN - 1);
+    const int jw = (et / BN) * (kCcMax / 2);
+    const int jx = part * (kCcMax / 4);
+    if (cc_out) {
+      if (et < kCcMax) ci_s[et] = et < count ? col_idx[et] : 0;
+      epi_sync();
+    }
     auto prefetch = [&](int tile) {
       if (OUT_I32 || tile >= num_tiles) return;
       const int m0 = (tile % m_tiles) * C::TILE_M + static_cast<int>(rank) * BM;
@@ -318,20 +336,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int n = n0 + et;
         sw_next = (n < N) ? w_scale[n] : 0.0f;
         if constexpr (ZP) ws_next = (n < N) ? w_rowsum[n] : 0;
-        if (cc_out && n < N) {
-          const uint4* src = reinterpret_cast<const uint4*>(W_O + static_cast<size_t>(n) * ld);
-          wo_next[0] = src[0];
-          wo_next[1] = src[1];
-        } else {
-          wo_next[0] = wo_next[1] = make_uint4(0, 0, 0, 0);
-        }
       }
-      if (cc_out && row < M) {
-        const uint4* src = reinterpret_cast<const uint4*>(X_O + static_cast<size_t>(row) * ld);
-        xo_next[0] = src[0];
-        xo_next[1] = src[1];
-      } else {
-        xo_next[0] = xo_next[1] = make_uint4(0, 0, 0, 0);
+      if (cc_out) {
+        const int n = n0 + n_l;
+        const __half* wrow = W + static_cast<size_t>(n < N ? n : 0) * K;
+#pragma unroll
+        for (int i = 0; i < kCcMax / 2; ++i)
+          wv[i] = (n < N && jw + i < count) ? wrow[ci_s[jw + i]] : __float2half_rn(0.0f);
+        const __half* xrow = X + static_cast<size_t>(row < M ? row : 0) * K;
+#pragma unroll
+        for (int i = 0; i < kCcMax / 4; ++i)
+          xv[i] = (row < M && jx + i < count) ? xrow[ci_s[jx + i]] : __float2half_rn(0.0f);
       }
     };
     prefetch(unit);
@@ -345,26 +360,35 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t aph = tc_out ? (local & 1) : ((local >> 1) & 1);
       const int row = m0 + q * 32 + lane;
 
-      // Stage this tile's column data in shared memory; keep the row data in registers.
-      __half2 xo2[kCcMax / 2];
+      // Stage this tile's column data (and the outlier values) in shared memory.
       const float rs = rs_next;
       const int32_t zr = zr_next;
       if (!OUT_I32) {
         if (et < BN) {
           sw_s[et] = sw_next;
           if constexpr (ZP) zs_s[et] = ws_next;
-          if (cc_out) {
-            const __half* h = reinterpret_cast<const __half*>(wo_next);
-#pragma unroll
-            for (int j = 0; j < kCcMax; ++j) wo_s[j * BN + et] = h[j];
-          }
         }
-        const __half2* h2 = reinterpret_cast<const __half2*>(xo_next);
+        if (cc_out) {
 #pragma unroll
-        for (int j = 0; j < kCcMax / 2; ++j) xo2[j] = h2[j];
+          for (int i = 0; i < kCcMax / 2; ++i) wo_s[(jw + i) * BN + n_l] = wv[i];
+#pragma unroll
+          for (int i = 0; i < kCcMax / 4; ++i) xo_s[(q * 32 + lane) * kCcMax + jx + i] = xv[i];
+        }
       }
       epi_sync();
-      prefetch(tile + units);
+      // The outlier activations of this thread's row, kept in registers.
+      __half2 xo2[kCcMax / 2];
+      if (cc_out) {
+        const uint4* xr = reinterpret_cast<const uint4*>(xo_s + (q * 32 + lane) * kCcMax);
+        const uint4 lo4 = xr[0], hi4 = xr[1];
+        const __half2* l2 = reinterpret_cast<const __half2*>(&lo4);
+        const __half2* h2 = reinterpret_cast<const __half2*>(&hi4);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          xo2[j] = l2[j];
+          xo2[4 + j] = h2[j];
+        }
+      }
 
       // Warp-uniform, so that a timed-out wait can never split the warp before
       // the warp-collective TMEM loads below.
@@ -508,6 +532,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         chunks(std::true_type{});
       else
         chunks(std::false_type{});
+      // The next tile's operands: issued now, so that their registers are not
+      // live during the chunk loop; the wait for the next accumulator covers
+      // their latency.
+      prefetch(tile + units);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) {
@@ -633,7 +661,7 @@ cudaError_t launch(const GemmArgs& a, cudaStream_t s) {
   cfg.numAttrs = na;
   e = cudaLaunchKernelEx(&cfg, kern, maps[0], maps[1], maps[2], maps[3], maps[4], y_tma,
                          a.x_scale, a.w_scale, a.x_zero, a.w_rowsum,
-                         OUT_I32 ? nullptr : a.n_outliers, a.X_O, a.W_O, a.ld, a.out, a.M, a.N,
+                         OUT_I32 ? nullptr : a.n_outliers, a.X, a.W, a.col_idx, a.out, a.M, a.N,
                          a.K, a.status);
   if (e != cudaSuccess) (void)cudaGetLastError();   // do not leave it for the next launch
   return e;
