@@ -78,7 +78,7 @@ constexpr uint32_t kBarList = 2;    // the first X warp publishes the outlier li
 // Shared-memory layout for nbox Wq boxes per CTA (offsets from a 1024-byte
 // aligned base).
 struct DecodeSmem {
-  int ring, bop, xs, recv, msg, bits, lidx, red, tok, misc, bars, tslot, bytes;
+  int ring, bop, xs, recv, cm, msg, bits, lidx, red, tok, misc, bars, tslot, bytes;
 };
 __host__ __device__ inline DecodeSmem decode_layout(int nbox) {
   DecodeSmem L;
@@ -87,13 +87,14 @@ __host__ __device__ inline DecodeSmem decode_layout(int nbox) {
   L.bop = off;   off += nbox * kTok * kKB;                // [nbox][16][128] i8 (swizzled)
   L.xs = off;    off += nbox * kKB * kTok * 2;            // [nbox/2][16][256] f16
   L.recv = off;  off += kRecvRows * 64;                   // [rows][4][16 B] fp32 partials
+  L.cm = off;    off += 4 * 128 * 16;                     // [4 token quarters][128 groups] column maxima
   L.msg = off;   off += kMaxCluster * kMsgWords * 4;      // [8 ranks][20] words
   L.bits = off;  off += 32 * 4;                           // outlier bitmap of the columns
   L.lidx = off;  off += kMaxCols * 2;                     // ascending outlier list
   L.red = off;   off += kMaxXWarps * kTok * 4;            // [warps][16] f32
   L.tok = off;   off += 3 * kTok * 4;                     // amax, amax/127^2, 1/amax
   L.misc = off;  off += 16;                               // lcount, prefix
-  L.bars = off;  off += (kMaxBoxes + 5) * 8;              // full[8] xbar codes done xchg red
+  L.bars = off;  off += (2 * kMaxBoxes + 5) * 8;          // full[8] codes[8] xbar - done xchg red
   L.tslot = off; off += 16;
   L.bytes = off + 1024;                                   // alignment slack
   return L;
@@ -122,6 +123,7 @@ __global__ void __launch_bounds__(64 + 32 * kMaxXWarps, 1)
   uint8_t* bop = sm + L.bop;
   __half* xs = reinterpret_cast<__half*>(sm + L.xs);
   uint8_t* recv = sm + L.recv;
+  uint8_t* cmx_s = sm + L.cm;
   uint32_t* msg = reinterpret_cast<uint32_t*>(sm + L.msg);
   uint32_t* bits = reinterpret_cast<uint32_t*>(sm + L.bits);
   uint16_t* lidx = reinterpret_cast<uint16_t*>(sm + L.lidx);
@@ -131,8 +133,8 @@ __global__ void __launch_bounds__(64 + 32 * kMaxXWarps, 1)
   float* ra_s = amax_s + 2 * kTok;
   int32_t* misc = reinterpret_cast<int32_t*>(sm + L.misc);
   uint64_t* full = reinterpret_cast<uint64_t*>(sm + L.bars);
-  uint64_t* xbar = full + kMaxBoxes;
-  uint64_t* codes_bar = xbar + 1;
+  uint64_t* cbar = full + kMaxBoxes;        // codes of K-block b written
+  uint64_t* xbar = cbar + kMaxBoxes;
   uint64_t* done = xbar + 2;
   uint64_t* xchg = xbar + 3;
   uint64_t* redbar = xbar + 4;
@@ -162,7 +164,7 @@ __global__ void __launch_bounds__(64 + 32 * kMaxXWarps, 1)
   if (tid == 0) {
     for (int b = 0; b < kMaxBoxes; ++b) mbar_init(&full[b], 1);
     mbar_init(xbar, 1);
-    mbar_init(codes_bar, nxw);
+    for (int b = 0; b < kMaxBoxes; ++b) mbar_init(&cbar[b], 2);   // the two warps of a block
     mbar_init(done, 1);
     mbar_init(xchg, 1);
     mbar_init(redbar, 1);
@@ -202,13 +204,15 @@ __global__ void __launch_bounds__(64 + 32 * kMaxXWarps, 1)
   } else if (warp == 1) {
     // ---------------------------------------------------------------- MMA issuer
     cluster_wait();
-    ok = __all_sync(0xffffffffu, mbar_wait(codes_bar, 0));
-    // Orders the MMAs after the X workers' code stores (a thread sync). The
-    // Wq boxes come from TMA and need only their mbarrier.
-    tc_fence_after();
     constexpr uint32_t idesc = make_idesc(2 /*s32*/, 1 /*signed*/, kTileRows, kTok);
     const uint64_t a0 = sw128_kmajor_desc(smem_addr(ring));
     const uint64_t b0 = sw128_kmajor_desc(smem_addr(bop));
+    // All the codes first, then one tcgen05 fence: a fence per K-block costs
+    // more in MMA issue than waiting for the last block's codes.
+    for (int b = 0; b < nb && ok; ++b) ok = __all_sync(0xffffffffu, mbar_wait(&cbar[b], 0));
+    // Orders the MMAs after the X workers' code stores (a thread sync). The
+    // Wq boxes come from TMA and need only their mbarrier.
+    tc_fence_after();
     for (int b = 0; b < nb && ok; ++b) {
       ok = __all_sync(0xffffffffu, mbar_wait(&full[b], 0));
       if (!ok) break;
@@ -230,45 +234,81 @@ __global__ void __launch_bounds__(64 + 32 * kMaxXWarps, 1)
     // warps, and straight-line code would be bound by instruction fetch.
     const int xw = warp - 2;
     const int xi = tid - 64;
-    const int c0 = 2 * xi;                   // the thread's 2 columns (CTA-local)
-    const bool cv = c0 < kw;                 // kw is a multiple of 16
     const float thr = a.threshold;
     const bool epi = (warp >= 4 && warp < 8);
-    // Column pair c0 of token t: box c0/256, row t, column c0%256.
-    const uint32_t* xcol =
-        reinterpret_cast<const uint32_t*>(xs + (c0 >> 8) * (kTok * kXBox) + (c0 & (kXBox - 1)));
-    constexpr int xstride = kXBox / 2;       // uint32 per token row of a box
+    constexpr int xvs = kXBox / 8;           // 16-byte vectors per token row of an X box
+    const int ng = kw >> 3;                  // 8-column groups of this CTA's slice
+    // Group g of the slice: box g / 32, columns 8g % 256 .. +7.
+    auto xgroup = [&](int g) -> const uint4* {
+      return reinterpret_cast<const uint4*>(xs + (g >> 5) * (kTok * kXBox) + ((8 * g) & (kXBox - 1)));
+    };
 
     ok = __all_sync(0xffffffffu, mbar_wait(xbar, 0));
 
-    // Outlier flags of the 2 columns: the max of |x| over all tokens against the threshold.
-    __half2 cm = __float2half2_rn(0.0f);
-    if (cv) {
-#pragma unroll 4
-      for (int t = 0; t < M; ++t) cm = __hmax2(cm, habs2_bits(xcol[t * xstride]));
-    }
-    const float2 cf = __half22float2(cm);
-    const uint32_t f2 = (cf.x > thr ? 1u : 0u) | (cf.y > thr ? 2u : 0u);
-    const uint32_t keep = ((f2 & 1u) ? 0u : 0x0000FFFFu) | ((f2 & 2u) ? 0u : 0xFFFF0000u);
-    const uint32_t keepq = ((f2 & 1u) ? 0u : 0x00FFu) | ((f2 & 2u) ? 0u : 0xFF00u);
+    // Thread (g, tq): the 8 columns of group g = xi % 128 for the tokens
+    // 4tq .. 4tq+3, tq = xi / 128 (one token quarter per warp).
+    const int g = xi & 127;
+    const int tq = xi >> 7;
+    const bool gv = g < ng;
+    uint4 xv[4];
     {
-      // Bitmap word of 32 columns = 16 threads x 2 flags.
-      uint32_t word = f2 << (2 * (lane & 15));
+      __half2 cm[4];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) cm[k] = __float2half2_rn(0.0f);
+      const uint4* xg = xgroup(gv ? g : 0);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int t = 4 * tq + j;
+        xv[j] = (gv && t < M) ? xg[t * xvs] : make_uint4(0, 0, 0, 0);
+        const uint32_t* wd = reinterpret_cast<const uint32_t*>(&xv[j]);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) cm[k] = __hmax2(cm[k], habs2_bits(wd[k]));
+      }
+      reinterpret_cast<uint4*>(cmx_s)[tq * 128 + g] = *reinterpret_cast<const uint4*>(cm);
+    }
+    named_bar_sync(kBarX, nxt);
+    // Outlier flags of the 8 columns: the max of |x| over all tokens against the threshold.
+    uint32_t f8 = 0;
+    {
+      __half2 cm[4];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) cm[k] = __float2half2_rn(0.0f);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const uint4 u = reinterpret_cast<const uint4*>(cmx_s)[q * 128 + g];
+        const __half2* h = reinterpret_cast<const __half2*>(&u);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) cm[k] = __hmax2(cm[k], h[k]);
+      }
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const float2 m = __half22float2(cm[k]);
+        f8 |= (m.x > thr ? 1u : 0u) << (2 * k);
+        f8 |= (m.y > thr ? 1u : 0u) << (2 * k + 1);
+      }
+      if (!gv) f8 = 0;
+    }
+    if (tq == 0) {
+      // Bitmap word of 32 columns = 4 consecutive groups.
+      uint32_t word = f8 << (8 * (lane & 3));
       word |= __shfl_xor_sync(0xffffffffu, word, 1);
       word |= __shfl_xor_sync(0xffffffffu, word, 2);
-      word |= __shfl_xor_sync(0xffffffffu, word, 4);
-      word |= __shfl_xor_sync(0xffffffffu, word, 8);
-      if ((lane & 15) == 0) bits[xi >> 4] = word;
+      if ((lane & 3) == 0 && gv) bits[g >> 2] = word;
     }
     // Per-token max of |x| over the non-outlier columns, per warp with one
-    // redux (non-negative floats order like their bit patterns).
-#pragma unroll 2
-    for (int t = 0; t < M; ++t) {
-      const uint32_t v = cv ? xcol[t * xstride] : 0u;
-      const float2 f = __half22float2(habs2_bits(v & keep));
+    // redux (non-negative floats order like their bit patterns); the warp's
+    // slots of the other quarters' tokens hold 0.
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const uint32_t* wd = reinterpret_cast<const uint32_t*>(&xv[j]);
+      __half2 h = __float2half2_rn(0.0f);
+#pragma unroll
+      for (int k = 0; k < 4; ++k) h = __hmax2(h, habs2_bits(wd[k] & keep_half2(f8, k)));
+      const float2 f = __half22float2(h);
       const uint32_t wm = __reduce_max_sync(0xffffffffu, __float_as_uint(fmaxf(f.x, f.y)));
-      if (lane == 0) red[xw * kTok + t] = __uint_as_float(wm);
+      if (lane == 0) red[xw * kTok + 4 * tq + j] = __uint_as_float(wm);
     }
+    if (lane < kTok && (lane >> 2) != tq) red[xw * kTok + lane] = 0.0f;
     named_bar_sync(kBarX, nxt);
 
     if (xw == 0) {
@@ -367,26 +407,43 @@ __global__ void __launch_bounds__(64 + 32 * kMaxXWarps, 1)
       for (int i = xi; i < lc; i += nxt) a.col_idx[prefix + i] = k0 + lidx[i];
     }
 
-    // INT8 codes of the 2 columns for every token, into the B operand (and Xq).
-    if (c0 < nb * kKB) {
-      const uint32_t kc = static_cast<uint32_t>(c0) & 127u;
-      uint8_t* dst = bop + (c0 >> 7) * (kTok * kKB) + (kc & 15u);
-      int8_t* xq = a.Xq + k0 + c0;
-#pragma unroll 2
-      for (int t = 0; t < kTok; ++t) {
-        uint32_t qv = 0u;
-        if (cv && t < M) {
-          qv = codes2(xcol[t * xstride], amax_s[t], ra_s[t]) & keepq;
-          if (writer)
-            *reinterpret_cast<uint16_t*>(xq + static_cast<size_t>(t) * K) = static_cast<uint16_t>(qv);
+    // INT8 codes into the B operand (and Xq): thread xi takes K-block
+    // b = xi / 64 (two warps per block, each block with its own barrier), group
+    // gi = xi % 16 of the block's 16, and the tokens 4tc .. 4tc+3,
+    // tc = (xi / 16) % 4.
+    {
+      const int b = xi >> 6;
+      const int gi = xi & 15;
+      const int tc = (xi >> 4) & 3;
+      const int gg = b * 16 + gi;
+      if (b < nb) {
+        const bool live = gg < ng;
+        const uint32_t m8 = live ? (bits[gg >> 2] >> (8 * (gg & 3))) & 0xFFu : 0xFFu;
+        const uint4* xg = xgroup(live ? gg : 0);
+        uint8_t* dst = bop + b * (kTok * kKB) + (gi & 1) * 8;
+        int8_t* xq = a.Xq + k0 + 8 * gg;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const int t = 4 * tc + j;
+          uint2 qv = make_uint2(0u, 0u);
+          if (live && t < M) {
+            qv = codes8(xg[t * xvs], amax_s[t], ra_s[t]);
+            if (m8) {
+              qv.x &= keep_bytes(m8 & 0xFu);
+              qv.y &= keep_bytes(m8 >> 4);
+            }
+            if (writer) *reinterpret_cast<uint2*>(xq + static_cast<size_t>(t) * K) = qv;
+          }
+          // Row t of the 128-byte-swizzled K-major operand: 16-byte chunk gi/2
+          // of the block's 128 columns, XOR the row's position in its 8-row group.
+          const uint32_t off = (t >> 3) * 1024 + (t & 7) * 128 + ((((gi >> 1) ^ (t & 7))) << 4);
+          *reinterpret_cast<uint2*>(dst + off) = qv;
         }
-        const uint32_t off = (t >> 3) * 1024 + (t & 7) * 128 + (((kc >> 4) ^ (t & 7)) << 4);
-        *reinterpret_cast<uint16_t*>(dst + off) = static_cast<uint16_t>(qv);
+        fence_proxy_async_smem();   // the tensor core reads what the generic proxy wrote
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&cbar[b]);
       }
     }
-    fence_proxy_async_smem();   // the tensor core reads what the generic proxy wrote
-    __syncwarp();
-    if (lane == 0) mbar_arrive(codes_bar);
 
     if (!epi) {
       cluster_arrive();
