@@ -107,10 +107,8 @@ size_t int8_mixed_matmul_workspace_size(int M, int N, int K);
  * caller or a test read the outlier set, codes and scales of the last call.
  * The outlier panels have row stride panel_ld elements (fp16) and hold the
  * compacted outlier columns in ascending column order, zero-padded to a
- * multiple of 64 columns; they are written only when there are more than 16
- * outlier columns (the GEMM multiplies them on the tensor cores). With 1..16
- * the GEMM epilogue reads the outlier values of X and W through col_idx and
- * adds the product on CUDA cores, and the panels are not written.
+ * multiple of 64 columns (the GEMM multiplies them on the tensor cores).
+ * Nothing is written to them when there are no outliers.
  */
 typedef struct {
   size_t n_outliers;   /* int32 [1] */

@@ -22,7 +22,7 @@ CASES = [
     (300, 512, 384, 5, [0, 100, 300]),
     (300, 512, 384, 5, [0, 0, 7, 300]),          # an empty rank, a rank with 7 tokens
     (1024, 4096, 1024, 6, [0, 256, 512, 768, 1024]),
-    (256, 1024, 512, 40, [0, 130, 256]),        # > 16 outliers: tensor-core outlier product
+    (256, 1024, 512, 40, [0, 130, 256]),        # 40 outlier columns: one 64-column panel block
 ]
 
 

@@ -44,7 +44,7 @@ CASES = [
     (256, 1024, 512, 6, 6.0),
     (300, 1040, 136, 3, 6.0),
     (2048, 4096, 1024, 6, 6.0),
-    (256, 1024, 512, 40, 6.0),            # > 16 outliers: tensor-core outlier product
+    (256, 1024, 512, 40, 6.0),            # 40 outlier columns: one 64-column panel block
     (16, 512, 256, 2, 6.0),               # small M: single-CTA GEMM tiles
     (256, 1024, 512, 6, float("inf")),    # pure zero-point W8A8
     (128, 512, 256, 4, 0.0),              # every nonzero column an outlier

@@ -319,9 +319,6 @@ int mixed_matmul_impl(const void* X, const int8_t* Wq, const float* w_scale, con
   g.Wq = Wq;
   g.X_O = XO;
   g.W_O = WO;
-  g.X = Xh;
-  g.W = Wh;
-  g.col_idx = idx;
   g.ld = L.l.panel_ld;
   g.x_scale = xs;
   g.w_scale = w_scale;

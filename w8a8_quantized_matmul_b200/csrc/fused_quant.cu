@@ -16,31 +16,31 @@
 // is done; the others redo their rows with O. The results are the same either
 // way; only the time differs.
 //
-// Each CTA owns a contiguous block of R rows of X and of the rows of W. Its
-// rows stream through a ring of S row slots in shared memory (bulk copies, one
-// mbarrier per slot), visited in chunks: a chunk's slots are refilled with the
-// rows S visits later once every thread is done with it.
-//   pass A   forward over the rows: thread t owns the 16-byte vectors
-//            v = t + 512*c of every row and keeps a packed-fp16 running max of
-//            |x| per owned column; the column maxima against the threshold
-//            give the CTA's outlier flags, ORed into the global bitmap (atomics
-//            only for non-zero words); then the CTA arrives at the grid barrier
-//            and does not wait
-//   local    the ascending list of the CTA's outlier columns; the W_O gathers of
-//            the CTA's weight rows are issued with it (kept in registers)
-//   pass B   backward over the rows (the last rows of pass A are still in their
-//            slots): teams of warps own rows; per row the absmax over the
-//            non-outlier columns (redux per warp; one block barrier per chunk
-//            when a row is shared by several warps), INT8 codes with paired
-//            fp32 arithmetic, the row of the X_O panel
-//   check    wait at the grid barrier (bounded); if the global bitmap holds a
-//            column the CTA's own set lacks, pass B runs again forward with the
-//            global set and the W_O rows are gathered again
-//   W_O      the CTA's rows of the compacted weight panel are stored.
-// The panels are kCcMaxOutliers columns wide (zero-padded) when the GEMM
-// epilogue adds the outlier product itself, or a multiple of 64 wide when the
-// GEMM multiplies them on the tensor cores.
-//
+// Each CTA owns a contiguous block of R rows of X and of the rows of W.
+//   pass A   all 16 warps: the rows stream through a ring of S row slots in
+//            shared memory (bulk copies, one mbarrier per slot; a chunk's slots
+//            are refilled with the rows S further on once every thread is done
+//            with it). Thread t owns the 16-byte vectors v = t + 512*c of every
+//            row and keeps a packed-fp16 running max of |x| per owned column;
+//            the column maxima against the threshold give the CTA's outlier
+//            flags, ORed into the batch bitmap (atomics only for non-zero
+//            words). Afterwards the slots hold the last min(R, S) rows.
+//   pass B   warps 0-14: per row the absmax over the non-outlier columns of the
+//            CTA's own set (redux per warp; teams of warps share a row through
+//            named barrier 1) and the INT8 codes with paired fp32 arithmetic;
+//            the rows still in their slots are read from shared memory, the
+//            others again from L2 into registers, a few rows per round.
+//   control  warp 15, meanwhile: arrives at the grid barrier, builds the CTA's
+//            ascending outlier list, waits at the barrier (bounded) and compares
+//            the batch bitmap with the CTA's.
+//   redo     only if the batch has a column the CTA's rows missed: pass B and
+//            the list again with the batch's set.
+//   panels   with any outlier column, by the workers right after pass B (with
+//            the CTA's list; again after a redo): the CTA's rows of the
+//            compacted fp16 panels X_O (from the slots or L2) and W_O (gathered
+//            from W), a multiple of 64 columns wide and zero-padded. The GEMM
+//            multiplies them on the tensor cores.
+
 // The code of x is rint(fl32(fl32(x*127)/a)) clamped to +-127. The correctly
 // rounded quotient is formed without a division (codes8 in quant_common.cuh:
 // Markstein's FMA-corrected product with fl(1/a), exact for every pair of fp16
@@ -66,6 +66,7 @@ constexpr int kWarps = kThreads / 32;
 // themselves on named barrier 1.
 constexpr int kWorkers = kWarps - 1;
 constexpr uint32_t kWorkBar = 1;
+constexpr uint32_t kListBar = 2;   // the control warp has built the CTA's list
 constexpr int kMaxSlots = 16;                 // row slots in shared memory
 constexpr uint64_t kBarrierLimitNs = 2000000000ull;
 
@@ -445,8 +446,52 @@ __global__ void __launch_bounds__(kThreads, VPT <= 2 ? 2 : 1)
     if (lane == 31) s_misc[0] = incl;
   };
 
+  // ------------------------------------------------------------ panels
+  // The CTA's rows of the compacted fp16 panels for the list in s_idx, a
+  // multiple of 64 columns wide and zero-padded: X_O (from the slots or L2)
+  // and W_O (gathered from W). Run by the threads [t0, t0 + nt).
+  const int nper = (a.N + gridDim.x - 1) / gridDim.x;
+  const int wn0 = min(a.N, static_cast<int>(blockIdx.x) * nper);
+  const int wn1 = min(a.N, wn0 + nper);
+  auto panels = [&](int count, int t0, int nt) {
+    if (count == 0) return;
+    const int pw = (count + 63) & ~63;
+    for (int e = tid - t0; e < R * pw; e += nt) {
+      const int row = e / pw;
+      const int p = e - row * pw;
+      __half v = __float2half_rn(0.0f);
+      if (p < count) {
+        v = (row >= R - nres)
+                ? reinterpret_cast<const __half*>(s_rows + static_cast<size_t>(row % S) * row_bytes)[s_idx[p]]
+                : X[static_cast<size_t>(r0 + row) * K + s_idx[p]];
+      }
+      a.X_O[static_cast<size_t>(r0 + row) * a.ld + p] = v;
+    }
+    const int chunks = pw >> 3;
+    const int items = (wn1 - wn0) * chunks;
+    // One item = 8 consecutive panel columns of one weight row: up to 8
+    // independent gathers, one 16-byte store.
+    for (int it = tid - t0; it < items; it += nt) {
+      const int n = wn0 + it / chunks;
+      const int ch = it - (n - wn0) * chunks;
+      const __half* wrow = W + static_cast<size_t>(n) * K;
+      uint4 o;
+      __half* h = reinterpret_cast<__half*>(&o);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int p = ch * 8 + i;
+        h[i] = (p < count) ? wrow[s_idx[p]] : __float2half_rn(0.0f);
+      }
+      reinterpret_cast<uint4*>(a.W_O + static_cast<size_t>(n) * a.ld)[ch] = o;
+    }
+  };
+
   if (warp < kWorkers) {
     quantise(s_lbits);
+    // The panels with the CTA's own list (the batch's, unless the check below
+    // finds a column the CTA's rows missed), while the control warp waits.
+    named_bar_sync(kListBar, kThreads);
+    panels(s_misc[0], 0, 32 * kWorkers);
   } else {
     // Control warp: arrive at the grid barrier, build this CTA's list (the
     // batch's list unless the check below finds a column it lacks), wait at the
@@ -457,6 +502,8 @@ __global__ void __launch_bounds__(kThreads, VPT <= 2 ? 2 : 1)
     }
     __syncwarp();
     build_list(s_lbits);
+    __syncwarp();
+    named_bar_arrive(kListBar, kThreads);
     int extra = 0;
     if (!given) {
       if (lane == 0) {
@@ -482,54 +529,19 @@ __global__ void __launch_bounds__(kThreads, VPT <= 2 ? 2 : 1)
   }
   __syncthreads();
   if (s_misc[1]) {
-    // This CTA's rows missed an outlier column of the batch: codes and list
-    // again with the batch's set.
+    // This CTA's rows missed an outlier column of the batch: codes, list and
+    // panels again with the batch's set.
     if (warp < kWorkers)
       quantise(s_gbits);
     else
       build_list(s_gbits);
     __syncthreads();
+    panels(s_misc[0], 0, kThreads);
   }
   const int count = s_misc[0];
   if (blockIdx.x == 0) {
     for (int p = tid; p < count; p += kThreads) a.col_idx[p] = s_idx[p];
     if (tid == 0) *a.n_outliers = count;
-  }
-  // Up to kCcMaxOutliers outlier columns the GEMM epilogue reads the outlier
-  // values of X and W itself; beyond, the tensor cores multiply compacted fp16
-  // panels, a multiple of 64 columns wide (zero-padded), built here.
-  if (count <= kCcMaxOutliers) return;
-  const int pw = (count + 63) & ~63;
-  for (int e = tid; e < R * pw; e += kThreads) {
-    const int row = e / pw;
-    const int p = e - row * pw;
-    __half v = __float2half_rn(0.0f);
-    if (p < count) {
-      v = (!given && row >= R - nres)
-              ? reinterpret_cast<const __half*>(s_rows + static_cast<size_t>(row % S) * row_bytes)[s_idx[p]]
-              : X[static_cast<size_t>(r0 + row) * K + s_idx[p]];
-    }
-    a.X_O[static_cast<size_t>(r0 + row) * a.ld + p] = v;
-  }
-  const int nper = (a.N + gridDim.x - 1) / gridDim.x;
-  const int wn0 = min(a.N, static_cast<int>(blockIdx.x) * nper);
-  const int wn1 = min(a.N, wn0 + nper);
-  const int chunks = pw >> 3;
-  const int items = (wn1 - wn0) * chunks;
-  // One item = 8 consecutive panel columns of one weight row: up to 8
-  // independent gathers, one 16-byte store.
-  for (int it = tid; it < items; it += kThreads) {
-    const int n = wn0 + it / chunks;
-    const int ch = it - (n - wn0) * chunks;
-    const __half* wrow = W + static_cast<size_t>(n) * K;
-    uint4 o;
-    __half* h = reinterpret_cast<__half*>(&o);
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const int p = ch * 8 + i;
-      h[i] = (p < count) ? wrow[s_idx[p]] : __float2half_rn(0.0f);
-    }
-    reinterpret_cast<uint4*>(a.W_O + static_cast<size_t>(n) * a.ld)[ch] = o;
   }
   (void)ok;
 }

@@ -2,7 +2,8 @@
 //
 //   Y[i][n] = fp16( C_i32[i][n] * x_scale[i] * w_scale[n] / 127^2 + C_out[i][n] )
 //   C_i32   = Xq . Wq^T          tcgen05.mma kind::i8, INT32 accumulator in TMEM
-//   C_out   = X_O . W_O^T        the FP16 product over the outlier columns
+//   C_out   = X_O . W_O^T        the FP16 product over the outlier columns,
+//                                tcgen05.mma kind::f16, FP32 accumulator in TMEM
 //
 // Method: AIInfra "05Infer/06CompDistill/05Quantization01", LLM.int8() section:
 // INT8 matmul accumulated in INT32, dequantisation by the outer product of the
@@ -22,16 +23,18 @@
 //   warps 2-17  epilogue: tcgen05.ld (thread = output row, four warps per TMEM
 //               lane quarter splitting the 256 columns), dequantise, add the
 //               outlier product, round to fp16, store
-// Two ways of forming C_out, chosen on the device from the outlier count:
-//   count <= kCcMax  on CUDA cores in the epilogue (fp16 products are exact in
-//                    fp32; <= 16 FMAs per output), from the outlier values of X
-//                    and W gathered through the column list one tile ahead. The
-//                    two 256-column INT32 accumulators are double-buffered, so
-//                    the epilogue of one tile overlaps the MMAs of the next.
-//   count >  kCcMax  on the tensor cores: the compacted fp16 panels X_O, W_O are
-//                    streamed through the same ring after the int8 K-blocks and
-//                    multiplied with kind::f16 into an FP32 accumulator in the
-//                    other half of TMEM (single-buffered).
+// The mode is chosen on the device from the outlier count:
+//   count == 0  INT8 only; the two 256-column INT32 accumulators are
+//               double-buffered, so the epilogue of one tile overlaps the MMAs
+//               of the next.
+//   count >  0  the compacted fp16 panels X_O, W_O (64-column blocks) are
+//               streamed through the same ring after the int8 K-blocks and
+//               multiplied with kind::f16 into an FP32 accumulator in the other
+//               half of TMEM (single-buffered). Measured on B200 with 6-7
+//               outlier columns, this beat forming the outlier product on CUDA
+//               cores in a double-buffered epilogue (OPT-6.7B FFN-up GEMM
+//               101 against 108 us): the CUDA-core work and its gathers slowed
+//               the main loop more than the lost overlap costs.
 // The outlier count is read from device memory, so the host never syncs.
 // No TMA load uses cluster multicast: both CTAs of a pair load their own halves,
 // completing on the even CTA's barrier. Every mbarrier wait is bounded;
@@ -60,7 +63,6 @@ constexpr int KB_I8 = 128;           // int8 columns per K-block (128 bytes)
 constexpr int KB_F16 = 64;           // fp16 columns per panel block (128 bytes)
 constexpr int kEpiWarps = 16;          // four per TMEM lane quarter, 64 columns each
 constexpr int kThreads = 64 + 32 * kEpiWarps;
-constexpr int kCcMax = kCcMaxOutliers;   // outlier counts handled on CUDA cores
 constexpr int kStatusTimeout = -5;   // == I8MM_ERR_TIMEOUT
 constexpr uint32_t TMEM_COLS = 512;
 
@@ -81,13 +83,9 @@ struct Cfg {
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr int RING_BYTES = STAGES * STAGE_BYTES;
   static constexpr int STG_BYTES = kEpiWarps * 2 * STG_BUF_BYTES;
-  static constexpr int WO_BYTES = kCcMax * BN * 2;   // W outlier tile, fp16, [j][column]
-  static constexpr int XO_BYTES = BM * kCcMax * 2;   // X outlier rows, fp16, [row][j]
   static constexpr int SW_BYTES = BN * 4;            // w_scale tile
   static constexpr int ZS_BYTES = BN * 4;            // weight row sums (zero-point mode)
-  static constexpr int CI_BYTES = kCcMax * 4;        // outlier column list (<= kCcMax)
-  static constexpr int BAR_OFF = RING_BYTES + STG_BYTES + WO_BYTES + XO_BYTES + SW_BYTES +
-                                 ZS_BYTES + CI_BYTES;
+  static constexpr int BAR_OFF = RING_BYTES + STG_BYTES + SW_BYTES + ZS_BYTES;
   static constexpr int BAR_BYTES = (2 * STAGES + 4) * 8 + 16;
   static constexpr int SMEM_BYTES = 1024 /*alignment slack*/ + BAR_OFF + BAR_BYTES;
 };
@@ -115,9 +113,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                               const float* __restrict__ w_scale,
                               const int32_t* __restrict__ x_zero,
                               const int32_t* __restrict__ w_rowsum,
-                              const int32_t* __restrict__ n_outliers,
-                              const __half* __restrict__ X, const __half* __restrict__ W,
-                              const int32_t* __restrict__ col_idx, void* __restrict__ out,
+                              const int32_t* __restrict__ n_outliers, void* __restrict__ out,
                               int M, int N, int K, int32_t* status) {
   using C = Cfg<PAIR>;
   constexpr int STAGES = C::STAGES;
@@ -127,12 +123,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   // the shared state space and compiles to shared-memory loads and stores.
   uint8_t* smem = smem_raw + ((1024u - (smem_addr(smem_raw) & 1023u)) & 1023u);
   uint8_t* stg = smem + C::RING_BYTES;                                          // staging
-  __half* wo_s = reinterpret_cast<__half*>(stg + C::STG_BYTES);                // [kCcMax][BN]
-  __half* xo_s = reinterpret_cast<__half*>(stg + C::STG_BYTES + C::WO_BYTES);   // [BM][kCcMax]
-  float* sw_s = reinterpret_cast<float*>(stg + C::STG_BYTES + C::WO_BYTES + C::XO_BYTES);  // [BN]
-  int32_t* zs_s = reinterpret_cast<int32_t*>(stg + C::STG_BYTES + C::WO_BYTES + C::XO_BYTES +
-                                             C::SW_BYTES);
-  int32_t* ci_s = zs_s + BN;                                                    // [kCcMax]
+  float* sw_s = reinterpret_cast<float*>(stg + C::STG_BYTES);                  // [BN]
+  int32_t* zs_s = reinterpret_cast<int32_t*>(stg + C::STG_BYTES + C::SW_BYTES);  // [BN]
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::BAR_OFF);
   uint64_t* empty = full + STAGES;
   uint64_t* acc_full = empty + STAGES;   // [2]
@@ -159,6 +151,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&acc_full[b], 1);
       mbar_init(&acc_empty[b], (PAIR ? 2 : 1) * kEpiWarps);   // epilogue warps of the pair
     }
+
     *abort_flag = 0;
     fence_mbarrier_init();
     tma_prefetch_desc(&tmA);
@@ -188,10 +181,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   griddep_wait();
 
   const int count = (!OUT_I32 && n_outliers) ? *n_outliers : 0;
-  const bool tc_out = count > kCcMax;          // outlier product on the tensor cores
+  const bool tc_out = count > 0;               // outlier product on the tensor cores
   const int nk = (K + KB_I8 - 1) / KB_I8;
   const int np = tc_out ? (count + KB_F16 - 1) / KB_F16 : 0;
   const int iters = nk + np;
+
 
   if (warp == 0) {
     if (lane == 0) {
@@ -298,32 +292,17 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else {
     // -------------------------------------------------------------- epilogue
     // Warp w reads TMEM lane quarter (w % 4) and the 64 columns [part*64, part*64+64)
-    // of the tile. The per-tile operands of the epilogue (scales, and with few
-    // outliers the outlier values of X and W) are fetched one tile ahead into
-    // registers and staged in shared memory at the start of the tile.
+    // of the tile. The per-tile scales of the epilogue are fetched one tile ahead
+    // into registers; the column scales are staged in shared memory.
     const int q = warp & 3;
     const int part = (warp - 2) >> 2;
     const int et = threadIdx.x - 64;        // 0 .. 32*kEpiWarps-1
-    const bool cc_out = !OUT_I32 && !tc_out && count > 0;
     const bool vec_ok = (N % 8) == 0;
     const int col_lo = part * (BN / 4);
 
     float sw_next = 0.0f;
     int32_t ws_next = 0, zr_next = 0;
     float rs_next = 0.0f;
-    // Few outliers: the epilogue gathers the outlier values itself through the
-    // column list, one tile ahead. Thread et takes, for column n0 + (et % 256),
-    // the weights of list entries [jw, jw + 8); for its row, the activations of
-    // entries [jx, jx + 4) (the four threads of a row share them through xo_s).
-    __half wv[kCcMax / 2];
-    __half xv[kCcMax / 4];
-    const int n_l = et & (BN - 1);
-    const int jw = (et / BN) * (kCcMax / 2);
-    const int jx = part * (kCcMax / 4);
-    if (cc_out) {
-      if (et < kCcMax) ci_s[et] = et < count ? col_idx[et] : 0;
-      epi_sync();
-    }
     auto prefetch = [&](int tile) {
       if (OUT_I32 || tile >= num_tiles) return;
       const int m0 = (tile % m_tiles) * C::TILE_M + static_cast<int>(rank) * BM;
@@ -337,17 +316,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         sw_next = (n < N) ? w_scale[n] : 0.0f;
         if constexpr (ZP) ws_next = (n < N) ? w_rowsum[n] : 0;
       }
-      if (cc_out) {
-        const int n = n0 + n_l;
-        const __half* wrow = W + static_cast<size_t>(n < N ? n : 0) * K;
-#pragma unroll
-        for (int i = 0; i < kCcMax / 2; ++i)
-          wv[i] = (n < N && jw + i < count) ? wrow[ci_s[jw + i]] : __float2half_rn(0.0f);
-        const __half* xrow = X + static_cast<size_t>(row < M ? row : 0) * K;
-#pragma unroll
-        for (int i = 0; i < kCcMax / 4; ++i)
-          xv[i] = (row < M && jx + i < count) ? xrow[ci_s[jx + i]] : __float2half_rn(0.0f);
-      }
     };
     prefetch(unit);
 
@@ -360,35 +328,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t aph = tc_out ? (local & 1) : ((local >> 1) & 1);
       const int row = m0 + q * 32 + lane;
 
-      // Stage this tile's column data (and the outlier values) in shared memory.
+      // Stage this tile's column scales in shared memory; the row scale stays in a register.
       const float rs = rs_next;
       const int32_t zr = zr_next;
-      if (!OUT_I32) {
-        if (et < BN) {
-          sw_s[et] = sw_next;
-          if constexpr (ZP) zs_s[et] = ws_next;
-        }
-        if (cc_out) {
-#pragma unroll
-          for (int i = 0; i < kCcMax / 2; ++i) wo_s[(jw + i) * BN + n_l] = wv[i];
-#pragma unroll
-          for (int i = 0; i < kCcMax / 4; ++i) xo_s[(q * 32 + lane) * kCcMax + jx + i] = xv[i];
-        }
+      if (!OUT_I32 && et < BN) {
+        sw_s[et] = sw_next;
+        if constexpr (ZP) zs_s[et] = ws_next;
       }
       epi_sync();
-      // The outlier activations of this thread's row, kept in registers.
-      __half2 xo2[kCcMax / 2];
-      if (cc_out) {
-        const uint4* xr = reinterpret_cast<const uint4*>(xo_s + (q * 32 + lane) * kCcMax);
-        const uint4 lo4 = xr[0], hi4 = xr[1];
-        const __half2* l2 = reinterpret_cast<const __half2*>(&lo4);
-        const __half2* h2 = reinterpret_cast<const __half2*>(&hi4);
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          xo2[j] = l2[j];
-          xo2[4 + j] = h2[j];
-        }
-      }
 
       // Warp-uniform, so that a timed-out wait can never split the warp before
       // the warp-collective TMEM loads below.
@@ -457,30 +404,6 @@ __global__ void __launch_bounds__(kThreads, 1)
               if constexpr (TC) {
 #pragma unroll
                 for (int j = 0; j < 16; ++j) y[j] += __uint_as_float(oacc[j]);
-              } else if (cc_out) {
-                float o[16];
-#pragma unroll
-                for (int j = 0; j < 16; ++j) o[j] = 0.0f;
-#pragma unroll
-                for (int t = 0; t < kCcMax; ++t) {
-                  if (t < count) {
-                    const float xt = (t & 1) ? __high2float(xo2[t >> 1]) : __low2float(xo2[t >> 1]);
-                    const uint4* w8 = reinterpret_cast<const uint4*>(wo_s + t * BN + c);
-#pragma unroll
-                    for (int j = 0; j < 2; ++j) {
-                      const uint4 wv = w8[j];
-                      const __half2* w2 = reinterpret_cast<const __half2*>(&wv);
-#pragma unroll
-                      for (int i = 0; i < 4; ++i) {
-                        const float2 w = __half22float2(w2[i]);
-                        o[8 * j + 2 * i] = fmaf(xt, w.x, o[8 * j + 2 * i]);
-                        o[8 * j + 2 * i + 1] = fmaf(xt, w.y, o[8 * j + 2 * i + 1]);
-                      }
-                    }
-                  }
-                }
-#pragma unroll
-                for (int j = 0; j < 16; ++j) y[j] += o[j];
               }
               __half* orow = reinterpret_cast<__half*>(out) + static_cast<size_t>(row) * N;
               if (y_tma) {
@@ -544,7 +467,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         else
           mbar_arrive(&acc_empty[buf]);
       }
-      epi_sync();   // the tile's sw_s / wo_s are no longer read
+      epi_sync();   // the tile's sw_s / zs_s are no longer read
       if (!ok || *abort_flag) break;
     }
     if (!OUT_I32 && y_tma && lane == 0) bulk_wait_group_all();
@@ -661,8 +584,7 @@ cudaError_t launch(const GemmArgs& a, cudaStream_t s) {
   cfg.numAttrs = na;
   e = cudaLaunchKernelEx(&cfg, kern, maps[0], maps[1], maps[2], maps[3], maps[4], y_tma,
                          a.x_scale, a.w_scale, a.x_zero, a.w_rowsum,
-                         OUT_I32 ? nullptr : a.n_outliers, a.X, a.W, a.col_idx, a.out, a.M, a.N,
-                         a.K, a.status);
+                         OUT_I32 ? nullptr : a.n_outliers, a.out, a.M, a.N, a.K, a.status);
   if (e != cudaSuccess) (void)cudaGetLastError();   // do not leave it for the next launch
   return e;
 }

@@ -13,10 +13,6 @@ namespace i8mm {
 constexpr int kDetectRows = 32;        // rows of X per detection CTA
 constexpr int kQuantRowsPerWarp = 1;   // rows of X per warp in the quantisation kernel
 constexpr int kPanelAlign = 64;        // outlier panels are padded to this many columns
-// Up to this many outlier columns the GEMM adds the fp16 outlier product on CUDA
-// cores in its epilogue (reading X and W through the column list); beyond it the
-// compacted panels X_O, W_O are multiplied on the tensor cores.
-constexpr int kCcMaxOutliers = 16;
 
 __global__ void quantize_weight_rows_kernel(const __half* W, int N, int K, int8_t* Wq,
                                             float* w_scale);
@@ -72,9 +68,6 @@ struct GemmArgs {
   const int8_t* Wq;           // [N][K]
   const __half* X_O;          // [M][ld] compacted outlier columns of X (or nullptr)
   const __half* W_O;          // [N][ld] compacted outlier columns of W (or nullptr)
-  const __half* X;            // [M][K] fp16 activations (outlier values, few outliers)
-  const __half* W;            // [N][K] fp16 weight (outlier values, few outliers)
-  const int32_t* col_idx;     // ascending outlier columns
   int ld;                     // row stride of the panels, multiple of 64
   const float* x_scale;       // [M]
   const float* w_scale;       // [N]
