@@ -280,16 +280,22 @@ def n_sets_for(w, l2_bytes):
 # summaries and their commands are in profiles/. A kernel changed since its
 # capture has no entry (its traffic is reported as null).
 NCU_TRAFFIC = {
+    ("gemm", "llama-70b-ffn-prefill"): {
+        "bytes": 371393280 + 217390848,
+        "source": "profiles/gemm_i8_persistent_llama-70b-ffn-prefill.md"},
+    ("quantize", "llama-70b-ffn-prefill"): {
+        "bytes": 96364032 + 7122688,
+        "source": "profiles/detect_quantize_compact_llama-70b-ffn-prefill.md"},
     ("gemm", "opt-6.7b-ffn-up-prefill"): {
-        "bytes": 78.027008e6 + 34.86208e6,
+        "bytes": 80.357632e6 + 37.069568e6,
         "source": "profiles/gemm_i8_persistent_opt-6.7b-ffn-up-prefill.md"},
     ("quantize", "opt-6.7b-ffn-up-prefill"): {
-        "bytes": 27.326976e6 + 1.792e3,
+        "bytes": 27.340544e6 + 3.072e3,
         "source": "profiles/detect_quantize_compact_opt-6.7b-ffn-up-prefill.md"},
     ("rotate", "opt-6.7b-ffn-up-prefill"): {
         "bytes": 16.804608e6, "source": "profiles/rotate_rows_opt-6.7b-ffn-up-prefill.md"},
     ("decode", "decode"): {
-        "bytes": 19.596544e6, "source": "profiles/decode_kernel_decode-16x4096x4096.md"},
+        "bytes": 19.60192e6, "source": "profiles/decode_kernel_decode-16x4096x4096.md"},
 }
 
 
@@ -359,9 +365,11 @@ def measure_prefill(w, args, stream, l2, pk, X=None, W=None, steps=None):
             "value": round(ops / (ms / 1e3) / 1e12, 2), "unit": "TOPS",
             "frac_of_peak": round(ops / (ms / 1e3) / 1e12 / peak, 4),
             "peak": ("fp16 dense = measured bf16 burst" if fp16 else "int8 dense = 2 x measured bf16 burst"),
-            "gemm": {"ms": g_ms, "achieved": round(gt, 2), "frac": round(gt / peak, 4)},
+            "gemm": {"ms": g_ms, "achieved": round(gt, 2), "frac": round(gt / peak, 4),
+                     "traffic": traffic("gemm", w.name)[0]},
             "quantize": {"ms": q_ms, "achieved_gbs": round(qb / (q_ms / 1e3) / 1e9, 1),
-                         "algorithmic_bytes": qb, "frac_of_hbm": round(qb / (q_ms / 1e3) / 1e9 / pk.hbm, 4)},
+                         "algorithmic_bytes": qb, "frac_of_hbm": round(qb / (q_ms / 1e3) / 1e9 / pk.hbm, 4),
+                         "traffic": traffic("quantize", w.name)[0]},
             "calls_timed": n}
 
 
