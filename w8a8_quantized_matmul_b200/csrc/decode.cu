@@ -74,6 +74,7 @@ constexpr int kStatusTimeout = -5;
 // Named barriers (0 is __syncthreads).
 constexpr uint32_t kBarX = 1;       // the X workers
 constexpr uint32_t kBarList = 2;    // the first X warp publishes the outlier list to warps 4-7
+constexpr uint32_t kBarCodes = 3;   // the X workers' codes are in the B operand (MMA warps wait)
 
 // Shared-memory layout for nbox Wq boxes per CTA (offsets from a 1024-byte
 // aligned base).
@@ -164,8 +165,8 @@ __global__ void __launch_bounds__(64 + 32 * kMaxXWarps, 1)
   if (tid == 0) {
     for (int b = 0; b < kMaxBoxes; ++b) mbar_init(&full[b], 1);
     mbar_init(xbar, 1);
-    for (int b = 0; b < kMaxBoxes; ++b) mbar_init(&cbar[b], 2);   // the two warps of a block
-    mbar_init(done, 1);
+
+    mbar_init(done, 2);   // the two MMA-issuing warps commit
     mbar_init(xchg, 1);
     mbar_init(redbar, 1);
     // The peers' stores are counted in bytes; the one local arrival is made now.
@@ -198,29 +199,33 @@ __global__ void __launch_bounds__(64 + 32 * kMaxXWarps, 1)
   const uint32_t tmem = *tslot;
   bool ok = true;
 
-  if (warp == 0) {
+  if (warp <= 1) {
+    // ---------------------------------------------------------------- MMA issuers
+    // Two warps issue the MMAs, each into its own 16-column TMEM accumulator:
+    // warp 1 the first ceil(nb/2) K-blocks, warp 0 the rest (one issuing lane
+    // of a converged warp issues an MMA every few tens of cycles; two halve the
+    // issue time). The epilogue adds the two accumulators.
     cluster_wait();
-    cluster_arrive();
-  } else if (warp == 1) {
-    // ---------------------------------------------------------------- MMA issuer
-    cluster_wait();
+    const int half = nb - nb / 2;
+    const int b_lo = warp == 1 ? 0 : half;
+    const int b_hi = warp == 1 ? half : nb;
+    const uint32_t acc = tmem + (warp == 1 ? 0u : static_cast<uint32_t>(kTok));
+    // The X workers' code stores are fenced to the async proxy and released
+    // through named barrier kBarCodes (a thread sync); the Wq boxes come from
+    // TMA and need only their mbarrier.
+    named_bar_sync(kBarCodes, 64 + nxt);
+    tc_fence_after();
     constexpr uint32_t idesc = make_idesc(2 /*s32*/, 1 /*signed*/, kTileRows, kTok);
     const uint64_t a0 = sw128_kmajor_desc(smem_addr(ring));
     const uint64_t b0 = sw128_kmajor_desc(smem_addr(bop));
-    // All the codes first, then one tcgen05 fence: a fence per K-block costs
-    // more in MMA issue than waiting for the last block's codes.
-    for (int b = 0; b < nb && ok; ++b) ok = __all_sync(0xffffffffu, mbar_wait(&cbar[b], 0));
-    // Orders the MMAs after the X workers' code stores (a thread sync). The
-    // Wq boxes come from TMA and need only their mbarrier.
-    tc_fence_after();
-    for (int b = 0; b < nb && ok; ++b) {
+    for (int b = b_lo; b < b_hi && ok; ++b) {
       ok = __all_sync(0xffffffffu, mbar_wait(&full[b], 0));
       if (!ok) break;
 #pragma unroll
       for (int kk = 0; kk < 4; ++kk)
-        mma_i8_elect(tmem, a0 + static_cast<uint64_t>((b * kBoxBytes + 32 * kk) >> 4),
+        mma_i8_elect(acc, a0 + static_cast<uint64_t>((b * kBoxBytes + 32 * kk) >> 4),
                      b0 + static_cast<uint64_t>((b * kTok * kKB + 32 * kk) >> 4), idesc,
-                     (b | kk) != 0);
+                     ((b - b_lo) | kk) != 0);
     }
     // Always committed, so the epilogue's wait ends even after a failed wait here.
     mma_commit_elect(done);
@@ -377,7 +382,9 @@ __global__ void __launch_bounds__(64 + 32 * kMaxXWarps, 1)
       wsr = (n < N) ? a.w_scale[n] : 0.0f;
     }
 
-    // Token absmax over the whole cluster, its inverse, the outlier prefix.
+    // Token absmax over the whole cluster, its inverse, the outlier prefix
+    // (for the epilogue, x_scale and the outlier list; the code warps take
+    // their tokens' absmax from the messages themselves).
     ok = __all_sync(0xffffffffu, mbar_wait(xchg, 0)) && ok;
     if (xw == 0) {
       if (lane < kTok) {
@@ -399,18 +406,9 @@ __global__ void __launch_bounds__(64 + 32 * kMaxXWarps, 1)
         if (writer && rank == 0) *a.n_outliers = total;
       }
     }
-    named_bar_sync(kBarX, nxt);
-
-    if (writer) {
-      if (xi < ((kw + 31) >> 5)) a.bitmap[(k0 >> 5) + xi] = bits[xi];
-      const int lc = misc[0], prefix = misc[1];
-      for (int i = xi; i < lc; i += nxt) a.col_idx[prefix + i] = k0 + lidx[i];
-    }
-
     // INT8 codes into the B operand (and Xq): thread xi takes K-block
-    // b = xi / 64 (two warps per block, each block with its own barrier), group
-    // gi = xi % 16 of the block's 16, and the tokens 4tc .. 4tc+3,
-    // tc = (xi / 16) % 4.
+    // b = xi / 64, group gi = xi % 16 of the block's 16, and the tokens
+    // 4tc .. 4tc+3, tc = (xi / 16) % 4.
     {
       const int b = xi >> 6;
       const int gi = xi & 15;
@@ -427,7 +425,9 @@ __global__ void __launch_bounds__(64 + 32 * kMaxXWarps, 1)
           const int t = 4 * tc + j;
           uint2 qv = make_uint2(0u, 0u);
           if (live && t < M) {
-            qv = codes8(xg[t * xvs], amax_s[t], ra_s[t]);
+            float am = 0.0f;
+            for (int s2 = 0; s2 < S; ++s2) am = fmaxf(am, __uint_as_float(msg[s2 * kMsgWords + t]));
+            qv = codes8(xg[t * xvs], am, quant_rcp(am));
             if (m8) {
               qv.x &= keep_bytes(m8 & 0xFu);
               qv.y &= keep_bytes(m8 >> 4);
@@ -440,9 +440,15 @@ __global__ void __launch_bounds__(64 + 32 * kMaxXWarps, 1)
           *reinterpret_cast<uint2*>(dst + off) = qv;
         }
         fence_proxy_async_smem();   // the tensor core reads what the generic proxy wrote
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&cbar[b]);
       }
+    }
+    named_bar_arrive(kBarCodes, 64 + nxt);
+    named_bar_sync(kBarX, nxt);   // amax_s, rs_s and the prefix of the first X warp
+
+    if (writer) {
+      if (xi < ((kw + 31) >> 5)) a.bitmap[(k0 >> 5) + xi] = bits[xi];
+      const int lc = misc[0], prefix = misc[1];
+      for (int i = xi; i < lc; i += nxt) a.col_idx[prefix + i] = k0 + lidx[i];
     }
 
     if (!epi) {
@@ -474,6 +480,14 @@ __global__ void __launch_bounds__(64 + 32 * kMaxXWarps, 1)
       if (got) {
         tc_fence_after();
         tmem_ld_32x32b_x16(tmem + (static_cast<uint32_t>(q * 32) << 16), acc);
+        if (nb >= 2) {
+          uint32_t acc2[kTok];
+          tmem_ld_32x32b_x16(tmem + (static_cast<uint32_t>(q * 32) << 16) + kTok, acc2);
+          tmem_ld_wait();
+#pragma unroll
+          for (int t = 0; t < kTok; ++t)
+            acc[t] = static_cast<uint32_t>(static_cast<int32_t>(acc[t]) + static_cast<int32_t>(acc2[t]));
+        }
         tmem_ld_wait();
       } else {
 #pragma unroll

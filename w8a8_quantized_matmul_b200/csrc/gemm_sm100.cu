@@ -182,7 +182,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int count = (!OUT_I32 && n_outliers) ? *n_outliers : 0;
   const bool tc_out = count > 0;               // outlier product on the tensor cores
-  const int nk = (K + KB_I8 - 1) / KB_I8;
+  // With every column an outlier (threshold 0 on data without zeros) all INT8
+  // codes and row scales are 0: the INT8 K-blocks are skipped and the epilogue
+  // takes C_i32 as 0.
+  const bool no_i8 = !OUT_I32 && count >= K;
+  const int nk = no_i8 ? 0 : (K + KB_I8 - 1) / KB_I8;
   const int np = tc_out ? (count + KB_F16 - 1) / KB_F16 : 0;
   const int iters = nk + np;
 
@@ -361,7 +365,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           // per-row condition (tc_out and ok are uniform across the warp).
           uint32_t acc[16];
           uint32_t oacc[TC ? 16 : 1];
-          tmem_ld_32x32b_x16(lane_base + buf * BN + c, acc);
+          if (!no_i8) {
+            tmem_ld_32x32b_x16(lane_base + buf * BN + c, acc);
+          } else {
+#pragma unroll
+            for (int j = 0; j < 16; ++j) acc[j] = 0u;
+          }
           if constexpr (TC) tmem_ld_32x32b_x16(lane_base + BN + c, oacc);
           tmem_ld_wait();
           const int col0 = n0 + c;
