@@ -45,7 +45,10 @@ def test_topk_parity_opt_like(k):
     _check(X, W, k)
 
 
-@pytest.mark.parametrize("case", [(300, 1040, 136, 3, 10), (17, 512, 200, 2, 5), (129, 272, 264, 0, 3)])
+# K up to 8192 takes the rank select, larger K the one-CTA radix select: both sides of the switch.
+@pytest.mark.parametrize("case", [(300, 1040, 136, 3, 10), (17, 512, 200, 2, 5), (129, 272, 264, 0, 3),
+                                  (40, 8192, 136, 4, 82), (40, 8208, 136, 4, 82),
+                                  (40, 20480, 136, 0, 400)])
 def test_topk_parity_shapes(case):
     M, K, N, n_out, k = case
     X, W, _ = synth.random_case(M, K, N, n_out, seed=M + K + N)
@@ -68,3 +71,13 @@ def test_k0_equals_threshold_inf():
     Yk, _ = m.int8_mixed_matmul_topk(Xd, Wq, ws, Wd, 0)
     Yi, _ = m.int8_mixed_matmul(Xd, Wq, ws, Wd, float("inf"))
     assert torch.equal(Yk, Yi)
+
+
+def test_topk_ties_go_to_lower_index_radix_select():
+    X, W, _ = synth.random_case(32, 20480, 128, 0, seed=19)
+    X[:, :] = np.clip(X, -1.0, 1.0)
+    X[1, 18000:18100] = 3.0      # 100 tied columns, high in K
+    X[2, 50:60] = 3.0            # 10 more, low in K
+    _check(X, W, 30)             # 50..59, then 18000..18019
+    mask = oracle.find_topk_cols(X, 30)
+    assert np.nonzero(mask)[0].tolist() == list(range(50, 60)) + list(range(18000, 18020))

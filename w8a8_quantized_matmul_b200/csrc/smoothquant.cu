@@ -68,13 +68,23 @@ __global__ void __launch_bounds__(kThreads) column_absmax_kernel(const __half* _
 #pragma unroll
   for (int i = 0; i < 4; ++i) m[i] = __float2half2_rn(0.0f);
   if (live) {
-    for (int r = r0 + rl; r < r1; r += 8) {
-      const uint4 u = __ldg(reinterpret_cast<const uint4*>(X + static_cast<size_t>(r) * K) + v);
-      const uint32_t* w = reinterpret_cast<const uint32_t*>(&u);
+    // Four rows' loads in flight per thread (independent), then their maxima.
+    const uint4* col = reinterpret_cast<const uint4*>(X) + v;
+    const size_t rstride = static_cast<size_t>(K) / 8;
+    for (int r = r0 + rl; r < r1; r += 32) {
+      uint4 u[4];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const uint32_t ab = w[i] & 0x7FFF7FFFu;
-        m[i] = __hmax2(m[i], *reinterpret_cast<const __half2*>(&ab));
+      for (int j = 0; j < 4; ++j)
+        u[j] = (r + 8 * j < r1) ? __ldg(col + static_cast<size_t>(r + 8 * j) * rstride)
+                                : make_uint4(0, 0, 0, 0);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const uint32_t* w = reinterpret_cast<const uint32_t*>(&u[j]);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const uint32_t ab = w[i] & 0x7FFF7FFFu;
+          m[i] = __hmax2(m[i], *reinterpret_cast<const __half2*>(&ab));
+        }
       }
     }
   }
@@ -198,8 +208,9 @@ cudaError_t launch_column_absmax(const __half* X, int rows, int K, float* colmax
                                  cudaStream_t s) {
   const int nv = K / 8;
   const int col_blocks = (nv + 31) / 32;
-  // about four CTAs per SM over the whole matrix, at least 8 rows per slice
-  int slices = (4 * 148 + col_blocks - 1) / col_blocks;
+  // about two CTAs per SM over the whole matrix (fewer slices, fewer atomics),
+  // at least 8 rows per slice
+  int slices = (2 * 148 + col_blocks - 1) / col_blocks;
   int row_slice = (rows + slices - 1) / slices;
   row_slice = row_slice < 8 ? 8 : row_slice;
   dim3 grid(col_blocks, (rows + row_slice - 1) / row_slice);

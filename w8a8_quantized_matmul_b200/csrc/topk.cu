@@ -3,8 +3,10 @@
 // FP16): the outlier set is the k columns with the largest max |x| over the
 // tokens, ties to the lower column index.
 //
-// One CTA: radix select of the k-th largest key over the column maxima (fp32
-// >= 0, whose bit patterns order like the values), held in registers; four
+// Up to 8192 columns each column is ranked against all others across the grid
+// and selected when its rank is below k. Beyond, one CTA runs a radix select
+// of the k-th largest key over the column maxima (fp32 >= 0, whose bit
+// patterns order like the values), held in registers; four
 // passes of 8-bit digits, each a shared-memory histogram (one atomic per
 // distinct digit per warp) and a warp scan of its 256 bins; then every key
 // above the k-th is selected, and of the keys equal to it the ones with the
@@ -150,11 +152,76 @@ __global__ void __launch_bounds__(kThreads) topk_select_kernel(const float* __re
   for (int w = tid; w < nw; w += kThreads) bitmap[w] = words[w];
 }
 
+// Up to kRankMax columns, by ranks: column i is selected when fewer than k
+// columns come before it in the order (key descending, column ascending), i.e.
+// when #{j : key_j > key_i} + #{j < i : key_j == key_i} < k, key the bit pattern
+// of the column maximum (non-negative fp32 orders like its bits). Every CTA
+// stages all K keys in shared memory and ranks 32 columns, the ones of one
+// bitmap word: lane l of each warp holds column 32*blockIdx + l and counts over
+// a sixteenth of the j range (broadcast reads, four keys per load); the sixteen
+// partial counts are summed and the word is written whole. K*K comparisons over
+// the grid replace the one-CTA passes of the radix select.
+constexpr int kRankMax = 8192;
+constexpr int kRankThreads = 512;
+constexpr int kRankWarps = kRankThreads / 32;
+
+__global__ void __launch_bounds__(kRankThreads) topk_rank_kernel(const float* __restrict__ colmax,
+                                                                 int K, int k,
+                                                                 uint32_t* __restrict__ bitmap) {
+  __shared__ __align__(16) unsigned int keys[kRankMax];
+  __shared__ unsigned int part[kRankWarps][32];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int K4 = (K + 3) & ~3;   // keys padded with 0, which never count (see below)
+  for (int j = tid; j < K4; j += kRankThreads)
+    keys[j] = j < K ? __float_as_uint(__ldg(colmax + j)) : 0u;
+  __syncthreads();
+  const int base = 32 * blockIdx.x;
+  const int i = base + lane;
+  const unsigned int ki = i < K ? keys[i] : 0u;
+  // this warp's share of j, a multiple of 4 long
+  const int span = ((K4 / 4 + kRankWarps - 1) / kRankWarps) * 4;
+  const int j0 = warp * span;
+  const int j1 = min(j0 + span, K4);
+  unsigned int c = 0u;
+  // A padded key (0, at j >= K > i) never counts: 0 > ki is false and j < i is false.
+  if (j1 <= base) {
+    // every j < i: ties count
+    for (int j = j0; j < j1; j += 4) {
+      const uint4 v = *reinterpret_cast<const uint4*>(keys + j);
+      c += (v.x >= ki) + (v.y >= ki) + (v.z >= ki) + (v.w >= ki);
+    }
+  } else if (j0 >= base + 32) {
+    // every j > i: only larger keys count
+    for (int j = j0; j < j1; j += 4) {
+      const uint4 v = *reinterpret_cast<const uint4*>(keys + j);
+      c += (v.x > ki) + (v.y > ki) + (v.z > ki) + (v.w > ki);
+    }
+  } else {
+    for (int j = j0; j < j1; ++j) {
+      const unsigned int kj = keys[j];
+      c += (kj > ki) || (kj == ki && j < i);
+    }
+  }
+  part[warp][lane] = c;
+  __syncthreads();
+  if (warp == 0) {
+    unsigned int r = 0u;
+#pragma unroll
+    for (int w = 0; w < kRankWarps; ++w) r += part[w][lane];
+    const unsigned int word = __ballot_sync(0xffffffffu, i < K && r < static_cast<unsigned int>(k));
+    if (lane == 0) bitmap[blockIdx.x] = word;
+  }
+}
+
 }  // namespace
 
 cudaError_t launch_topk_select(const float* colmax, int K, int k, uint32_t* bitmap,
                                cudaStream_t s) {
   if (K <= 0 || K > 65536) return cudaErrorInvalidValue;
+  if (K <= kRankMax) {
+    topk_rank_kernel<<<(K + 31) / 32, kRankThreads, 0, s>>>(colmax, K, k < 0 ? 0 : k, bitmap);
+    return cudaGetLastError();
+  }
   if (K <= 4 * kThreads)
     topk_select_kernel<4><<<1, kThreads, 0, s>>>(colmax, K, k, bitmap);
   else if (K <= 16 * kThreads)
