@@ -16,7 +16,9 @@
  *     caller. The library never allocates or frees device memory.
  *   - Matrices are row-major and dense (row stride = number of columns):
  *     X [M][K] fp16, W [N][K] fp16 (out-features x in-features), Wq [N][K]
- *     int8, Y [M][N] fp16. fp16 is IEEE binary16, passed as `const void*`.
+ *     int8, Y [M][N] fp16; the mixed-matmul entry points take the fp16
+ *     weight transposed, Wt [K][N] (see int8_transpose_weight). fp16 is IEEE
+ *     binary16, passed as `const void*`.
  *   - Every call is asynchronous on `stream` (a cudaStream_t; NULL = the
  *     legacy default stream) and does no host synchronisation. Device-side
  *     results such as the outlier count stay on the device.
@@ -71,6 +73,19 @@ int int8_quantize_weight_rows(const void* W, int N, int K, int8_t* Wq, float* w_
                               i8mm_stream_t stream);
 
 /*
+ * Offline layout of the fp16 weight for the outlier product: Wt[k][n] = W[n][k].
+ * AIInfra LLM.int8() section: W is h x o (input features x outputs) and the
+ * outlier term multiplies the rows W^h of the outlier dimensions h, which are
+ * contiguous rows of Wt. The mixed-matmul entry points take this Wt.
+ *   W   in : fp16 [N][K] (out features x in features, the PyTorch Linear layout)
+ *   Wt  out: fp16 [K][N]; must not overlap W
+ * Errors: I8MM_ERR_INVALID_ARG (null pointer, bad sizes), I8MM_ERR_ALIGNMENT
+ * (pointers not 16-byte aligned or K not a multiple of 16), I8MM_ERR_CUDA.
+ * Off the per-call hot path, like int8_quantize_weight_rows.
+ */
+int int8_transpose_weight(const void* W, int N, int K, void* Wt, i8mm_stream_t stream);
+
+/*
  * Outlier feature-column detection (AIInfra LLM.int8() section, "detection:
  * set a magnitude threshold"; tanjunchen section 1.2: a channel whose
  * activation magnitude exceeds the threshold, 6.0 by default).
@@ -107,8 +122,9 @@ size_t int8_mixed_matmul_workspace_size(int M, int N, int K);
  * caller or a test read the outlier set, codes and scales of the last call.
  * The outlier panels have row stride panel_ld elements (fp16) and hold the
  * compacted outlier columns in ascending column order, zero-padded to a
- * multiple of 64 columns (the GEMM multiplies them on the tensor cores).
- * Nothing is written to them when there are no outliers.
+ * multiple of 16 columns (one K step of the tensor-core outlier product; the
+ * zero-point and given-set paths pad to 64). Columns past the padding are
+ * never read. Nothing is written to them when there are no outliers.
  */
 typedef struct {
   size_t n_outliers;   /* int32 [1] */
@@ -131,8 +147,11 @@ int int8_mixed_matmul_workspace_layout(int M, int N, int K, i8mm_workspace_layou
  * C_f16 = C_outlier + C_normal).
  *   X          in : fp16 [M][K] activations
  *   Wq,w_scale in : from int8_quantize_weight_rows
- *   W_fp16     in : fp16 [N][K], the unquantised weight; only its outlier
- *                   columns are read
+ *   Wt_fp16    in : fp16 [K][N], the unquantised weight in the pages' h x o
+ *                   orientation (row k holds input feature k for every output
+ *                   n; int8_transpose_weight makes it from the [N][K] weight
+ *                   once, offline); only the rows of the outlier features are
+ *                   read, each contiguously
  *   threshold  in : outlier magnitude threshold (6.0 in the pages)
  *   Y          out: fp16 [M][N], Y = fp16(C_i32*x_scale*w_scale/127^2 + C_outlier),
  *                   the sum formed in fp32 and rounded once
@@ -142,7 +161,7 @@ int int8_mixed_matmul_workspace_layout(int M, int N, int K, i8mm_workspace_layou
  * back to back on `stream`; the outlier count never leaves the device.
  */
 int int8_mixed_matmul(const void* X, const int8_t* Wq, const float* w_scale,
-                      const void* W_fp16, int M, int N, int K, float threshold, void* Y,
+                      const void* Wt_fp16, int M, int N, int K, float threshold, void* Y,
                       void* workspace, size_t workspace_bytes, i8mm_stream_t stream);
 
 /*
@@ -155,7 +174,7 @@ int int8_mixed_matmul(const void* X, const int8_t* Wq, const float* w_scale,
  * device durations of the memory-bound stage and of the tensor-core GEMM.
  */
 int int8_mixed_matmul_profiled(const void* X, const int8_t* Wq, const float* w_scale,
-                               const void* W_fp16, int M, int N, int K, float threshold,
+                               const void* Wt_fp16, int M, int N, int K, float threshold,
                                void* Y, void* workspace, size_t workspace_bytes,
                                i8mm_stream_t stream, void* const* events);
 
@@ -181,7 +200,7 @@ int int8_weight_rowsum(const int8_t* Wq, int N, int K, int32_t* rowsum, i8mm_str
 // aligned). Always runs the prefill kernels.
 size_t int8_mixed_matmul_zp_workspace_size(int M, int N, int K);
 int int8_mixed_matmul_zp(const void* X, const int8_t* Wq, const float* w_scale,
-                         const int32_t* w_rowsum, const void* W_fp16, int M, int N, int K,
+                         const int32_t* w_rowsum, const void* Wt_fp16, int M, int N, int K,
                          float threshold, void* Y, void* workspace, size_t workspace_bytes,
                          i8mm_stream_t stream);
 
@@ -197,7 +216,7 @@ int int8_mixed_matmul_zp(const void* X, const int8_t* Wq, const float* w_scale,
 // count and list describe the selected set. Always runs the prefill kernels.
 size_t int8_mixed_matmul_topk_workspace_size(int M, int N, int K);
 int int8_mixed_matmul_topk(const void* X, const int8_t* Wq, const float* w_scale,
-                           const void* W_fp16, int M, int N, int K, int k, void* Y,
+                           const void* Wt_fp16, int M, int N, int K, int k, void* Y,
                            void* workspace, size_t workspace_bytes, i8mm_stream_t stream);
 
 // ---------------------------------------------------------------- SmoothQuant W8A8
@@ -319,7 +338,7 @@ int int4_rotated_matmul(const void* X, const int8_t* Wq4, const float* w_absmax,
 //   other arguments, layout, workspace and errors as int8_mixed_matmul; the
 //   workspace's bitmap holds the OR afterwards. Always runs the prefill kernels.
 int int8_mixed_matmul_sharded(const void* X, const int8_t* Wq, const float* w_scale,
-                              const void* W_fp16, int M, int N, int K, const uint32_t* bitmaps,
+                              const void* Wt_fp16, int M, int N, int K, const uint32_t* bitmaps,
                               int n_bitmaps, void* Y, void* workspace, size_t workspace_bytes,
                               i8mm_stream_t stream);
 
@@ -335,7 +354,7 @@ int int8_mixed_matmul_sharded(const void* X, const int8_t* Wq, const float* w_sc
  * I8MM_ERR_INVALID_ARG.
  */
 int int8_mixed_matmul_stage(int stage, const void* X, const int8_t* Wq, const float* w_scale,
-                            const void* W_fp16, int M, int N, int K, float threshold, void* Y,
+                            const void* Wt_fp16, int M, int N, int K, float threshold, void* Y,
                             void* workspace, size_t workspace_bytes, i8mm_stream_t stream);
 
 /*
@@ -391,7 +410,7 @@ int int8_device_status(const void* workspace, i8mm_stream_t stream);
  */
 #define I8MM_NOALLOC_SCRATCH_BYTES ((size_t)64 << 20)
 int int8_mixed_matmul_noalloc(const void* X, const int8_t* Wq, const float* w_scale,
-                              const void* W_fp16, int M, int N, int K, float threshold,
+                              const void* Wt_fp16, int M, int N, int K, float threshold,
                               void* Y, i8mm_stream_t stream);
 
 /*

@@ -36,6 +36,11 @@ def mm():
     return m
 
 
+def wt(W):
+    """The fp16 weight in the transposed [K][N] layout the mixed-matmul calls take."""
+    return mm().int8_transpose_weight(W)
+
+
 def dev(a):
     return torch.from_numpy(np.ascontiguousarray(a)).cuda()
 
@@ -60,7 +65,7 @@ def run_mixed(X, W, thr):
     m = mm()
     Xd, Wd = dev(X), dev(W)
     Wq, ws = m.int8_quantize_weight_rows(Wd)
-    Y, work = m.int8_mixed_matmul(Xd, Wq, ws, Wd, thr)
+    Y, work = m.int8_mixed_matmul(Xd, Wq, ws, wt(Wd), thr)
     views = m.workspace_views(work, X.shape[0], W.shape[0], X.shape[1])
     out = {k: host(v) for k, v in views.items()}
     assert m.int8_device_status(work) == 0
@@ -77,11 +82,12 @@ def check_intermediates(ref, got, K):
 
 
 def check_panels(X, W, ref, got):
-    """Compacted fp16 outlier panels, 64-padded (the tensor-core outlier product)."""
+    """Compacted fp16 outlier panels, zero-padded to a multiple of 16 columns
+    (one kind::f16 K step; the GEMM multiplies only the steps that hold columns)."""
     count = ref["count"]
     if count == 0 or X.shape[0] <= 16:   # no panels (or the decode path)
         return
-    pad = (count + 63) // 64 * 64
+    pad = (count + 15) // 16 * 16
     idx = ref["idx"]
     assert np.array_equal(got["X_O"][:, :count], X[:, idx])
     assert np.all(got["X_O"][:, count:pad] == 0)
@@ -98,6 +104,16 @@ def test_quantize_weight_rows_bitexact(N, K):
     rq, rs = oracle.quantize_weight_rows(W)
     assert np.array_equal(host(Wq), rq)
     assert np.array_equal(host(ws).view(np.uint32), rs.view(np.uint32))
+
+
+# ---------------------------------------------------------------- weight layout
+@pytest.mark.parametrize("N,K", [(256, 256), (33, 48), (1, 16), (129, 4096), (70000, 16), (8, 12288)])
+def test_transpose_weight_exact(N, K):
+    """int8_transpose_weight gives W^T element for element (ragged tiles included)."""
+    W = synth.make_weight(N, K, 0.02, seed=N * 3 + K)
+    Wt = mm().int8_transpose_weight(dev(W))
+    assert tuple(Wt.shape) == (K, N)
+    assert np.array_equal(host(Wt).view(np.uint16), np.ascontiguousarray(W.T).view(np.uint16))
 
 
 # ---------------------------------------------------------------- detection
@@ -272,7 +288,7 @@ def test_mixed_matmul_guard_bands():
     need = m.int8_mixed_matmul_workspace_size(M, N, K)
     wbuf = torch.full((2 * G + need,), 0x5A, dtype=torch.uint8, device="cuda")
     work = wbuf[G:G + need]
-    m.int8_mixed_matmul(Xd, Wq, ws, Wd, 6.0, Y=Y, workspace=work)
+    m.int8_mixed_matmul(Xd, Wq, ws, wt(Wd), 6.0, Y=Y, workspace=work)
     yb = host(ybuf)
     wb = host(wbuf)
     assert np.all(yb[:G] == 0xA5) and np.all(yb[G + M * N * 2:] == 0xA5)
@@ -287,9 +303,9 @@ def test_mixed_matmul_repeated_calls_reuse_workspace():
     X2, _, _ = synth.random_case(150, 512, 200, 9, seed=22)
     Wd = dev(W)
     Wq, ws = m.int8_quantize_weight_rows(Wd)
-    Y1, work = m.int8_mixed_matmul(dev(X1), Wq, ws, Wd, 6.0)
+    Y1, work = m.int8_mixed_matmul(dev(X1), Wq, ws, wt(Wd), 6.0)
     y1 = host(Y1).copy()
-    Y2, _ = m.int8_mixed_matmul(dev(X2), Wq, ws, Wd, 6.0, workspace=work)
+    Y2, _ = m.int8_mixed_matmul(dev(X2), Wq, ws, wt(Wd), 6.0, workspace=work)
     assert_y_close(host(Y2), oracle.llm_int8_matmul(X2, W, 6.0)["Y"], "second call")
     assert_y_close(y1, oracle.llm_int8_matmul(X1, W, 6.0)["Y"], "first call")
 
@@ -300,14 +316,14 @@ def test_stage_hook_reproduces_full_call():
     X, W, _ = synth.random_case(300, 1024, 520, 6, seed=31)
     Xd, Wd = dev(X), dev(W)
     Wq, ws = m.int8_quantize_weight_rows(Wd)
-    Y1, work = m.int8_mixed_matmul(Xd, Wq, ws, Wd, 6.0)
+    Y1, work = m.int8_mixed_matmul(Xd, Wq, ws, wt(Wd), 6.0)
     y1 = host(Y1).copy()
     Y2 = torch.zeros_like(Y1)
     work2 = torch.zeros_like(work)
-    m.int8_mixed_matmul_stage(1, Xd, Wq, ws, Wd, 6.0, Y2, work2)
-    m.int8_mixed_matmul_stage(2, Xd, Wq, ws, Wd, 6.0, Y2, work2)
+    m.int8_mixed_matmul_stage(1, Xd, Wq, ws, wt(Wd), 6.0, Y2, work2)
+    m.int8_mixed_matmul_stage(2, Xd, Wq, ws, wt(Wd), 6.0, Y2, work2)
     assert np.array_equal(host(Y2), y1)
-    m.int8_mixed_matmul_stage(2, Xd, Wq, ws, Wd, 6.0, Y2, work2)   # GEMM alone again
+    m.int8_mixed_matmul_stage(2, Xd, Wq, ws, wt(Wd), 6.0, Y2, work2)   # GEMM alone again
     assert np.array_equal(host(Y2), y1)
 
 
@@ -316,7 +332,7 @@ def test_empty_problem_is_a_noop():
     W = dev(synth.make_weight(64, 64, 0.02, seed=1))
     Wq, ws = m.int8_quantize_weight_rows(W)
     X = torch.empty((0, 64), dtype=torch.float16, device="cuda")
-    Y, _ = m.int8_mixed_matmul(X, Wq, ws, W, 6.0)
+    Y, _ = m.int8_mixed_matmul(X, Wq, ws, wt(W), 6.0)
     assert tuple(Y.shape) == (0, 64)
 
 

@@ -17,6 +17,11 @@ import w8a8_quantized_matmul_b200 as m
 
 pytestmark = pytest.mark.gpu
 
+
+def wt(W):
+    """The fp16 weight in the transposed [K][N] layout the mixed-matmul calls take."""
+    return m.int8_transpose_weight(W)
+
 CASES = [
     # M, K, N, n_outliers, row bounds of the ranks
     (300, 512, 384, 5, [0, 100, 300]),
@@ -33,13 +38,13 @@ def test_sharded_equals_whole_batch(case):
     Xd = torch.from_numpy(X).cuda()
     Wd = torch.from_numpy(W).cuda()
     Wq, ws = m.int8_quantize_weight_rows(Wd)
-    Y_full, _ = m.int8_mixed_matmul(Xd, Wq, ws, Wd, 6.0)
+    Y_full, _ = m.int8_mixed_matmul(Xd, Wq, ws, wt(Wd), 6.0)
     parts = [Xd[bounds[r]:bounds[r + 1]].contiguous() for r in range(len(bounds) - 1)]
     bitmaps = torch.stack([m.int8_find_outlier_cols(p, 6.0)[0] for p in parts])
     ys = []
     ref = oracle.llm_int8_matmul(X, W)
     for r, p in enumerate(parts):
-        Y, work = m.int8_mixed_matmul_sharded(p, Wq, ws, Wd, bitmaps)
+        Y, work = m.int8_mixed_matmul_sharded(p, Wq, ws, wt(Wd), bitmaps)
         ys.append(Y)
         torch.cuda.synchronize()
         if p.shape[0] == 0:

@@ -12,6 +12,11 @@ import w8a8_quantized_matmul_b200 as m
 
 pytestmark = pytest.mark.gpu
 
+
+def wt(W):
+    """The fp16 weight in the transposed [K][N] layout the mixed-matmul calls take."""
+    return m.int8_transpose_weight(W)
+
 MAX_REL, MEAN_REL = 1e-2, 1e-3
 
 
@@ -20,7 +25,7 @@ def _check(X, W, k):
     N = W.shape[0]
     Xd, Wd = torch.from_numpy(X).cuda(), torch.from_numpy(W).cuda()
     Wq, ws = m.int8_quantize_weight_rows(Wd)
-    Y, work = m.int8_mixed_matmul_topk(Xd, Wq, ws, Wd, k)
+    Y, work = m.int8_mixed_matmul_topk(Xd, Wq, ws, wt(Wd), k)
     torch.cuda.synchronize()
     mask = oracle.find_topk_cols(X, k)
     ref = oracle.llm_int8_matmul(X, W, outlier_mask=mask)
@@ -68,8 +73,8 @@ def test_k0_equals_threshold_inf():
     X, W, _ = synth.random_case(512, 1024, 256, 6, seed=12)
     Xd, Wd = torch.from_numpy(X).cuda(), torch.from_numpy(W).cuda()
     Wq, ws = m.int8_quantize_weight_rows(Wd)
-    Yk, _ = m.int8_mixed_matmul_topk(Xd, Wq, ws, Wd, 0)
-    Yi, _ = m.int8_mixed_matmul(Xd, Wq, ws, Wd, float("inf"))
+    Yk, _ = m.int8_mixed_matmul_topk(Xd, Wq, ws, wt(Wd), 0)
+    Yi, _ = m.int8_mixed_matmul(Xd, Wq, ws, wt(Wd), float("inf"))
     assert torch.equal(Yk, Yi)
 
 

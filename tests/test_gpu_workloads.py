@@ -52,7 +52,7 @@ def test_workload_parity(name):
     Xd = torch.from_numpy(X).cuda()
     Wd = torch.from_numpy(W).cuda()
     Wq, ws = m.int8_quantize_weight_rows(Wd)
-    Y, work = m.int8_mixed_matmul(Xd, Wq, ws, Wd, w.threshold)
+    Y, work = m.int8_mixed_matmul(Xd, Wq, ws, m.int8_transpose_weight(Wd), w.threshold)
     torch.cuda.synchronize()
     assert m.int8_device_status(work) == 0
     views = m.workspace_views(work, w.M, w.N, w.K)

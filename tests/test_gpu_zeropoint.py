@@ -12,6 +12,11 @@ import w8a8_quantized_matmul_b200 as m
 
 pytestmark = pytest.mark.gpu
 
+
+def wt(W):
+    """The fp16 weight in the transposed [K][N] layout the mixed-matmul calls take."""
+    return m.int8_transpose_weight(W)
+
 MAX_REL, MEAN_REL = 1e-2, 1e-3
 
 
@@ -21,7 +26,7 @@ def _run(X, W, thr):
     Xd, Wd = torch.from_numpy(X).cuda(), torch.from_numpy(W).cuda()
     Wq, ws = m.int8_quantize_weight_rows(Wd)
     rsum = m.int8_weight_rowsum(Wq)
-    Y, work = m.int8_mixed_matmul_zp(Xd, Wq, ws, rsum, Wd, thr)
+    Y, work = m.int8_mixed_matmul_zp(Xd, Wq, ws, rsum, wt(Wd), thr)
     torch.cuda.synchronize()
     ref = oracle.llm_int8_matmul(X, W, thr, zeropoint=True)
     np.testing.assert_array_equal(rsum.cpu().numpy(), ref["wsum"])
@@ -65,7 +70,7 @@ def test_one_sided_rows():
     exact = X.astype(np.float64) @ W.astype(np.float64).T
     Xd, Wd = torch.from_numpy(X).cuda(), torch.from_numpy(W).cuda()
     Wq, ws = m.int8_quantize_weight_rows(Wd)
-    Ya, _ = m.int8_mixed_matmul(Xd, Wq, ws, Wd, float("inf"))
+    Ya, _ = m.int8_mixed_matmul(Xd, Wq, ws, wt(Wd), float("inf"))
     e_zp = np.abs(Yz - exact).mean()
     e_abs = np.abs(Ya.cpu().numpy().astype(np.float64) - exact).mean()
     assert e_zp < 0.8 * e_abs

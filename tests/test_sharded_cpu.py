@@ -31,13 +31,13 @@ def _find(X_local, threshold):
     return torch.from_numpy(bitmap.view(np.int32).copy())
 
 
-def _apply(X_local, Wq, w_scale, W, bitmaps, Y=None, workspace=None):
+def _apply(X_local, Wq, w_scale, Wt, bitmaps, Y=None, workspace=None):
     words = bitmaps.numpy().view(np.uint32)
     orw = np.bitwise_or.reduce(words, axis=0)
     K = X_local.shape[1]
     mask = ((orw[np.arange(K) // 32] >> (np.arange(K) % 32).astype(np.uint32)) & 1).astype(bool)
-    out = oracle.llm_int8_matmul(X_local.numpy(), W.numpy(), Wq=Wq.numpy(), w_scale=w_scale.numpy(),
-                                 outlier_mask=mask)
+    out = oracle.llm_int8_matmul(X_local.numpy(), np.ascontiguousarray(Wt.numpy().T), Wq=Wq.numpy(),
+                                 w_scale=w_scale.numpy(), outlier_mask=mask)
     return torch.from_numpy(out["Y"]), torch.from_numpy(orw.view(np.int32).copy())
 
 
@@ -55,7 +55,8 @@ def _worker(rank, world, port, bounds, case, q):
         r0, r1 = bounds[rank], bounds[rank + 1]
         Xl = torch.from_numpy(np.ascontiguousarray(X[r0:r1]))
         Y, orw = token_sharded_mixed_matmul(Xl, torch.from_numpy(Wq), torch.from_numpy(w_scale),
-                                           torch.from_numpy(W), 6.0, find=_find, apply=_apply)
+                                           torch.from_numpy(np.ascontiguousarray(W.T)), 6.0,
+                                           find=_find, apply=_apply)
         q.put((rank, Y.numpy(), orw.numpy()))
     finally:
         dist.destroy_process_group()
@@ -118,7 +119,8 @@ def _failing_worker(rank, world, port, mode, q):
     t0 = time.perf_counter()
     try:
         token_sharded_mixed_matmul(torch.from_numpy(X), torch.from_numpy(Wq),
-                                   torch.from_numpy(w_scale), torch.from_numpy(W), 6.0,
+                                   torch.from_numpy(w_scale),
+                                   torch.from_numpy(np.ascontiguousarray(W.T)), 6.0,
                                    find=_find, apply=_apply)
         msg = ("no error", time.perf_counter() - t0)
     except Exception as e:  # the collective's failure reaches the host as an exception
@@ -145,9 +147,9 @@ def test_lost_rank_ends_the_exchange_with_an_error(mode):
                 p.kill()
 
 
-def _apply_cols(X, Wq_local, w_scale_local, W_local, threshold, Y=None, workspace=None):
-    out = oracle.llm_int8_matmul(X.numpy(), W_local.numpy(), threshold, Wq=Wq_local.numpy(),
-                                 w_scale=w_scale_local.numpy())
+def _apply_cols(X, Wq_local, w_scale_local, Wt_local, threshold, Y=None, workspace=None):
+    out = oracle.llm_int8_matmul(X.numpy(), np.ascontiguousarray(Wt_local.numpy().T), threshold,
+                                 Wq=Wq_local.numpy(), w_scale=w_scale_local.numpy())
     return torch.from_numpy(out["Y"])
 
 
@@ -165,11 +167,11 @@ def _cols_worker(rank, world, port, case, q):
         Wq, w_scale = oracle.quantize_weight_rows(W[n0:n1])
         Y_local = column_sharded_mixed_matmul(torch.from_numpy(X), torch.from_numpy(Wq),
                                               torch.from_numpy(w_scale),
-                                              torch.from_numpy(np.ascontiguousarray(W[n0:n1])),
+                                              torch.from_numpy(np.ascontiguousarray(W[n0:n1].T)),
                                               6.0, apply=_apply_cols)
         Y_full = column_sharded_mixed_matmul(torch.from_numpy(X), torch.from_numpy(Wq),
                                              torch.from_numpy(w_scale),
-                                             torch.from_numpy(np.ascontiguousarray(W[n0:n1])),
+                                             torch.from_numpy(np.ascontiguousarray(W[n0:n1].T)),
                                              6.0, N=N, gather=True, apply=_apply_cols)
         q.put((rank, n0, n1, Y_local.numpy(), Y_full.numpy()))
     finally:

@@ -63,6 +63,9 @@ def _pair(lib, M, K, N, cases):
     stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
     assert lib.int8_quantize_weight_rows(Wd.data_ptr(), N, K, Wq.data_ptr(), ws.data_ptr(),
                                          stream) == 0
+    # The mixed-matmul calls take the fp16 weight transposed, [K][N].
+    Wt = torch.empty((K, N), dtype=torch.float16, device="cuda")
+    assert lib.int8_transpose_weight(Wd.data_ptr(), N, K, Wt.data_ptr(), stream) == 0
     Xs = [torch.from_numpy(X).cuda() for X in Xs_h]
 
     # Regular entry point, caller-provided workspace.
@@ -71,7 +74,7 @@ def _pair(lib, M, K, N, cases):
     refs = []
     for Xd in Xs:
         Y = torch.empty((M, N), dtype=torch.float16, device="cuda")
-        st = lib.int8_mixed_matmul(Xd.data_ptr(), Wq.data_ptr(), ws.data_ptr(), Wd.data_ptr(),
+        st = lib.int8_mixed_matmul(Xd.data_ptr(), Wq.data_ptr(), ws.data_ptr(), Wt.data_ptr(),
                                    M, N, K, 6.0, Y.data_ptr(), work.data_ptr(), need, stream)
         assert st == _lib.I8MM_OK
         refs.append(Y)
@@ -80,7 +83,7 @@ def _pair(lib, M, K, N, cases):
     outs = [torch.full((M, N), float("nan"), dtype=torch.float16, device="cuda") for _ in Xs]
     for Xd, Y in zip(Xs, outs):
         st = lib.int8_mixed_matmul_noalloc(Xd.data_ptr(), Wq.data_ptr(), ws.data_ptr(),
-                                           Wd.data_ptr(), M, N, K, 6.0, Y.data_ptr(), stream)
+                                           Wt.data_ptr(), M, N, K, 6.0, Y.data_ptr(), stream)
         assert st == _lib.I8MM_OK
     assert lib.int8_noalloc_device_status(stream) == _lib.I8MM_OK
     torch.cuda.synchronize()

@@ -29,6 +29,7 @@ from ._lib import (  # noqa: F401
 
 __all__ = [
     "int8_quantize_weight_rows",
+    "int8_transpose_weight",
     "int8_find_outlier_cols",
     "int8_quantize_act_rows",
     "int8_mixed_matmul_workspace_size",
@@ -86,6 +87,17 @@ def int8_quantize_weight_rows(W, Wq=None, w_scale=None, stream=None):
     return Wq, w_scale
 
 
+def int8_transpose_weight(W, Wt=None, stream=None):
+    """W fp16 [N, K] -> Wt fp16 [K, N] (offline layout of the fp16 weight that the
+    mixed-matmul calls read the outlier features from)."""
+    N, K = W.shape
+    _need(W, "W", torch.float16, (N, K))
+    Wt = torch.empty((K, N), dtype=torch.float16, device=W.device) if Wt is None else Wt
+    _need(Wt, "Wt", torch.float16, (K, N))
+    check("int8_transpose_weight", load().int8_transpose_weight(_ptr(W), N, K, _ptr(Wt), _stream(stream)))
+    return Wt
+
+
 def int8_find_outlier_cols(X, threshold=6.0, col_bitmap=None, n_outliers=None, col_idx=None,
                            stream=None):
     """X fp16 [M, K] -> (bitmap uint32-as-int32 [ceil(K/32)], count int32 [1], col_idx int32 [K])."""
@@ -130,27 +142,27 @@ def int8_mixed_matmul_workspace_layout(M: int, N: int, K: int) -> WorkspaceLayou
     return lay
 
 
-def int8_mixed_matmul(X, Wq, w_scale, W_fp16, threshold=6.0, Y=None, workspace=None, stream=None):
+def int8_mixed_matmul(X, Wq, w_scale, Wt_fp16, threshold=6.0, Y=None, workspace=None, stream=None):
     """Y = LLM.int8() decomposition of X . W^T; returns (Y fp16 [M, N], workspace uint8)."""
     M, K = X.shape
     N = Wq.shape[0]
     _need(X, "X", torch.float16, (M, K))
     _need(Wq, "Wq", torch.int8, (N, K))
     _need(w_scale, "w_scale", torch.float32, (N,))
-    _need(W_fp16, "W_fp16", torch.float16, (N, K))
+    _need(Wt_fp16, "Wt_fp16", torch.float16, (K, N))
     Y = torch.empty((M, N), dtype=torch.float16, device=X.device) if Y is None else Y
     _need(Y, "Y", torch.float16, (M, N))
     need = int8_mixed_matmul_workspace_size(M, N, K)
     if workspace is None:
         workspace = torch.empty((max(need, 1),), dtype=torch.uint8, device=X.device)
     check("int8_mixed_matmul",
-          load().int8_mixed_matmul(_ptr(X), _ptr(Wq), _ptr(w_scale), _ptr(W_fp16), M, N, K,
+          load().int8_mixed_matmul(_ptr(X), _ptr(Wq), _ptr(w_scale), _ptr(Wt_fp16), M, N, K,
                                    float(threshold), _ptr(Y), _ptr(workspace),
                                    workspace.numel() * workspace.element_size(), _stream(stream)))
     return Y, workspace
 
 
-def int8_mixed_matmul_profiled(X, Wq, w_scale, W_fp16, threshold, Y, workspace, events,
+def int8_mixed_matmul_profiled(X, Wq, w_scale, Wt_fp16, threshold, Y, workspace, events,
                                stream=None):
     """int8_mixed_matmul that also records three torch.cuda.Event objects on the stream:
     before the call, between the quantisation stage and the GEMM, and after the GEMM."""
@@ -164,26 +176,26 @@ def int8_mixed_matmul_profiled(X, Wq, w_scale, W_fp16, threshold, Y, workspace, 
         handles.append(ev.cuda_event)
     arr = (ctypes.c_void_p * 3)(*handles)
     check("int8_mixed_matmul_profiled",
-          load().int8_mixed_matmul_profiled(_ptr(X), _ptr(Wq), _ptr(w_scale), _ptr(W_fp16), M, N, K,
+          load().int8_mixed_matmul_profiled(_ptr(X), _ptr(Wq), _ptr(w_scale), _ptr(Wt_fp16), M, N, K,
                                             float(threshold), _ptr(Y), _ptr(workspace),
                                             workspace.numel() * workspace.element_size(),
                                             ctypes.c_void_p(s.cuda_stream), arr))
     return Y
 
 
-def int8_mixed_matmul_stage(stage, X, Wq, w_scale, W_fp16, threshold, Y, workspace, stream=None):
+def int8_mixed_matmul_stage(stage, X, Wq, w_scale, Wt_fp16, threshold, Y, workspace, stream=None):
     """One stage of int8_mixed_matmul (1: quantisation kernel, 2: GEMM kernel) for timing."""
     M, K = X.shape
     N = Wq.shape[0]
     check("int8_mixed_matmul_stage",
-          load().int8_mixed_matmul_stage(int(stage), _ptr(X), _ptr(Wq), _ptr(w_scale), _ptr(W_fp16),
+          load().int8_mixed_matmul_stage(int(stage), _ptr(X), _ptr(Wq), _ptr(w_scale), _ptr(Wt_fp16),
                                          M, N, K, float(threshold), _ptr(Y), _ptr(workspace),
                                          workspace.numel() * workspace.element_size(),
                                          _stream(stream)))
     return Y
 
 
-def int8_mixed_matmul_sharded(X, Wq, w_scale, W_fp16, bitmaps, Y=None, workspace=None,
+def int8_mixed_matmul_sharded(X, Wq, w_scale, Wt_fp16, bitmaps, Y=None, workspace=None,
                               stream=None):
     """One rank's part of a token-sharded int8_mixed_matmul.
 
@@ -195,7 +207,7 @@ def int8_mixed_matmul_sharded(X, Wq, w_scale, W_fp16, bitmaps, Y=None, workspace
     _need(X, "X", torch.float16, (M, K))
     _need(Wq, "Wq", torch.int8, (N, K))
     _need(w_scale, "w_scale", torch.float32, (N,))
-    _need(W_fp16, "W_fp16", torch.float16, (N, K))
+    _need(Wt_fp16, "Wt_fp16", torch.float16, (K, N))
     words = (K + 31) // 32
     if bitmaps.dim() != 2:
         raise ValueError("bitmaps must be [n_ranks, ceil(K/32)]")
@@ -206,7 +218,7 @@ def int8_mixed_matmul_sharded(X, Wq, w_scale, W_fp16, bitmaps, Y=None, workspace
     if workspace is None:
         workspace = torch.empty((max(need, 1),), dtype=torch.uint8, device=X.device)
     check("int8_mixed_matmul_sharded",
-          load().int8_mixed_matmul_sharded(_ptr(X), _ptr(Wq), _ptr(w_scale), _ptr(W_fp16), M, N,
+          load().int8_mixed_matmul_sharded(_ptr(X), _ptr(Wq), _ptr(w_scale), _ptr(Wt_fp16), M, N,
                                            K, _ptr(bitmaps), int(bitmaps.shape[0]), _ptr(Y),
                                            _ptr(workspace),
                                            workspace.numel() * workspace.element_size(),
@@ -214,7 +226,7 @@ def int8_mixed_matmul_sharded(X, Wq, w_scale, W_fp16, bitmaps, Y=None, workspace
     return Y, workspace
 
 
-def int8_mixed_matmul_topk(X, Wq, w_scale, W_fp16, k, Y=None, workspace=None, stream=None):
+def int8_mixed_matmul_topk(X, Wq, w_scale, Wt_fp16, k, Y=None, workspace=None, stream=None):
     """LLM.int8() matmul whose outlier set is the k columns of largest max |x|.
     Returns (Y fp16 [M, N], workspace); workspace_views() reads the intermediates."""
     M, K = X.shape
@@ -222,14 +234,14 @@ def int8_mixed_matmul_topk(X, Wq, w_scale, W_fp16, k, Y=None, workspace=None, st
     _need(X, "X", torch.float16, (M, K))
     _need(Wq, "Wq", torch.int8, (N, K))
     _need(w_scale, "w_scale", torch.float32, (N,))
-    _need(W_fp16, "W_fp16", torch.float16, (N, K))
+    _need(Wt_fp16, "Wt_fp16", torch.float16, (K, N))
     Y = torch.empty((M, N), dtype=torch.float16, device=X.device) if Y is None else Y
     _need(Y, "Y", torch.float16, (M, N))
     need = int(load().int8_mixed_matmul_topk_workspace_size(M, N, K))
     if workspace is None:
         workspace = torch.empty((max(need, 1),), dtype=torch.uint8, device=X.device)
     check("int8_mixed_matmul_topk",
-          load().int8_mixed_matmul_topk(_ptr(X), _ptr(Wq), _ptr(w_scale), _ptr(W_fp16), M, N, K,
+          load().int8_mixed_matmul_topk(_ptr(X), _ptr(Wq), _ptr(w_scale), _ptr(Wt_fp16), M, N, K,
                                         int(k), _ptr(Y), _ptr(workspace),
                                         workspace.numel() * workspace.element_size(),
                                         _stream(stream)))
@@ -246,7 +258,7 @@ def int8_weight_rowsum(Wq, rowsum=None, stream=None):
     return rowsum
 
 
-def int8_mixed_matmul_zp(X, Wq, w_scale, w_rowsum, W_fp16, threshold=6.0, Y=None,
+def int8_mixed_matmul_zp(X, Wq, w_scale, w_rowsum, Wt_fp16, threshold=6.0, Y=None,
                          workspace=None, stream=None):
     """The decomposition with zero-point codes for the non-outlier part.
     Returns (Y fp16 [M, N], workspace); zero points via zeropoint_views()."""
@@ -256,7 +268,7 @@ def int8_mixed_matmul_zp(X, Wq, w_scale, w_rowsum, W_fp16, threshold=6.0, Y=None
     _need(Wq, "Wq", torch.int8, (N, K))
     _need(w_scale, "w_scale", torch.float32, (N,))
     _need(w_rowsum, "w_rowsum", torch.int32, (N,))
-    _need(W_fp16, "W_fp16", torch.float16, (N, K))
+    _need(Wt_fp16, "Wt_fp16", torch.float16, (K, N))
     Y = torch.empty((M, N), dtype=torch.float16, device=X.device) if Y is None else Y
     _need(Y, "Y", torch.float16, (M, N))
     need = int(load().int8_mixed_matmul_zp_workspace_size(M, N, K))
@@ -264,7 +276,7 @@ def int8_mixed_matmul_zp(X, Wq, w_scale, w_rowsum, W_fp16, threshold=6.0, Y=None
         workspace = torch.empty((max(need, 1),), dtype=torch.uint8, device=X.device)
     check("int8_mixed_matmul_zp",
           load().int8_mixed_matmul_zp(_ptr(X), _ptr(Wq), _ptr(w_scale), _ptr(w_rowsum),
-                                      _ptr(W_fp16), M, N, K, float(threshold), _ptr(Y),
+                                      _ptr(Wt_fp16), M, N, K, float(threshold), _ptr(Y),
                                       _ptr(workspace), workspace.numel() * workspace.element_size(),
                                       _stream(stream)))
     return Y, workspace

@@ -27,6 +27,7 @@ class WorkspaceLayout(ctypes.Structure):
 
 PROTOTYPES = {
     "int8_quantize_weight_rows": (_i, [_vp, _i, _i, _vp, _vp, _vp]),
+    "int8_transpose_weight": (_i, [_vp, _i, _i, _vp, _vp]),
     "int8_find_outlier_cols": (_i, [_vp, _i, _i, _f, _vp, _vp, _vp, _vp]),
     "int8_quantize_act_rows": (_i, [_vp, _i, _i, _vp, _vp, _vp, _vp]),
     "int8_mixed_matmul_workspace_size": (_sz, [_i, _i, _i]),

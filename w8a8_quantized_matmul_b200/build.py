@@ -13,7 +13,7 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libint8mm.so")
-SOURCES = ["api.cu", "quant_kernels.cu", "fused_quant.cu", "gemm_sm100.cu", "decode.cu", "noalloc.cu", "smoothquant.cu", "topk.cu", "rotation.cu", "gemm_groups.cu", "selftest.cu"]
+SOURCES = ["api.cu", "quant_kernels.cu", "fused_quant.cu", "stream_quant.cu", "gemm_sm100.cu", "decode.cu", "noalloc.cu", "smoothquant.cu", "topk.cu", "rotation.cu", "gemm_groups.cu", "selftest.cu"]
 HEADERS = ["ptx.cuh", "kernels.cuh", "quant_common.cuh"]
 
 

@@ -178,6 +178,18 @@ int int8_quantize_weight_rows(const void* W, int N, int K, int8_t* Wq, float* w_
   return cuda_status(cudaGetLastError());
 }
 
+int int8_transpose_weight(const void* W, int N, int K, void* Wt, i8mm_stream_t stream) {
+  int st = check_sizes(1, N, K);
+  if (st != I8MM_OK) return st;
+  if (N == 0) return I8MM_OK;
+  if (!W || !Wt) return I8MM_ERR_INVALID_ARG;
+  if (!aligned16(W) || !aligned16(Wt)) return I8MM_ERR_ALIGNMENT;
+  if ((st = check_device()) != I8MM_OK) return st;
+  return cuda_status(launch_transpose_weight(static_cast<const __half*>(W), N, K,
+                                             static_cast<__half*>(Wt),
+                                             static_cast<cudaStream_t>(stream)));
+}
+
 int int8_find_outlier_cols(const void* X, int M, int K, float threshold, uint32_t* col_bitmap,
                            int32_t* n_outliers, int32_t* col_idx, i8mm_stream_t stream) {
   int st = check_sizes(M, 1, K);
@@ -228,7 +240,7 @@ namespace {
 
 // stages: bit 0 = control-word clear + fused quantisation kernel, bit 1 = GEMM.
 // given / given_n: token-sharded mode (outlier set = OR of the given bitmaps).
-int mixed_matmul_impl(const void* X, const int8_t* Wq, const float* w_scale, const void* W_fp16,
+int mixed_matmul_impl(const void* X, const int8_t* Wq, const float* w_scale, const void* Wt_fp16,
                       int M, int N, int K, float threshold, void* Y, void* workspace,
                       size_t workspace_bytes, cudaStream_t stream, cudaEvent_t const* ev,
                       int stages = 3, const uint32_t* given = nullptr, int given_n = 0,
@@ -237,8 +249,8 @@ int mixed_matmul_impl(const void* X, const int8_t* Wq, const float* w_scale, con
   if (st != I8MM_OK) return st;
   if ((st = check_threshold(threshold)) != I8MM_OK) return st;
   if (M == 0 || N == 0) return I8MM_OK;
-  if (!X || !Wq || !w_scale || !W_fp16 || !Y) return I8MM_ERR_INVALID_ARG;
-  if (!aligned16(X) || !aligned16(Wq) || !aligned16(w_scale) || !aligned16(W_fp16) ||
+  if (!X || !Wq || !w_scale || !Wt_fp16 || !Y) return I8MM_ERR_INVALID_ARG;
+  if (!aligned16(X) || !aligned16(Wq) || !aligned16(w_scale) || !aligned16(Wt_fp16) ||
       !aligned16(Y))
     return I8MM_ERR_ALIGNMENT;
   Layout L;
@@ -259,7 +271,7 @@ int mixed_matmul_impl(const void* X, const int8_t* Wq, const float* w_scale, con
   __half* XO = reinterpret_cast<__half*>(ws + L.l.X_O);
   __half* WO = reinterpret_cast<__half*>(ws + L.l.W_O);
   const __half* Xh = static_cast<const __half*>(X);
-  const __half* Wh = static_cast<const __half*>(W_fp16);
+  const __half* Wh = static_cast<const __half*>(Wt_fp16);
 
   // Decode shapes: one clustered kernel for the whole call.
   if (stages == 3 && !ev && !given && !x_zero && decode_supported(M, K)) {
@@ -340,18 +352,18 @@ int mixed_matmul_impl(const void* X, const int8_t* Wq, const float* w_scale, con
 
 extern "C" {
 
-int int8_mixed_matmul(const void* X, const int8_t* Wq, const float* w_scale, const void* W_fp16,
+int int8_mixed_matmul(const void* X, const int8_t* Wq, const float* w_scale, const void* Wt_fp16,
                       int M, int N, int K, float threshold, void* Y, void* workspace,
                       size_t workspace_bytes, i8mm_stream_t stream) {
-  return mixed_matmul_impl(X, Wq, w_scale, W_fp16, M, N, K, threshold, Y, workspace,
+  return mixed_matmul_impl(X, Wq, w_scale, Wt_fp16, M, N, K, threshold, Y, workspace,
                            workspace_bytes, stream, nullptr);
 }
 
 int int8_mixed_matmul_stage(int stage, const void* X, const int8_t* Wq, const float* w_scale,
-                            const void* W_fp16, int M, int N, int K, float threshold, void* Y,
+                            const void* Wt_fp16, int M, int N, int K, float threshold, void* Y,
                             void* workspace, size_t workspace_bytes, i8mm_stream_t stream) {
   if (stage != 1 && stage != 2) return I8MM_ERR_INVALID_ARG;
-  return mixed_matmul_impl(X, Wq, w_scale, W_fp16, M, N, K, threshold, Y, workspace,
+  return mixed_matmul_impl(X, Wq, w_scale, Wt_fp16, M, N, K, threshold, Y, workspace,
                            workspace_bytes, stream, nullptr, stage);
 }
 
@@ -365,7 +377,7 @@ size_t int8_mixed_matmul_zp_workspace_size(int M, int N, int K) {
 }
 
 int int8_mixed_matmul_zp(const void* X, const int8_t* Wq, const float* w_scale,
-                         const int32_t* w_rowsum, const void* W_fp16, int M, int N, int K,
+                         const int32_t* w_rowsum, const void* Wt_fp16, int M, int N, int K,
                          float threshold, void* Y, void* workspace, size_t workspace_bytes,
                          i8mm_stream_t stream) {
   const int st = check_sizes(M, N, K);
@@ -378,7 +390,7 @@ int int8_mixed_matmul_zp(const void* X, const int8_t* Wq, const float* w_scale,
   if (workspace_bytes < int8_mixed_matmul_zp_workspace_size(M, N, K)) return I8MM_ERR_WORKSPACE;
   int32_t* x_zero = reinterpret_cast<int32_t*>(static_cast<uint8_t*>(workspace) +
                                                ((L.l.total + 255) & ~static_cast<size_t>(255)));
-  return mixed_matmul_impl(X, Wq, w_scale, W_fp16, M, N, K, threshold, Y, workspace,
+  return mixed_matmul_impl(X, Wq, w_scale, Wt_fp16, M, N, K, threshold, Y, workspace,
                            workspace_bytes, static_cast<cudaStream_t>(stream), nullptr, 3, nullptr,
                            0, x_zero, w_rowsum);
 }
@@ -394,7 +406,7 @@ size_t int8_mixed_matmul_topk_workspace_size(int M, int N, int K) {
 }
 
 int int8_mixed_matmul_topk(const void* X, const int8_t* Wq, const float* w_scale,
-                           const void* W_fp16, int M, int N, int K, int k, void* Y,
+                           const void* Wt_fp16, int M, int N, int K, int k, void* Y,
                            void* workspace, size_t workspace_bytes, i8mm_stream_t stream) {
   int st = check_sizes(M, N, K);
   if (st != I8MM_OK) return st;
@@ -420,29 +432,29 @@ int int8_mixed_matmul_topk(const void* X, const int8_t* Wq, const float* w_scale
   if (e != cudaSuccess) return cuda_fail("column_absmax_kernel launch", e);
   e = launch_topk_select(colmax, K, k, sel, s);
   if (e != cudaSuccess) return cuda_fail("topk_select_kernel launch", e);
-  return mixed_matmul_impl(X, Wq, w_scale, W_fp16, M, N, K, 0.0f, Y, workspace, workspace_bytes,
+  return mixed_matmul_impl(X, Wq, w_scale, Wt_fp16, M, N, K, 0.0f, Y, workspace, workspace_bytes,
                            s, nullptr, 3, sel, 1);
 }
 
 int int8_mixed_matmul_sharded(const void* X, const int8_t* Wq, const float* w_scale,
-                              const void* W_fp16, int M, int N, int K, const uint32_t* bitmaps,
+                              const void* Wt_fp16, int M, int N, int K, const uint32_t* bitmaps,
                               int n_bitmaps, void* Y, void* workspace, size_t workspace_bytes,
                               i8mm_stream_t stream) {
   if (!bitmaps || n_bitmaps < 1 || n_bitmaps > 65536) return I8MM_ERR_INVALID_ARG;
   if ((reinterpret_cast<uintptr_t>(bitmaps) & 3u) != 0) return I8MM_ERR_ALIGNMENT;
   // The threshold only enters detection, which the caller has done per rank.
-  return mixed_matmul_impl(X, Wq, w_scale, W_fp16, M, N, K, 0.0f, Y, workspace, workspace_bytes,
+  return mixed_matmul_impl(X, Wq, w_scale, Wt_fp16, M, N, K, 0.0f, Y, workspace, workspace_bytes,
                            stream, nullptr, 3, bitmaps, n_bitmaps);
 }
 
 int int8_mixed_matmul_profiled(const void* X, const int8_t* Wq, const float* w_scale,
-                               const void* W_fp16, int M, int N, int K, float threshold, void* Y,
+                               const void* Wt_fp16, int M, int N, int K, float threshold, void* Y,
                                void* workspace, size_t workspace_bytes, i8mm_stream_t stream,
                                void* const* events) {
   if (!events || !events[0] || !events[1] || !events[2]) return I8MM_ERR_INVALID_ARG;
   cudaEvent_t ev[3] = {static_cast<cudaEvent_t>(events[0]), static_cast<cudaEvent_t>(events[1]),
                        static_cast<cudaEvent_t>(events[2])};
-  return mixed_matmul_impl(X, Wq, w_scale, W_fp16, M, N, K, threshold, Y, workspace,
+  return mixed_matmul_impl(X, Wq, w_scale, Wt_fp16, M, N, K, threshold, Y, workspace,
                            workspace_bytes, stream, ev);
 }
 

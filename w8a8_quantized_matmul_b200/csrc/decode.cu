@@ -375,10 +375,12 @@ __global__ void __launch_bounds__(64 + 32 * kMaxXWarps, 1)
     if (epi) {
       named_bar_sync(kBarList, 32 + 128);
       lcount = misc[0];
-      const __half* wrow = a.W + static_cast<size_t>(n < N ? n : 0) * K + k0;
+      // Outlier feature k of the weight is row k of Wt ([K][N]): consecutive
+      // threads read consecutive n.
+      const __half* wcol = a.W + static_cast<size_t>(k0) * N + (n < N ? n : 0);
 #pragma unroll
       for (int i = 0; i < kWPrefetch; ++i)
-        wv[i] = (n < N && i < lcount) ? wrow[lidx[i]] : __float2half(0.0f);
+        wv[i] = (n < N && i < lcount) ? wcol[static_cast<size_t>(lidx[i]) * N] : __float2half(0.0f);
       wsr = (n < N) ? a.w_scale[n] : 0.0f;
     }
 
@@ -458,7 +460,7 @@ __global__ void __launch_bounds__(64 + 32 * kMaxXWarps, 1)
       float o[kTok];
 #pragma unroll
       for (int t = 0; t < kTok; ++t) o[t] = 0.0f;
-      const __half* wrow = a.W + static_cast<size_t>(n < N ? n : 0) * K + k0;
+      const __half* wcol = a.W + static_cast<size_t>(k0) * N + (n < N ? n : 0);
 #pragma unroll 1
       for (int jj = 0; jj < lcount; ++jj) {
         const int col = lidx[jj];
@@ -466,7 +468,7 @@ __global__ void __launch_bounds__(64 + 32 * kMaxXWarps, 1)
 #pragma unroll
         for (int i = 0; i < kWPrefetch; ++i)
           if (i == jj) wh = wv[i];
-        if (jj >= kWPrefetch && n < N) wh = wrow[col];
+        if (jj >= kWPrefetch && n < N) wh = wcol[static_cast<size_t>(col) * N];
         const float w = __half2float(wh);
         const __half* xc = xs + (col >> 8) * (kTok * kXBox) + (col & (kXBox - 1));
 #pragma unroll

@@ -38,7 +38,8 @@
 //   panels   with any outlier column, by the workers right after pass B (with
 //            the CTA's list; again after a redo): the CTA's rows of the
 //            compacted fp16 panels X_O (from the slots or L2) and W_O (gathered
-//            from W), a multiple of 64 columns wide and zero-padded. The GEMM
+//            from the rows of the transposed weight Wt [K][N] that the list
+//            names), a multiple of 64 columns wide and zero-padded. The GEMM
 //            multiplies them on the tensor cores.
 
 // The code of x is rint(fl32(fl32(x*127)/a)) clamped to +-127. The correctly
@@ -449,7 +450,7 @@ __global__ void __launch_bounds__(kThreads, VPT <= 2 ? 2 : 1)
   // ------------------------------------------------------------ panels
   // The CTA's rows of the compacted fp16 panels for the list in s_idx, a
   // multiple of 64 columns wide and zero-padded: X_O (from the slots or L2)
-  // and W_O (gathered from W). Run by the threads [t0, t0 + nt).
+  // and W_O (gathered from Wt). Run by the threads [t0, t0 + nt).
   const int nper = (a.N + gridDim.x - 1) / gridDim.x;
   const int wn0 = min(a.N, static_cast<int>(blockIdx.x) * nper);
   const int wn1 = min(a.N, wn0 + nper);
@@ -469,18 +470,20 @@ __global__ void __launch_bounds__(kThreads, VPT <= 2 ? 2 : 1)
     }
     const int chunks = pw >> 3;
     const int items = (wn1 - wn0) * chunks;
-    // One item = 8 consecutive panel columns of one weight row: up to 8
-    // independent gathers, one 16-byte store.
+    // One item = 8 consecutive panel columns of one weight row n, read from the
+    // rows idx[p] of Wt ([K][N]); consecutive items are consecutive n, so the
+    // loads are coalesced across a warp. One 16-byte store.
+    const int nr = wn1 - wn0;
     for (int it = tid - t0; it < items; it += nt) {
-      const int n = wn0 + it / chunks;
-      const int ch = it - (n - wn0) * chunks;
-      const __half* wrow = W + static_cast<size_t>(n) * K;
+      const int ch = it / nr;
+      const int n = wn0 + (it - ch * nr);
+      const __half* wcol = W + n;
       uint4 o;
       __half* h = reinterpret_cast<__half*>(&o);
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
         const int p = ch * 8 + i;
-        h[i] = (p < count) ? wrow[s_idx[p]] : __float2half_rn(0.0f);
+        h[i] = (p < count) ? wcol[static_cast<size_t>(s_idx[p]) * a.N] : __float2half_rn(0.0f);
       }
       reinterpret_cast<uint4*>(a.W_O + static_cast<size_t>(n) * a.ld)[ch] = o;
     }
@@ -556,6 +559,8 @@ int fused_vpt(int K) {
 }
 
 cudaError_t launch_detect_quantize_compact(const FusedArgs& a, cudaStream_t s) {
+  // Absmax codes with detection: the single-pass kernel of stream_quant.cu.
+  if (a.x_zero == nullptr && a.given == nullptr) return launch_detect_quantize_stream(a, s);
   const int vpt = fused_vpt(a.K);
   const void* fn = nullptr;
   const bool zp = a.x_zero != nullptr;

@@ -45,7 +45,7 @@ struct FusedArgs {
   int8_t* Xq;             // out: [M][K]
   float* x_scale;         // out: [M]
   __half* X_O;            // out: [M][ld]
-  const __half* W;        // in : [N][K]
+  const __half* W;        // in : [K][N], the fp16 weight transposed (row k = feature k)
   __half* W_O;            // out: [N][ld]
   int ld;
   int32_t* status;        // device status word
@@ -60,6 +60,9 @@ struct FusedArgs {
 };
 
 cudaError_t launch_detect_quantize_compact(const FusedArgs& a, cudaStream_t s);
+// Single-pass form of the same step for the absmax codes with detection
+// (stream_quant.cu); the launcher above hands those calls to it.
+cudaError_t launch_detect_quantize_stream(const FusedArgs& a, cudaStream_t s);
 
 // Host-side launchers of the tensor-core GEMM (gemm_sm100.cu). They encode the
 // TMA tensor maps and launch; the return value is the cudaError_t of the launch.
@@ -103,7 +106,7 @@ inline bool make_tmap_sw128(CUtensorMap* m, const void* base, CUtensorMapDataTyp
 // Decode-shape path (M <= 16): one clustered kernel (decode.cu).
 struct DecodeArgs {
   const __half* X;        // [M][K]
-  const __half* W;        // [N][K] fp16 weight (outlier columns are read)
+  const __half* W;        // [K][N] fp16 weight, transposed (outlier rows are read)
   const int8_t* Wq;       // [N][K]
   const float* w_scale;   // [N]
   __half* Y;              // [M][N]
@@ -128,6 +131,9 @@ cudaError_t launch_column_absmax(const __half* X, int rows, int K, float* colmax
 cudaError_t launch_topk_select(const float* colmax, int K, int k, uint32_t* bitmap,
                                cudaStream_t s);
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t s);
+
+// Offline: Wt[k][n] = W[n][k] for an fp16 [N][K] weight (quant_kernels.cu).
+cudaError_t launch_transpose_weight(const __half* W, int N, int K, __half* Wt, cudaStream_t s);
 
 // The C-ABI layer's device check (I8MM_OK or I8MM_ERR_UNSUPPORTED_DEVICE /
 // I8MM_ERR_CUDA) and its error recorder (the text int8_last_error_string

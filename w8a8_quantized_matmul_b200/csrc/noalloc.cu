@@ -72,16 +72,16 @@ static_assert(kNoAllocScratchBytes == I8MM_NOALLOC_SCRATCH_BYTES, "header and ar
 extern "C" {
 
 int int8_mixed_matmul_noalloc(const void* X, const int8_t* Wq, const float* w_scale,
-                              const void* W_fp16, int M, int N, int K, float threshold,
+                              const void* Wt_fp16, int M, int N, int K, float threshold,
                               void* Y, i8mm_stream_t stream) {
   if (M == 0 || N == 0) {
     // Same empty-problem rule as int8_mixed_matmul, without touching the device.
-    return int8_mixed_matmul(X, Wq, w_scale, W_fp16, M, N, K, threshold, Y, nullptr, 0, stream);
+    return int8_mixed_matmul(X, Wq, w_scale, Wt_fp16, M, N, K, threshold, Y, nullptr, 0, stream);
   }
   const size_t need = int8_mixed_matmul_workspace_size(M, N, K);
   if (need == 0) {
     // Invalid sizes: let the regular entry point report which check failed.
-    return int8_mixed_matmul(X, Wq, w_scale, W_fp16, M, N, K, threshold, Y, nullptr, 0, stream);
+    return int8_mixed_matmul(X, Wq, w_scale, Wt_fp16, M, N, K, threshold, Y, nullptr, 0, stream);
   }
   if (need > kNoAllocScratchBytes) return I8MM_ERR_WORKSPACE;   // too large for the array
   void* scratch = nullptr;
@@ -90,7 +90,7 @@ int int8_mixed_matmul_noalloc(const void* X, const int8_t* Wq, const float* w_sc
   // The regular path clears the control words it needs (count, status, barrier
   // counter, bitmap) at the start of every call, so the previous call's
   // contents of the array do not matter.
-  return int8_mixed_matmul(X, Wq, w_scale, W_fp16, M, N, K, threshold, Y, scratch,
+  return int8_mixed_matmul(X, Wq, w_scale, Wt_fp16, M, N, K, threshold, Y, scratch,
                            kNoAllocScratchBytes, stream);
 }
 

@@ -262,4 +262,31 @@ cudaError_t launch_weight_rowsum(const int8_t* Wq, int N, int K, int32_t* rowsum
   return cudaGetLastError();
 }
 
+// Offline layout change of the fp16 weight for the outlier product: Wt[k][n] =
+// W[n][k]. The LLM.int8() outlier term reads whole input features of the weight
+// (AIInfra "05Quantization01", LLM.int8() section: W in h x o orientation, the
+// rows W^h of the outlier dimensions h), which are contiguous rows of Wt.
+// 32 x 32 tiles through shared memory (one padding column against bank
+// conflicts); a block of 32 x 8 threads, four rows each.
+__global__ void __launch_bounds__(256) transpose_weight_kernel(const __half* __restrict__ W, int N,
+                                                               int K, __half* __restrict__ Wt) {
+  __shared__ __half tile[32][33];
+  const int n0 = blockIdx.x * 32, k0 = blockIdx.y * 32;   // N blocks in x: N may exceed 65535 * 32
+  for (int j = threadIdx.y; j < 32; j += 8) {
+    const int n = n0 + j, k = k0 + threadIdx.x;
+    if (n < N && k < K) tile[j][threadIdx.x] = W[static_cast<size_t>(n) * K + k];
+  }
+  __syncthreads();
+  for (int j = threadIdx.y; j < 32; j += 8) {
+    const int k = k0 + j, n = n0 + threadIdx.x;
+    if (n < N && k < K) Wt[static_cast<size_t>(k) * N + n] = tile[threadIdx.x][j];
+  }
+}
+
+cudaError_t launch_transpose_weight(const __half* W, int N, int K, __half* Wt, cudaStream_t s) {
+  dim3 grid((N + 31) / 32, (K + 31) / 32);
+  transpose_weight_kernel<<<grid, dim3(32, 8), 0, s>>>(W, N, K, Wt);
+  return cudaGetLastError();
+}
+
 }  // namespace i8mm

@@ -41,18 +41,18 @@ def _gather(bitmap, group=None):
     return torch.stack(parts)
 
 
-def _apply_cuda(X_local, Wq, w_scale, W_fp16, bitmaps, Y=None, workspace=None):
-    return _ops.int8_mixed_matmul_sharded(X_local, Wq, w_scale, W_fp16, bitmaps, Y=Y,
+def _apply_cuda(X_local, Wq, w_scale, Wt_fp16, bitmaps, Y=None, workspace=None):
+    return _ops.int8_mixed_matmul_sharded(X_local, Wq, w_scale, Wt_fp16, bitmaps, Y=Y,
                                           workspace=workspace)[0]
 
 
-def token_sharded_mixed_matmul(X_local, Wq, w_scale, W_fp16, threshold=6.0, group=None, Y=None,
+def token_sharded_mixed_matmul(X_local, Wq, w_scale, Wt_fp16, threshold=6.0, group=None, Y=None,
                                workspace=None, *, find=_find_cuda, gather=_gather,
                                apply=_apply_cuda):
     """This rank's rows of Y for a batch whose tokens are split over `group`."""
     bitmap = find(X_local, threshold)
     bitmaps = gather(bitmap, group)
-    return apply(X_local, Wq, w_scale, W_fp16, bitmaps, Y, workspace)
+    return apply(X_local, Wq, w_scale, Wt_fp16, bitmaps, Y, workspace)
 
 
 # ---------------------------------------------------------------------------
@@ -73,8 +73,8 @@ def column_block(N: int, rank: int, world: int):
     return n0, min(N, n0 + per)
 
 
-def _apply_cols_cuda(X, Wq_local, w_scale_local, W_local, threshold, Y=None, workspace=None):
-    return _ops.int8_mixed_matmul(X, Wq_local, w_scale_local, W_local, threshold, Y=Y,
+def _apply_cols_cuda(X, Wq_local, w_scale_local, Wt_local, threshold, Y=None, workspace=None):
+    return _ops.int8_mixed_matmul(X, Wq_local, w_scale_local, Wt_local, threshold, Y=Y,
                                   workspace=workspace)[0]
 
 
@@ -91,13 +91,15 @@ def _gather_cols(Y_local, N, group=None):
     return torch.cat(parts, dim=1)[:, :N]
 
 
-def column_sharded_mixed_matmul(X, Wq_local, w_scale_local, W_local, threshold=6.0, group=None,
+def column_sharded_mixed_matmul(X, Wq_local, w_scale_local, Wt_local, threshold=6.0, group=None,
                                 N=None, gather=False, Y=None, workspace=None, *,
                                 apply=_apply_cols_cuda):
     """This rank's column block of Y = X . W^T from its block of weight rows
-    (`column_block`); no collective unless gather=True, which returns the full
-    [M, N] Y on every rank (N is then required)."""
-    Y_local = apply(X, Wq_local, w_scale_local, W_local, threshold, Y, workspace)
+    (`column_block`: Wq_local and w_scale_local are rows [n0, n1) of Wq and
+    w_scale, Wt_local the columns [n0, n1) of the transposed fp16 weight as a
+    contiguous [K, n1 - n0] tensor); no collective unless gather=True, which
+    returns the full [M, N] Y on every rank (N is then required)."""
+    Y_local = apply(X, Wq_local, w_scale_local, Wt_local, threshold, Y, workspace)
     if not gather:
         return Y_local
     if N is None:
