@@ -102,6 +102,12 @@ def test_other_entry_points_validation(lib):
     assert lib.int8_quantize_weight_rows(None, 8, 64, A, A, None) == _lib.I8MM_ERR_INVALID_ARG
     assert lib.int8_quantize_weight_rows(A, 8, 64, MIS, A, None) == _lib.I8MM_ERR_ALIGNMENT
     assert lib.int8_quantize_weight_rows(A, 0, 64, None, None, None) == _lib.I8MM_OK
+    assert lib.int8_transpose_weight(A, 8, 40, A, None) == _lib.I8MM_ERR_ALIGNMENT
+    assert lib.int8_transpose_weight(None, 8, 64, A, None) == _lib.I8MM_ERR_INVALID_ARG
+    assert lib.int8_transpose_weight(A, 8, 64, None, None) == _lib.I8MM_ERR_INVALID_ARG
+    assert lib.int8_transpose_weight(A, 8, 64, MIS, None) == _lib.I8MM_ERR_ALIGNMENT
+    assert lib.int8_transpose_weight(A, -1, 64, A, None) == _lib.I8MM_ERR_INVALID_ARG
+    assert lib.int8_transpose_weight(A, 0, 64, None, None) == _lib.I8MM_OK
     assert lib.int8_find_outlier_cols(A, 4, 64, math.nan, A, A, A, None) == _lib.I8MM_ERR_INVALID_ARG
     assert lib.int8_find_outlier_cols(A, 4, 64, -0.5, A, A, A, None) == _lib.I8MM_ERR_INVALID_ARG
     assert lib.int8_find_outlier_cols(A, 4, 64, 6.0, None, A, A, None) == _lib.I8MM_ERR_INVALID_ARG

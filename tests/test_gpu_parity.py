@@ -275,6 +275,26 @@ def test_outliers_on_few_tokens_force_the_recheck(case):
     assert_y_close(Y, ref["Y"], f"recheck {case}")
 
 
+@pytest.mark.parametrize("thr", [6.001, 5.999, 65519.0, 70000.0, 1e-9, 2.0 ** -24, 0.5])
+def test_threshold_between_fp16_values(thr):
+    """Thresholds that no fp16 value equals (and the neighbours of the ones that
+    are): the prefill kernel's fp16 comparison selects the oracle's fp32 set."""
+    M, K, N = 96, 512, 136
+    X, W, _ = synth.random_case(M, K, N, 4, seed=77)
+    t16 = np.float16(thr)
+    near = [t16, np.nextafter(t16, np.float16(np.inf)), np.nextafter(t16, np.float16(0))]
+    near = [v for v in near if np.isfinite(v)]      # finite inputs only
+    for j, v in enumerate(near):                    # entries at and next to the threshold
+        X[3 + j, 7 * j + 1] = v
+        X[20 + j, 11 * j + 5] = -v
+    X[40, 100] = np.float16(65504.0)
+    Y, got, _, _ = run_mixed(X, W, thr)
+    ref = oracle.llm_int8_matmul(X, W, thr)
+    check_intermediates(ref, got, K)
+    check_panels(X, W, ref, got)
+    assert_y_close(Y, ref["Y"], f"threshold {thr}")
+
+
 def test_mixed_matmul_guard_bands():
     """Writes stay inside Y and the workspace (256-byte canaries on both sides)."""
     m = mm()

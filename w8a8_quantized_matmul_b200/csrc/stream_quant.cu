@@ -22,16 +22,16 @@
 // a warp's piece of a row is at most 256 vectors of 8 fp16 values (8 per lane,
 // held in registers): GW = 1 up to K = 2048, K/2048 beyond.
 //   stream   group g takes rows g, g + NG, ... of the block; each warp bulk-
-//            copies its pieces of the group's rows into its own ring of NS
-//            slots in shared memory (one mbarrier per slot, NS rows ahead),
-//            reads a piece into registers and at once refills the slot with the
-//            piece NS rows further on, so that the loads overlap the coding. From the registers: the lane's maximum |x|
-//            (only a lane whose maximum exceeds the threshold, rarely, takes
-//            the per-entry flags, a shared-memory atomicOr into the CTA's column
-//            bitmap, and the maximum over its unflagged entries), the row
-//            maximum m1 (warp reduction, then one named barrier of the group),
-//            and the codes with m1, stored straight to Xq. Groups never wait
-//            for one another.
+//            copies its piece of a row into its own slot in shared memory (one
+//            mbarrier per slot), reads it into registers and at once refills
+//            the slot with its piece of the group's next row, so that the load
+//            overlaps the coding. From the registers: the maximum |x| of each
+//            vector and of the lane (only a lane whose maximum exceeds the
+//            threshold, rarely, takes the per-entry flags of its vectors above
+//            it, a shared-memory atomicOr into the CTA's column bitmap, and the
+//            maximum over its unflagged entries), the row maximum m1 (warp
+//            reduction, then one named barrier of the group), and the codes
+//            with m1, stored straight to Xq. Groups never wait for one another.
 //   list     after the last row: warp 0 builds the ascending list L of the
 //            CTA's flagged columns (a subset of the batch's outlier set O; equal
 //            to it unless the CTA's rows miss a column that other rows flag);
@@ -71,7 +71,6 @@ namespace i8mm {
 namespace {
 
 constexpr int kMaxWarps = 16;     // warps per CTA
-constexpr int kMaxRing = 4;       // row slots per warp
 constexpr int kMaxGroups = 8;     // warp groups per CTA (named barriers 1..8)
 constexpr int kRowBlock = 64;     // rows of the fix-up per round (shared row maxima)
 constexpr int kMaxRedo = 32;      // rows of one CTA listed for a second coding
@@ -101,10 +100,53 @@ __device__ __forceinline__ float warp_max_nonneg(float v) {
   return __uint_as_float(__reduce_max_sync(0xffffffffu, __float_as_uint(v)));
 }
 
+// Codes of the fp16 pair w, each in the low byte of its fp32 lane: n = x*127
+// exactly (one mixed-precision FMA per value, fp16 operands, fp32 result),
+// q = fl(n*ra), r = fma(q, -a, n), q' = fma(r, ra, q) (the FMA-corrected
+// quotient of quant_common.cuh, the same operations in the same order), then
+// the 1.5*2^23 rounding. ra2 = (ra, ra), na2 = (-a, -a), magic2 = (1.5*2^23) x 2,
+// h127 = 127.0 in binary16.
+__device__ __forceinline__ uint64_t code_pair_h(uint32_t w, uint64_t ra2, uint64_t na2,
+                                                uint64_t magic2, uint16_t h127) {
+  uint64_t s;
+  asm("{\n\t"
+      ".reg .b16 l, h;\n\t"
+      ".reg .f32 n0, n1;\n\t"
+      ".reg .b64 n, q, r;\n\t"
+      "mov.b32 {l, h}, %1;\n\t"
+      "fma.rn.f32.f16 n0, l, %5, %6;\n\t"
+      "fma.rn.f32.f16 n1, h, %5, %6;\n\t"
+      "mov.b64 n, {n0, n1};\n\t"
+      "mul.rn.f32x2 q, n, %2;\n\t"
+      "fma.rn.f32x2 r, q, %3, n;\n\t"
+      "fma.rn.f32x2 q, r, %2, q;\n\t"
+      "add.rn.f32x2 %0, q, %4;\n\t"
+      "}"
+      : "=l"(s)
+      : "r"(w), "l"(ra2), "l"(na2), "l"(magic2), "h"(h127), "f"(-0.0f));
+  return s;
+}
+
+// Eight INT8 codes of the vector u (codes8 of quant_common.cuh, n formed by the
+// mixed-precision FMA).
+__device__ __forceinline__ uint2 codes8_h(const uint4& u, uint64_t ra2, uint64_t na2,
+                                          uint64_t magic2, uint16_t h127) {
+  const uint64_t s0 = code_pair_h(u.x, ra2, na2, magic2, h127);
+  const uint64_t s1 = code_pair_h(u.y, ra2, na2, magic2, h127);
+  const uint64_t s2 = code_pair_h(u.z, ra2, na2, magic2, h127);
+  const uint64_t s3 = code_pair_h(u.w, ra2, na2, magic2, h127);
+  const uint32_t w0 = __byte_perm(__byte_perm(static_cast<uint32_t>(s0), static_cast<uint32_t>(s0 >> 32), 0x0040),
+                                  __byte_perm(static_cast<uint32_t>(s1), static_cast<uint32_t>(s1 >> 32), 0x0040),
+                                  0x5410);
+  const uint32_t w1 = __byte_perm(__byte_perm(static_cast<uint32_t>(s2), static_cast<uint32_t>(s2 >> 32), 0x0040),
+                                  __byte_perm(static_cast<uint32_t>(s3), static_cast<uint32_t>(s3 >> 32), 0x0040),
+                                  0x5410);
+  return make_uint2(w0, w1);
+}
+
 // Shared-memory layout (16-byte aligned pieces):
-//   rows   [NW][NS] slots    a ring of NS slots per warp for its pieces of rows
-//                            (pv vectors each); after the stream the outlier
-//                            list [K] u16
+//   rows   [NW] slots        one slot per warp for its piece of a row (pv
+//                            vectors); after the stream the outlier list [K] u16
 //   lbits  [words] u32       the CTA's own column flags
 //   gbits  [words] u32       the batch bitmap, after the grid barrier
 //   gred   [kMaxGroups][2][kMaxWarps] f32  per-warp row maxima of each group,
@@ -113,7 +155,7 @@ __device__ __forceinline__ float warp_max_nonneg(float v) {
 //   mo     [kRowBlock] u32   fix-up maxima mO (fp32 bit patterns) of a round
 //   misc   [4] i32           list count, redo count
 //   redo   [kMaxRedo] i32    rows to code again
-//   bar    [kMaxWarps*kMaxRing] u64  one mbarrier per slot
+//   bar    [kMaxWarps] u64   one mbarrier per slot
 struct StreamSmem {
   size_t rows, lbits, gbits, gred, m1, mo, misc, redo, bar, total;
 };
@@ -133,16 +175,16 @@ __host__ __device__ inline StreamSmem stream_smem_layout(int K, size_t slot_byte
   L.mo = off;     off = up16(off + kRowBlock * 4);
   L.misc = off;   off = up16(off + 16);
   L.redo = off;   off = up16(off + kMaxRedo * 4);
-  L.bar = off;    off = up16(off + kMaxWarps * kMaxRing * 8);
+  L.bar = off;    off = up16(off + kMaxWarps * 8);
   L.total = off;
   return L;
 }
 
 }  // namespace
 
-template <int VPL>
+template <int VPL, bool FULL>
 __global__ void __launch_bounds__(32 * kMaxWarps, 1)
-    stream_quantize_kernel(FusedArgs a, uint32_t th2bits, int GW, int NS) {
+    stream_quantize_kernel(FusedArgs a, uint32_t th2bits, int GW) {
   extern __shared__ __align__(128) uint8_t ssm[];
   const int K = a.K;
   const int NW = static_cast<int>(blockDim.x) >> 5;
@@ -150,7 +192,7 @@ __global__ void __launch_bounds__(32 * kMaxWarps, 1)
   const int words = (K + 31) >> 5;
   const int nv = K >> 3;
   const int pv = (nv + GW - 1) / GW;   // vectors of a row per warp of a group
-  const StreamSmem L = stream_smem_layout(K, static_cast<size_t>(NW) * NS * pv * 16);
+  const StreamSmem L = stream_smem_layout(K, static_cast<size_t>(NW) * pv * 16);
   uint16_t* s_idx = reinterpret_cast<uint16_t*>(ssm + L.rows);   // valid after the stream
   uint32_t* s_lbits = reinterpret_cast<uint32_t*>(ssm + L.lbits);
   uint32_t* s_gbits = reinterpret_cast<uint32_t*>(ssm + L.gbits);
@@ -178,7 +220,7 @@ __global__ void __launch_bounds__(32 * kMaxWarps, 1)
   for (int w = tid; w < words; w += blockDim.x) s_lbits[w] = 0u;
   for (int r = tid; r < kRowBlock; r += blockDim.x) s_mo[r] = 0u;
   if (tid == 0) {
-    for (int s = 0; s < NW * NS; ++s) mbar_init(&s_bar[s], 1);
+    for (int s = 0; s < NW; ++s) mbar_init(&s_bar[s], 1);
     fence_mbarrier_init();
     s_misc[1] = 0;
   }
@@ -188,62 +230,63 @@ __global__ void __launch_bounds__(32 * kMaxWarps, 1)
   const int g = warp / GW;            // group
   const int gw = warp - g * GW;       // warp within the group
   const int v0 = gw * pv;             // first vector of this warp's piece of a row
-  const int npv = max(0, min(pv, nv - v0));
+  const int npv = FULL ? VPL * 32 : max(0, min(pv, nv - v0));
   const uint32_t piece_bytes = static_cast<uint32_t>(npv) * 16u;
   const int nrows = R > g ? (R - g + NG - 1) / NG : 0;   // rows of this group: g, g + NG, ...
-  // The warp's ring of NS slots: the group's i-th row in slot i % NS, the
-  // (i / NS)-th fill of that slot.
-  auto slot_of = [&](int i) {
-    return reinterpret_cast<uint4*>(ssm + L.rows + (static_cast<size_t>(warp) * NS + i % NS) * pv * 16);
-  };
-  auto bar_of = [&](int i) { return &s_bar[warp * NS + i % NS]; };
+  const uint4* slot = reinterpret_cast<const uint4*>(ssm + L.rows + static_cast<size_t>(warp) * pv * 16);
+  uint64_t* bar = &s_bar[warp];
+  const __half* xpiece = a.X + static_cast<size_t>(r0 + g) * K + static_cast<size_t>(v0) * 8;
+  const size_t row_step = static_cast<size_t>(NG) * K;   // elements from one row of the group to its next
   auto issue = [&](int i) {   // lane 0: this warp's piece of the group's i-th row
     // Earlier generic-proxy reads of the slot before the async-proxy write.
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-    mbar_arrive_expect_tx(bar_of(i), piece_bytes);
-    bulk_load(slot_of(i), a.X + static_cast<size_t>(r0 + g + i * NG) * K + static_cast<size_t>(v0) * 8,
-              piece_bytes, bar_of(i));
+    mbar_arrive_expect_tx(bar, piece_bytes);
+    bulk_load(const_cast<uint4*>(slot), xpiece + static_cast<size_t>(i) * row_step, piece_bytes, bar);
   };
-  if (lane == 0 && npv > 0)
-    for (int i = 0; i < NS && i < nrows; ++i) issue(i);
+  if (lane == 0 && npv > 0 && nrows > 0) issue(0);
+  // Loop-invariant operands of the code arithmetic.
+  const uint64_t magic2 = f2pack(kMagic, kMagic);
+  const uint16_t h127 = 0x57F0u;   // 127.0 in binary16
   bool ok = true;
-  const bool full = npv == VPL * 32;
-  for (int i = 0; i < nrows; ++i) {
-    const int row = g + i * NG;
+  uint2* dst = reinterpret_cast<uint2*>(a.Xq + static_cast<size_t>(r0 + g) * K) + v0 + lane;
+  const size_t dst_step = row_step / 8;                    // uint2 per group row step
+  for (int i = 0; i < nrows; ++i, dst += dst_step) {
     uint4 u[VPL];
     if (npv > 0) {
-      if (ok && !mbar_wait(bar_of(i), static_cast<uint32_t>((i / NS) & 1))) {
+      if (ok && !mbar_wait(bar, static_cast<uint32_t>(i & 1))) {
         ok = false;
         if (lane == 0) atomicCAS(a.status, 0, -5 /* I8MM_ERR_TIMEOUT */);
       }
-      const uint4* slot = slot_of(i);
 #pragma unroll
       for (int c = 0; c < VPL; ++c)
-        u[c] = (full || c * 32 + lane < npv) ? slot[c * 32 + lane] : make_uint4(0u, 0u, 0u, 0u);
-      // The piece is in registers: the slot takes the row NS further on now,
+        u[c] = (FULL || c * 32 + lane < npv) ? slot[c * 32 + lane] : make_uint4(0u, 0u, 0u, 0u);
+      // The piece is in registers: the slot takes the group's next row now,
       // while this one is coded.
       __syncwarp();
-      if (lane == 0 && i + NS < nrows) issue(i + NS);
+      if (lane == 0 && i + 1 < nrows) issue(i + 1);
     } else {
 #pragma unroll
       for (int c = 0; c < VPL; ++c) u[c] = make_uint4(0u, 0u, 0u, 0u);
     }
-    // Pass 1: the lane's maximum |x| (four independent accumulators). Only a
-    // lane whose maximum exceeds the threshold (rare) needs the per-entry
-    // flags and the maximum over its unflagged entries.
-    uint32_t am[4] = {0u, 0u, 0u, 0u};
+    // Pass 1: maximum |x| of each vector and of the lane. Only a lane whose
+    // maximum exceeds the threshold (rare) takes the per-entry flags of its
+    // vectors that exceed it and the maximum over its unflagged entries.
+    uint32_t vm[VPL];
 #pragma unroll
-    for (int c = 0; c < VPL; ++c) {
-      am[0] = hmax2_bits(am[0], u[c].x & 0x7FFF7FFFu);
-      am[1] = hmax2_bits(am[1], u[c].y & 0x7FFF7FFFu);
-      am[2] = hmax2_bits(am[2], u[c].z & 0x7FFF7FFFu);
-      am[3] = hmax2_bits(am[3], u[c].w & 0x7FFF7FFFu);
-    }
-    uint32_t rm = hmax2_bits(hmax2_bits(am[0], am[1]), hmax2_bits(am[2], am[3]));
+    for (int c = 0; c < VPL; ++c)
+      vm[c] = hmax2_bits(hmax2_bits(u[c].x & 0x7FFF7FFFu, u[c].y & 0x7FFF7FFFu),
+                         hmax2_bits(u[c].z & 0x7FFF7FFFu, u[c].w & 0x7FFF7FFFu));
+    uint32_t rm = vm[0];
+#pragma unroll
+    for (int c = 1; c < VPL; ++c) rm = hmax2_bits(rm, vm[c]);
     if (__hgt2_mask(*reinterpret_cast<const __half2*>(&rm), th2) != 0u) {
       rm = 0u;
 #pragma unroll
       for (int c = 0; c < VPL; ++c) {
+        if (__hgt2_mask(*reinterpret_cast<const __half2*>(&vm[c]), th2) == 0u) {
+          rm = hmax2_bits(rm, vm[c]);
+          continue;
+        }
         const uint32_t wd[4] = {u[c].x, u[c].y, u[c].z, u[c].w};
         uint32_t f8 = 0u;
 #pragma unroll
@@ -254,7 +297,7 @@ __global__ void __launch_bounds__(32 * kMaxWarps, 1)
           f8 |= ((fl & 1u) << (2 * k)) | (((fl >> 16) & 1u) << (2 * k + 1));
         }
         const int v = v0 + c * 32 + lane;
-        if (f8 != 0u && (full || c * 32 + lane < npv)) atomicOr(&s_lbits[v >> 2], f8 << (8 * (v & 3)));
+        if (FULL || c * 32 + lane < npv) atomicOr(&s_lbits[v >> 2], f8 << (8 * (v & 3)));
       }
     }
     float m1 = warp_max_nonneg(hpair_max(rm));
@@ -265,13 +308,14 @@ __global__ void __launch_bounds__(32 * kMaxWarps, 1)
       m1 = warp_max_nonneg(red[lane < GW ? lane : 0]);
     }
     const float ra = quant_rcp(m1);
+    const uint64_t ra2 = f2pack(ra, ra), na2 = f2pack(-m1, -m1);
     // Pass 2: the codes with m1 (entries the row flags itself get codes that
     // the fix-up overwrites with 0).
-    uint2* dst = reinterpret_cast<uint2*>(a.Xq + static_cast<size_t>(r0 + row) * K) + v0;
 #pragma unroll
     for (int c = 0; c < VPL; ++c)
-      if (full || c * 32 + lane < npv) dst[c * 32 + lane] = codes8(u[c], m1, ra);
+      if (FULL || c * 32 + lane < npv) dst[c * 32] = codes8_h(u[c], ra2, na2, magic2, h127);
     if (gw == 0 && lane == 0) {
+      const int row = g + i * NG;
       a.x_scale[r0 + row] = m1;
       if (row < kRowBlock) s_m1[row] = m1;
     }
@@ -549,20 +593,23 @@ cudaError_t launch_detect_quantize_stream(const FusedArgs& a, cudaStream_t s) {
   const int pv = (nv + GW - 1) / GW;
   int VPL = 1;
   while (VPL * 32 < pv) VPL *= 2;
+  // Every warp's piece full (no bounds checks in the stream) for the usual K.
+  const bool full = nv == GW * VPL * 32;
   const void* fn = nullptr;
   switch (VPL) {
-    case 1: fn = reinterpret_cast<const void*>(stream_quantize_kernel<1>); break;
-    case 2: fn = reinterpret_cast<const void*>(stream_quantize_kernel<2>); break;
-    case 4: fn = reinterpret_cast<const void*>(stream_quantize_kernel<4>); break;
-    case 8: fn = reinterpret_cast<const void*>(stream_quantize_kernel<8>); break;
-    default: fn = reinterpret_cast<const void*>(stream_quantize_kernel<16>); break;
+    case 1: fn = full ? reinterpret_cast<const void*>(stream_quantize_kernel<1, true>)
+                      : reinterpret_cast<const void*>(stream_quantize_kernel<1, false>); break;
+    case 2: fn = full ? reinterpret_cast<const void*>(stream_quantize_kernel<2, true>)
+                      : reinterpret_cast<const void*>(stream_quantize_kernel<2, false>); break;
+    case 4: fn = full ? reinterpret_cast<const void*>(stream_quantize_kernel<4, true>)
+                      : reinterpret_cast<const void*>(stream_quantize_kernel<4, false>); break;
+    case 8: fn = full ? reinterpret_cast<const void*>(stream_quantize_kernel<8, true>)
+                      : reinterpret_cast<const void*>(stream_quantize_kernel<8, false>); break;
+    default: fn = full ? reinterpret_cast<const void*>(stream_quantize_kernel<16, true>)
+                       : reinterpret_cast<const void*>(stream_quantize_kernel<16, false>); break;
   }
   const int NW = kMaxWarps;
-  const size_t piece = static_cast<size_t>(pv) * 16;
-  // One slot per warp: measured faster than deeper rings (more loads in flight
-  // slowed the stream and the W_O gather that follows it).
-  const int NS = 1;
-  const size_t smem = stream_smem_layout(a.K, static_cast<size_t>(NW) * NS * piece).total;
+  const size_t smem = stream_smem_layout(a.K, static_cast<size_t>(NW) * pv * 16).total;
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
@@ -573,9 +620,9 @@ cudaError_t launch_detect_quantize_stream(const FusedArgs& a, cudaStream_t s) {
   const int grid = max(1, min(ctas, want));
   const uint32_t th = half_floor_bits(a.threshold);
   uint32_t th2 = th | (th << 16);
-  int gw = GW, ns = NS;
+  int gw = GW;
   FusedArgs args = a;
-  void* params[] = {&args, &th2, &gw, &ns};
+  void* params[] = {&args, &th2, &gw};
   return cudaLaunchCooperativeKernel(fn, dim3(grid), dim3(32 * NW), params, smem, s);
 }
 
