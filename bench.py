@@ -321,13 +321,19 @@ NCU_TRAFFIC = {
     ("gemm", "llama-70b-ffn-prefill"): {
         "bytes": 371393280 + 217390848,
         "source": "profiles/gemm_i8_persistent_llama-70b-ffn-prefill.md"},
+    ("quantize", "llama-70b-ffn-prefill"): {
+        "bytes": 68038144 + 5652736,
+        "source": "profiles/stream_quantize_llama-70b-ffn-prefill.md"},
+    ("quantize", "opt-6.7b-ffn-up-prefill"): {
+        "bytes": 17046784 + 0,
+        "source": "profiles/stream_quantize_opt-6.7b-ffn-up-prefill.md"},
     ("gemm", "opt-6.7b-ffn-up-prefill"): {
         "bytes": 80.357632e6 + 37.069568e6,
         "source": "profiles/gemm_i8_persistent_opt-6.7b-ffn-up-prefill.md"},
     ("rotate", "opt-6.7b-ffn-up-prefill"): {
         "bytes": 16.804608e6, "source": "profiles/rotate_rows_opt-6.7b-ffn-up-prefill.md"},
     ("decode", "decode"): {
-        "bytes": 19.60192e6, "source": "profiles/decode_kernel_decode-16x4096x4096.md"},
+        "bytes": 17029376 + 0, "source": "profiles/decode_kernel_decode-16x4096x4096.md"},
 }
 
 
@@ -340,10 +346,10 @@ def quantize_stage_bytes(w, count):
     """Algorithmic bytes of detection + quantisation (+ compaction) per call."""
     b = 2 * w.M * w.K + w.M * w.K + 4 * w.M     # read X once; write Xq and x_scale
     if count > 0:
-        # X_O and W_O written zero-padded to 16 columns; the W_O gather reads one
-        # 32-byte sector per outlier per weight row, at most the whole row.
+        # X_O and W_O written zero-padded to 16 columns; W_O comes from the
+        # count contiguous rows of the transposed fp16 weight (2N bytes each).
         pad = (count + 15) // 16 * 16
-        b += 2 * w.M * pad + min(32 * count, 2 * w.K) * w.N + 2 * w.N * pad
+        b += 2 * w.M * pad + 2 * count * w.N + 2 * w.N * pad
     return b
 
 
