@@ -559,8 +559,8 @@ int fused_vpt(int K) {
 }
 
 cudaError_t launch_detect_quantize_compact(const FusedArgs& a, cudaStream_t s) {
-  // Absmax codes with detection: the single-pass kernel of stream_quant.cu.
-  if (a.x_zero == nullptr && a.given == nullptr) return launch_detect_quantize_stream(a, s);
+  // Absmax codes (with detection or a given set): the single-pass kernel of stream_quant.cu.
+  if (a.x_zero == nullptr) return launch_detect_quantize_stream(a, s);
   const int vpt = fused_vpt(a.K);
   const void* fn = nullptr;
   const bool zp = a.x_zero != nullptr;

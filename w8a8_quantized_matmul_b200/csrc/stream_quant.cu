@@ -182,7 +182,7 @@ __host__ __device__ inline StreamSmem stream_smem_layout(int K, size_t slot_byte
 
 }  // namespace
 
-template <int VPL, bool FULL>
+template <int VPL, bool FULL, bool GIVEN>
 __global__ void __launch_bounds__(32 * kMaxWarps, 1)
     stream_quantize_kernel(FusedArgs a, uint32_t th2bits, int GW) {
   extern __shared__ __align__(128) uint8_t ssm[];
@@ -217,7 +217,15 @@ __global__ void __launch_bounds__(32 * kMaxWarps, 1)
   // The GEMM that follows may launch now; it waits for this grid's completion
   // before reading anything written here.
   griddep_launch_dependents();
-  for (int w = tid; w < words; w += blockDim.x) s_lbits[w] = 0u;
+  // Given-set mode (token-sharded batches, top-k): the outlier set is the OR of
+  // the given bitmaps and final; the threshold plays no part.
+  constexpr bool given = GIVEN;
+  for (int w = tid; w < words; w += blockDim.x) {
+    uint32_t b = 0u;
+    if (given)
+      for (int r = 0; r < a.given_n; ++r) b |= __ldg(a.given + static_cast<size_t>(r) * words + w);
+    s_lbits[w] = b;
+  }
   for (int r = tid; r < kRowBlock; r += blockDim.x) s_mo[r] = 0u;
   if (tid == 0) {
     for (int s = 0; s < NW; ++s) mbar_init(&s_bar[s], 1);
@@ -247,6 +255,20 @@ __global__ void __launch_bounds__(32 * kMaxWarps, 1)
   // Loop-invariant operands of the code arithmetic.
   const uint64_t magic2 = f2pack(kMagic, kMagic);
   const uint16_t h127 = 0x57F0u;   // 127.0 in binary16
+  // Given-set mode: the set bits of the thread's vectors (the same columns on
+  // every row), four 8-bit masks per word.
+  uint32_t gmask[(VPL + 3) / 4];
+#pragma unroll
+  for (int j = 0; j < (VPL + 3) / 4; ++j) gmask[j] = 0u;
+  if (given) {
+#pragma unroll
+    for (int c = 0; c < VPL; ++c) {
+      const int v = v0 + c * 32 + lane;
+      const uint32_t m8 = (FULL || c * 32 + lane < npv) ? (s_lbits[v >> 2] >> (8 * (v & 3))) & 0xFFu : 0u;
+      gmask[c >> 2] |= m8 << (8 * (c & 3));
+    }
+  }
+  auto gm8 = [&](int c) { return (gmask[c >> 2] >> (8 * (c & 3))) & 0xFFu; };
   bool ok = true;
   uint2* dst = reinterpret_cast<uint2*>(a.Xq + static_cast<size_t>(r0 + g) * K) + v0 + lane;
   const size_t dst_step = row_step / 8;                    // uint2 per group row step
@@ -273,13 +295,24 @@ __global__ void __launch_bounds__(32 * kMaxWarps, 1)
     // vectors that exceed it and the maximum over its unflagged entries.
     uint32_t vm[VPL];
 #pragma unroll
-    for (int c = 0; c < VPL; ++c)
-      vm[c] = hmax2_bits(hmax2_bits(u[c].x & 0x7FFF7FFFu, u[c].y & 0x7FFF7FFFu),
-                         hmax2_bits(u[c].z & 0x7FFF7FFFu, u[c].w & 0x7FFF7FFFu));
+    for (int c = 0; c < VPL; ++c) {
+      uint32_t ax = u[c].x & 0x7FFF7FFFu, ay = u[c].y & 0x7FFF7FFFu;
+      uint32_t az = u[c].z & 0x7FFF7FFFu, aw = u[c].w & 0x7FFF7FFFu;
+      if (given) {
+        const uint32_t m8 = gm8(c);
+        if (m8 != 0u) {   // given outlier columns are left out of the maximum
+          ax &= keep_half2(m8, 0);
+          ay &= keep_half2(m8, 1);
+          az &= keep_half2(m8, 2);
+          aw &= keep_half2(m8, 3);
+        }
+      }
+      vm[c] = hmax2_bits(hmax2_bits(ax, ay), hmax2_bits(az, aw));
+    }
     uint32_t rm = vm[0];
 #pragma unroll
     for (int c = 1; c < VPL; ++c) rm = hmax2_bits(rm, vm[c]);
-    if (__hgt2_mask(*reinterpret_cast<const __half2*>(&rm), th2) != 0u) {
+    if (!given && __hgt2_mask(*reinterpret_cast<const __half2*>(&rm), th2) != 0u) {
       rm = 0u;
 #pragma unroll
       for (int c = 0; c < VPL; ++c) {
@@ -312,8 +345,19 @@ __global__ void __launch_bounds__(32 * kMaxWarps, 1)
     // Pass 2: the codes with m1 (entries the row flags itself get codes that
     // the fix-up overwrites with 0).
 #pragma unroll
-    for (int c = 0; c < VPL; ++c)
-      if (FULL || c * 32 + lane < npv) dst[c * 32] = codes8_h(u[c], ra2, na2, magic2, h127);
+    for (int c = 0; c < VPL; ++c) {
+      if (FULL || c * 32 + lane < npv) {
+        uint2 q = codes8_h(u[c], ra2, na2, magic2, h127);
+        if (given) {   // codes at the given outlier columns are 0
+          const uint32_t m8 = gm8(c);
+          if (m8 != 0u) {
+            q.x &= keep_bytes(m8 & 0xFu);
+            q.y &= keep_bytes(m8 >> 4);
+          }
+        }
+        dst[c * 32] = q;
+      }
+    }
     if (gw == 0 && lane == 0) {
       const int row = g + i * NG;
       a.x_scale[r0 + row] = m1;
@@ -455,6 +499,21 @@ __global__ void __launch_bounds__(32 * kMaxWarps, 1)
     }
   };
 
+  if (given) {
+    // The set is final: the list, the bitmap (CTA 0) and the panels; no check.
+    if (warp == 0) build_list(s_lbits);
+    if (blockIdx.x == 0)
+      for (int w = tid; w < words; w += blockDim.x) a.bitmap[w] = s_lbits[w];
+    __syncthreads();
+    fix_and_gather(s_misc[0], false, NW);
+    __syncthreads();
+    if (blockIdx.x == 0) {
+      const int count = s_misc[0];
+      for (int p = tid; p < count; p += blockDim.x) a.col_idx[p] = s_idx[p];
+      if (tid == 0) *a.n_outliers = count;
+    }
+    return;
+  }
   const int ctl = NW - 1;                  // control warp: batch bitmap and arrival
   const int nwork = NW > 1 ? NW - 1 : 1;   // warps of the fix-up
   if (warp == 0) build_list(s_lbits);
@@ -581,7 +640,7 @@ int coresident_ctas(const void* fn, int dev, int nw, size_t smem, cudaError_t* e
 
 }  // namespace
 
-// Absmax codes with detection (not the zero-point codes or a given outlier set).
+// Absmax codes, with detection or with a given outlier set (not the zero-point codes).
 cudaError_t launch_detect_quantize_stream(const FusedArgs& a, cudaStream_t s) {
   // 16 warps in groups of GW warps per row, GW the smallest power of two that
   // leaves each warp at most 256 vectors (8 per lane, held in registers) of a
@@ -595,19 +654,21 @@ cudaError_t launch_detect_quantize_stream(const FusedArgs& a, cudaStream_t s) {
   while (VPL * 32 < pv) VPL *= 2;
   // Every warp's piece full (no bounds checks in the stream) for the usual K.
   const bool full = nv == GW * VPL * 32;
+  const bool given = a.given != nullptr;
   const void* fn = nullptr;
+#define I8MM_STREAM_FN(V)                                                                      \
+  (full ? (given ? reinterpret_cast<const void*>(stream_quantize_kernel<V, true, true>)          \
+                 : reinterpret_cast<const void*>(stream_quantize_kernel<V, true, false>))       \
+        : (given ? reinterpret_cast<const void*>(stream_quantize_kernel<V, false, true>)        \
+                 : reinterpret_cast<const void*>(stream_quantize_kernel<V, false, false>)))
   switch (VPL) {
-    case 1: fn = full ? reinterpret_cast<const void*>(stream_quantize_kernel<1, true>)
-                      : reinterpret_cast<const void*>(stream_quantize_kernel<1, false>); break;
-    case 2: fn = full ? reinterpret_cast<const void*>(stream_quantize_kernel<2, true>)
-                      : reinterpret_cast<const void*>(stream_quantize_kernel<2, false>); break;
-    case 4: fn = full ? reinterpret_cast<const void*>(stream_quantize_kernel<4, true>)
-                      : reinterpret_cast<const void*>(stream_quantize_kernel<4, false>); break;
-    case 8: fn = full ? reinterpret_cast<const void*>(stream_quantize_kernel<8, true>)
-                      : reinterpret_cast<const void*>(stream_quantize_kernel<8, false>); break;
-    default: fn = full ? reinterpret_cast<const void*>(stream_quantize_kernel<16, true>)
-                       : reinterpret_cast<const void*>(stream_quantize_kernel<16, false>); break;
+    case 1: fn = I8MM_STREAM_FN(1); break;
+    case 2: fn = I8MM_STREAM_FN(2); break;
+    case 4: fn = I8MM_STREAM_FN(4); break;
+    case 8: fn = I8MM_STREAM_FN(8); break;
+    default: fn = I8MM_STREAM_FN(16); break;
   }
+#undef I8MM_STREAM_FN
   const int NW = kMaxWarps;
   const size_t smem = stream_smem_layout(a.K, static_cast<size_t>(NW) * pv * 16).total;
   int dev = 0;
