@@ -1,5 +1,7 @@
 // Fused detection + quantisation + compaction for the full LLM.int8() path,
-// one cooperative launch (all CTAs co-resident).
+// one cooperative launch (all CTAs co-resident), in its two-pass form. The
+// library uses it for the zero-point codes (scholia section 6); the absmax
+// codes run the single-pass kernel of stream_quant.cu.
 //
 // Method: AIInfra "05Infer/06CompDistill/05Quantization01", LLM.int8() section
 // (outlier feature dimensions by a magnitude threshold, vector-wise absmax INT8
@@ -87,7 +89,7 @@ __device__ __forceinline__ uint64_t gtimer() {
 
 // Shared-memory layout of one CTA (16-byte aligned pieces):
 //   rows    [S][K] fp16        row slots, filled by bulk copies
-//   lbits   [words] u32        the CTA's own outlier bitmap (or the given set)
+//   lbits   [words] u32        the CTA's own outlier bitmap
 //   gbits   [words] u32        the global bitmap, after the grid barrier
 //   red     [2][2][kWarps] f32 per-warp partial row maxima (and of -x, zero point),
 //                              alternating between consecutive rounds
@@ -142,7 +144,6 @@ __global__ void __launch_bounds__(kThreads, VPT <= 2 ? 2 : 1)
   const int rows_per = (a.M + gridDim.x - 1) / gridDim.x;
   const int r0 = min(a.M, static_cast<int>(blockIdx.x) * rows_per);
   const int R = min(a.M, r0 + rows_per) - r0;
-  const bool given = a.given != nullptr;   // outlier set supplied (token-sharded mode)
 
   // The GEMM that follows may launch now; it waits for this grid's completion
   // before reading anything written here.
@@ -158,7 +159,7 @@ __global__ void __launch_bounds__(kThreads, VPT <= 2 ? 2 : 1)
   // Rows stream through S slots (row r in slot r % S); after a chunk of rows
   // every thread is done with their slots and the rows S further on are loaded
   // into them. Each thread waits for each row itself (one mbarrier per slot).
-  if (!given) {
+  {
     uint32_t par = 0;   // bit s: parity of the next completion of slot s
     auto issue = [&](int row) {   // thread 0 only
       uint64_t* bar = &s_bar[row % S];
@@ -223,21 +224,12 @@ __global__ void __launch_bounds__(kThreads, VPT <= 2 ? 2 : 1)
       }
     }
     __syncthreads();
-  } else {
-    // The set is the OR of the ranks' bitmaps; it is final, nothing to check.
-    for (int w = tid; w < words; w += kThreads) {
-      uint32_t b = 0;
-      for (int r = 0; r < a.given_n; ++r) b |= __ldg(a.given + static_cast<size_t>(r) * words + w);
-      s_lbits[w] = b;
-      if (blockIdx.x == 0) a.bitmap[w] = b;
-    }
-    __syncthreads();
   }
 
   // ------------------------------------------------------------ pass B
   // After pass A the slots hold rows [R - nres, R) ("resident"); the others are
   // read again from global memory (L2) into registers.
-  const int nres = given ? 0 : min(R, S);
+  const int nres = min(R, S);
   int round = 0;   // selects the half of s_red a round of partial maxima uses
 
   // Row absmax over the non-outlier columns (zero-point codes: the largest x
@@ -499,7 +491,7 @@ __global__ void __launch_bounds__(kThreads, VPT <= 2 ? 2 : 1)
     // Control warp: arrive at the grid barrier, build this CTA's list (the
     // batch's list unless the check below finds a column it lacks), wait at the
     // barrier, then read the batch's bitmap and compare.
-    if (!given && lane == 0) {
+    if (lane == 0) {
       __threadfence();
       atomicAdd(a.sync_ctr, 1);
     }
@@ -508,7 +500,7 @@ __global__ void __launch_bounds__(kThreads, VPT <= 2 ? 2 : 1)
     __syncwarp();
     named_bar_arrive(kListBar, kThreads);
     int extra = 0;
-    if (!given) {
+    {
       if (lane == 0) {
         const uint64_t t0 = gtimer();
         while (ld_acquire(a.sync_ctr) < static_cast<int>(gridDim.x)) {
@@ -559,22 +551,18 @@ int fused_vpt(int K) {
 }
 
 cudaError_t launch_detect_quantize_compact(const FusedArgs& a, cudaStream_t s) {
-  // Absmax codes (with detection or a given set): the single-pass kernel of stream_quant.cu.
+  // Absmax codes (with detection or a given set): the single-pass kernel of
+  // stream_quant.cu. This kernel serves the zero-point codes with detection.
   if (a.x_zero == nullptr) return launch_detect_quantize_stream(a, s);
+  if (a.given != nullptr) return cudaErrorInvalidValue;
   const int vpt = fused_vpt(a.K);
   const void* fn = nullptr;
-  const bool zp = a.x_zero != nullptr;
   switch (vpt) {
-    case 1: fn = zp ? reinterpret_cast<const void*>(detect_quantize_compact_kernel<1, true>)
-                    : reinterpret_cast<const void*>(detect_quantize_compact_kernel<1, false>); break;
-    case 2: fn = zp ? reinterpret_cast<const void*>(detect_quantize_compact_kernel<2, true>)
-                    : reinterpret_cast<const void*>(detect_quantize_compact_kernel<2, false>); break;
-    case 4: fn = zp ? reinterpret_cast<const void*>(detect_quantize_compact_kernel<4, true>)
-                    : reinterpret_cast<const void*>(detect_quantize_compact_kernel<4, false>); break;
-    case 8: fn = zp ? reinterpret_cast<const void*>(detect_quantize_compact_kernel<8, true>)
-                    : reinterpret_cast<const void*>(detect_quantize_compact_kernel<8, false>); break;
-    default: fn = zp ? reinterpret_cast<const void*>(detect_quantize_compact_kernel<16, true>)
-                     : reinterpret_cast<const void*>(detect_quantize_compact_kernel<16, false>); break;
+    case 1: fn = reinterpret_cast<const void*>(detect_quantize_compact_kernel<1, true>); break;
+    case 2: fn = reinterpret_cast<const void*>(detect_quantize_compact_kernel<2, true>); break;
+    case 4: fn = reinterpret_cast<const void*>(detect_quantize_compact_kernel<4, true>); break;
+    case 8: fn = reinterpret_cast<const void*>(detect_quantize_compact_kernel<8, true>); break;
+    default: fn = reinterpret_cast<const void*>(detect_quantize_compact_kernel<16, true>); break;
   }
   // Row slots: about 110 KB when two CTAs share an SM (vpt <= 2), 220 KB otherwise.
   const size_t row_bytes = static_cast<size_t>(a.K) * 2;
