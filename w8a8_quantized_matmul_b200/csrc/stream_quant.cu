@@ -48,11 +48,16 @@
 //   check    wait at the grid barrier (bounded) and compare the batch bitmap
 //            with L; if the batch has a column the CTA's rows lack, every row of
 //            the CTA, X_O and W_O again with the batch's set.
+// With a given outlier set (the OR of the bitmaps of a token-sharded batch's
+// ranks, or a top-k selection) nothing is speculative: the given columns are
+// masked out of the row maximum and the codes from the start, and the list, the
+// panels and the bitmap follow with no check and no grid barrier.
 // The panels are zero-padded to a multiple of 16 columns (one kind::f16 K step
 // of the GEMM, which multiplies only the K steps that hold columns).
 //
-// Codes: rint(fl32(fl32(x*127)/a)) clamped to +-127 from the FMA-corrected
-// quotient (codes8 in quant_common.cuh). The threshold test |x| > t is taken on
+// Codes: rint(fl32(fl32(x*127)/a)) for |x| <= a (so within +-127 without a
+// clamp) from the FMA-corrected quotient of quant_common.cuh, with x*127 formed
+// by a mixed-precision FMA (codes8_h). The threshold test |x| > t is taken on
 // fp16 values against the largest fp16 value not above t, which selects the
 // same entries as the fp32 comparison.
 #include <cuda_fp16.h>
