@@ -123,8 +123,8 @@ size_t int8_mixed_matmul_workspace_size(int M, int N, int K);
  * The outlier panels have row stride panel_ld elements (fp16) and hold the
  * compacted outlier columns in ascending column order, zero-padded to a
  * multiple of 16 columns (one K step of the tensor-core outlier product; the
- * zero-point and given-set paths pad to 64). Columns past the padding are
- * never read. Nothing is written to them when there are no outliers.
+ * zero-point path pads to 64). Columns past the padding are never read.
+ * Nothing is written to them when there are no outliers.
  */
 typedef struct {
   size_t n_outliers;   /* int32 [1] */
